@@ -1,0 +1,178 @@
+"""fp64 reference implementation of PISA (test infrastructure only).
+
+Notation (PISA explainer, "PISA: Piecewise Sparse Attention Is Wiser for
+Efficient Diffusion Transformers", technical summary section 2):
+
+* tensors are [B, H, N, d]; block ``j`` holds tokens [j*b, min((j+1)*b, N))
+  and has ``n_j`` real tokens (the last block may be ragged);
+* for query block ``i`` the key/value blocks split into the critical set
+  ``S_i`` (computed exactly) and the non-critical set ``U_i`` (approximated);
+* ``x_t = scale * q_t`` is the scaled query of row ``t``;
+* ``kbar_j`` is block j's mean key (the block centroid), ``S0_j`` its value
+  sum, ``S1_j = sum_{n in j} (k_n - kbar_j) v_n^T`` (d x d, rows indexed by
+  the key dimension, columns by the value dimension);
+* ``alpha_{t,j} = exp(x_t . kbar_j)``.
+
+The output is ``o_t = N_t / D_t`` with
+
+    N_t = sum_{j in S_i} sum_n e^{x_t.k_{j,n}} v_{j,n}
+        + sum_{j in U_i} alpha_{t,j} (S0_j + [order >= 1] S1_j^T x_t)
+    D_t = sum_{j in S_i} sum_n e^{x_t.k_{j,n}} + sum_{j in U_i} n_j alpha_{t,j}
+
+(section 2, "Core algorithm": the exact sparse term, the block zeroth-order
+term with alpha defined from the block centroid, and a first-order term in the
+third slot of the numerator; "Key insights": the approximations sit inside the
+softmax numerator and denominator). The denominator's first-order part is
+``x_t . sum_n (k_n - kbar_j) = 0`` identically and is therefore absent.
+All exponents are shifted by the row maximum ``m_t`` before exponentiation;
+the shift cancels in N_t / D_t.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+NEAR_TIE_REL = 1e-5
+
+
+def block_bounds(N: int, block: int):
+    """[(start, end)] of every block; the last one may hold fewer than ``block`` tokens."""
+    nB = -(-N // block)
+    return [(j * block, min((j + 1) * block, N)) for j in range(nB)]
+
+
+def block_stats(K, V, block: int, order: int = 1):
+    """Block centroid, value sum and first-order matrix of every key/value block.
+
+    Section 2, "Hardware implementation", precompute step (block centroids and
+    value sums); the per-block first-order matrix is the Taylor term defined in
+    the module docstring.
+
+    Returns ``kbar`` [B,H,nB,d], ``S0`` [B,H,nB,d] and ``S1`` [B,H,nB,d,d]
+    (``None`` when ``order == 0``), all float64.
+    """
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    B, H, N, d = K.shape
+    bounds = block_bounds(N, block)
+    nB = len(bounds)
+    kbar = np.empty((B, H, nB, d))
+    S0 = np.empty((B, H, nB, d))
+    S1 = np.empty((B, H, nB, d, d)) if order >= 1 else None
+    for j, (s, e) in enumerate(bounds):
+        Kj = K[:, :, s:e, :]
+        Vj = V[:, :, s:e, :]
+        kbar[:, :, j] = Kj.sum(axis=2) / (e - s)
+        S0[:, :, j] = Vj.sum(axis=2)
+        if S1 is not None:
+            centred = Kj - kbar[:, :, j][:, :, None, :]
+            # S1[a, c] = sum_n centred[n, a] * v[n, c]
+            S1[:, :, j] = np.matmul(np.swapaxes(centred, -1, -2), Vj)
+    return kbar, S0, S1
+
+
+def pooled_queries(Q, block: int):
+    """Mean query of every query block (same partition as the key blocks)."""
+    Q = np.asarray(Q, dtype=np.float64)
+    B, H, N, d = Q.shape
+    bounds = block_bounds(N, block)
+    qbar = np.empty((B, H, len(bounds), d))
+    for i, (s, e) in enumerate(bounds):
+        qbar[:, :, i] = Q[:, :, s:e, :].sum(axis=2) / (e - s)
+    return qbar
+
+
+def select(Q, kbar, block: int, topk: int):
+    """Top-k critical blocks of every query block.
+
+    The page states only that the critical blocks are the ones with the highest
+    attention relevance (section 2, "Covariance-aware routing", first sentence
+    without the covariance term). Relevance here is the pooled score
+    ``qbar_i . kbar_j`` with ``qbar_i`` the mean query of block i. A positive
+    softmax scale cannot change the order, so the scores are unscaled.
+
+    Returns ``idx`` int32 [B,H,nB,topk] (each row ascending; ties between equal
+    scores go to the lower block index), ``near_tie`` bool [B,H,nB] (the k-th
+    and (k+1)-th scores agree to 1e-5 relative) and ``scores`` [B,H,nB,nB].
+    """
+    qbar = pooled_queries(Q, block)
+    kbar = np.asarray(kbar, dtype=np.float64)
+    B, H, nB, _ = qbar.shape
+    if not (0 <= topk <= nB):
+        raise ValueError("topk out of range")
+    scores = np.matmul(qbar, np.swapaxes(kbar, -1, -2))
+    idx = np.empty((B, H, nB, topk), dtype=np.int32)
+    near = np.zeros((B, H, nB), dtype=bool)
+    cols = np.arange(nB)
+    for b in range(B):
+        for h in range(H):
+            for i in range(nB):
+                row = scores[b, h, i]
+                # primary key: score descending; secondary key: block index ascending
+                order = np.lexsort((cols, -row))
+                idx[b, h, i] = np.sort(order[:topk])
+                if 0 < topk < nB:
+                    a, c = row[order[topk - 1]], row[order[topk]]
+                    near[b, h, i] = abs(a - c) <= NEAR_TIE_REL * max(abs(a), abs(c))
+    return idx, near, scores
+
+
+def _query_blocks(nB, query_blocks):
+    return range(nB) if query_blocks is None else query_blocks
+
+
+def attention(Q, K, V, kbar, S0, S1, idx, block: int, order: int, scale: float,
+              query_blocks=None, heads=None):
+    """PISA output rows (float64 [B,H,N,d]; rows of skipped query blocks are NaN).
+
+    ``idx`` [B,H,nB,k] lists the critical blocks of each query block (any
+    order; ``k`` may be 0). ``query_blocks`` / ``heads`` restrict the work to a
+    sample; ``heads`` is a list of (b, h) pairs.
+    """
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    B, H, N, d = Q.shape
+    bounds = block_bounds(N, block)
+    nB = len(bounds)
+    counts = np.array([e - s for s, e in bounds], dtype=np.float64)
+    O = np.full((B, H, N, d), np.nan)
+    pairs = [(b, h) for b in range(B) for h in range(H)] if heads is None else heads
+    for b, h in pairs:
+        for i in _query_blocks(nB, query_blocks):
+            s_i, e_i = bounds[i]
+            X = scale * Q[b, h, s_i:e_i]                       # scaled queries of block i
+            crit = sorted(set(int(j) for j in np.asarray(idx[b, h, i]).ravel()))
+            crit_set = set(crit)
+            rest = [j for j in range(nB) if j not in crit_set]
+            # exact sparse term over every key of every critical block
+            keys = [t for j in crit for t in range(*bounds[j])]
+            z_ex = X @ K[b, h, keys].T                        # [n_i, |keys|]
+            # zeroth-order exponents over the non-critical blocks
+            z_ap = X @ kbar[b, h, rest].T                     # [n_i, |U|]
+            m = np.full(e_i - s_i, -np.inf)
+            if z_ex.size:
+                m = np.maximum(m, z_ex.max(axis=1))
+            if z_ap.size:
+                m = np.maximum(m, z_ap.max(axis=1))
+            w = np.exp(z_ex - m[:, None])
+            alpha = np.exp(z_ap - m[:, None])
+            num = w @ V[b, h, keys] + alpha @ S0[b, h, rest]
+            den = w.sum(axis=1) + alpha @ counts[rest]
+            if order >= 1 and rest:
+                # S1_j^T x_t for every (t, j): first[t, j, c] = sum_a x[t, a] S1_j[a, c]
+                first = np.einsum("ta,jac->tjc", X, S1[b, h, rest])
+                num = num + np.einsum("tj,tjc->tc", alpha, first)
+            O[b, h, s_i:e_i] = num / den[:, None]
+    return O
+
+
+def dense_attention(Q, K, V, scale: float):
+    """Textbook softmax(scale Q K^T) V in float64."""
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    z = scale * np.matmul(Q, np.swapaxes(K, -1, -2))
+    z = z - z.max(axis=-1, keepdims=True)
+    p = np.exp(z)
+    return np.matmul(p, V) / p.sum(axis=-1, keepdims=True)
+

@@ -1,0 +1,325 @@
+"""Pins of the CPU oracle against facts the method and the mathematics fix.
+
+Each ``pin_*`` takes an oracle-like module (the real ``oracle`` package, or a
+copy with a planted mistake) and returns a non-negative error; the test suite
+asserts that the real oracle's errors are at round-off level and that every
+planted mistake pushes at least one pin far above it.
+
+None of these pins restates the oracle's vectorised formulas: they use scalar
+brute force, exhaustive subset search, textbook softmax attention (scipy), a
+second formulation of the first-order term, closed forms and convergence
+rates.
+"""
+from __future__ import annotations
+
+import itertools
+import math
+
+import numpy as np
+from scipy.special import softmax
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+# ----------------------------------------------------------------------------
+# block statistics
+# ----------------------------------------------------------------------------
+def pin_stats_bruteforce(orc, seed=0):
+    """Scalar loops over the definition of centroid, value sum and S1 (ragged N)."""
+    r = _rng(seed)
+    B, H, N, d, b = 1, 2, 11, 3, 4
+    K = r.standard_normal((B, H, N, d))
+    V = r.standard_normal((B, H, N, d))
+    kbar, S0, S1 = orc.block_stats(K, V, b, order=1)
+    err = 0.0
+    for h in range(H):
+        j = 0
+        for start in range(0, N, b):
+            toks = list(range(start, min(start + b, N)))
+            cen = [sum(K[0, h, t, a] for t in toks) / len(toks) for a in range(d)]
+            vs = [sum(V[0, h, t, c] for t in toks) for c in range(d)]
+            for a in range(d):
+                err = max(err, abs(kbar[0, h, j, a] - cen[a]))
+                err = max(err, abs(S0[0, h, j, a] - vs[a]))
+                for c in range(d):
+                    ref = sum((K[0, h, t, a] - cen[a]) * V[0, h, t, c] for t in toks)
+                    err = max(err, abs(S1[0, h, j, a, c] - ref))
+            j += 1
+    return err
+
+
+def pin_stats_covariance(orc, seed=1):
+    """With V = K, S1_j is n_j times the (biased) covariance of the block's keys."""
+    r = _rng(seed)
+    K = r.standard_normal((1, 1, 40, 5))
+    _, _, S1 = orc.block_stats(K, K, 8, order=1)
+    err = 0.0
+    for j in range(5):
+        ref = 8 * np.cov(K[0, 0, 8 * j:8 * j + 8].T, bias=True)
+        err = max(err, np.abs(S1[0, 0, j] - ref).max())
+    return err
+
+
+def pin_stats_constant_values(orc, seed=2):
+    """Constant value rows: S1 = 0 (centred keys sum to zero), S0 = n v."""
+    r = _rng(seed)
+    K = r.standard_normal((1, 1, 20, 4)) * 3 + 1
+    V = np.broadcast_to(r.standard_normal(4), (1, 1, 20, 4)).copy()
+    _, S0, S1 = orc.block_stats(K, V, 6, order=1)
+    err = np.abs(S1).max()
+    counts = [6, 6, 6, 2]
+    for j, n in enumerate(counts):
+        err = max(err, np.abs(S0[0, 0, j] - n * V[0, 0, 0]).max())
+    return err
+
+
+# ----------------------------------------------------------------------------
+# selection
+# ----------------------------------------------------------------------------
+def _brute_select(qbar_row, kbar, k):
+    """Subset of size k with the largest total score; ties -> lexicographically smallest."""
+    nB = kbar.shape[0]
+    sc = [sum(qbar_row[a] * kbar[j, a] for a in range(kbar.shape[1])) for j in range(nB)]
+    best, best_set = -math.inf, None
+    for sub in itertools.combinations(range(nB), k):      # lexicographic order
+        tot = sum(sc[j] for j in sub)
+        if tot > best + 1e-12:
+            best, best_set = tot, sub
+    return list(best_set)
+
+
+def pin_select_bruteforce(orc, seed=3, trials=30):
+    """Exhaustive subset search on 4-8 blocks, ragged N included. Returns #mismatches."""
+    r = _rng(seed)
+    bad = 0
+    for t in range(trials):
+        b = int(r.integers(1, 5))
+        nB = int(r.integers(4, 9))
+        N = b * nB - int(r.integers(0, b))
+        nB = -(-N // b)
+        d = int(r.integers(1, 5))
+        k = int(r.integers(1, nB + 1))
+        Q = r.standard_normal((1, 1, N, d))
+        kbar = r.standard_normal((1, 1, nB, d))
+        if t % 3 == 0:            # plant exact ties: duplicate some centroids
+            kbar[0, 0, nB - 1] = kbar[0, 0, 0]
+            kbar[0, 0, nB // 2] = kbar[0, 0, 1]
+        idx, _, _ = orc.select(Q, kbar, b, k)
+        for i in range(nB):
+            rows = [s for s in range(i * b, min(i * b + b, N))]
+            qbar = [sum(Q[0, 0, s, a] for s in rows) / len(rows) for a in range(d)]
+            ref = _brute_select(qbar, kbar[0, 0], k)
+            if list(idx[0, 0, i]) != ref:
+                bad += 1
+    return bad
+
+
+def pin_select_ties(orc):
+    """All centroids equal: every row must take blocks 0..k-1 (lower index wins)."""
+    Q = _rng(4).standard_normal((1, 1, 32, 3))
+    kbar = np.ones((1, 1, 8, 3))
+    idx, _, _ = orc.select(Q, kbar, 4, 3)
+    return int(np.any(idx != np.arange(3)))
+
+
+# ----------------------------------------------------------------------------
+# attention
+# ----------------------------------------------------------------------------
+def _textbook(Q, K, V, scale):
+    """softmax(scale Q K^T) V with scipy's softmax (independent of the oracle's)."""
+    z = scale * np.einsum("bhqd,bhkd->bhqk", Q, K)
+    return np.einsum("bhqk,bhkd->bhqd", softmax(z, axis=-1), V)
+
+
+def _full_idx(B, H, nB, k=None):
+    k = nB if k is None else k
+    return np.broadcast_to(np.arange(k, dtype=np.int32), (B, H, nB, k)).copy()
+
+
+def pin_all_selected_is_dense(orc, seed=5):
+    r = _rng(seed)
+    B, H, N, d, b = 1, 2, 45, 8, 8           # ragged last block
+    Q, K, V = (r.standard_normal((B, H, N, d)) for _ in range(3))
+    kbar, S0, S1 = orc.block_stats(K, V, b)
+    nB = -(-N // b)
+    out = orc.attention(Q, K, V, kbar, S0, S1, _full_idx(B, H, nB), b, 1, 0.4)
+    return np.abs(out - _textbook(Q, K, V, 0.4)).max()
+
+
+def pin_block_one_is_exact(orc, seed=6):
+    """Block size 1: kbar = k and S1 = 0, so any selection gives dense attention."""
+    r = _rng(seed)
+    B, H, N, d = 1, 1, 24, 4
+    Q, K, V = (r.standard_normal((B, H, N, d)) for _ in range(3))
+    kbar, S0, S1 = orc.block_stats(K, V, 1)
+    idx = np.stack([r.choice(N, 5, replace=False) for _ in range(N)])[None, None].astype(np.int32)
+    err = 0.0
+    for order in (0, 1):
+        out = orc.attention(Q, K, V, kbar, S0, S1, idx, 1, order, 0.7)
+        err = max(err, np.abs(out - _textbook(Q, K, V, 0.7)).max())
+    return err
+
+
+def pin_identical_keys_exact(orc, seed=7):
+    """A block of identical keys is exact at order 0 (and order 1, where S1 = 0)."""
+    r = _rng(seed)
+    B, H, N, d, b = 1, 1, 48, 6, 8
+    c = r.standard_normal((N // b, d))
+    K = np.repeat(c, b, axis=0)[None, None]
+    Q, V = (r.standard_normal((B, H, N, d)) for _ in range(2))
+    kbar, S0, S1 = orc.block_stats(K, V, b)
+    idx = np.full((1, 1, N // b, 1), 2, dtype=np.int32)
+    err = 0.0
+    for order in (0, 1):
+        out = orc.attention(Q, K, V, kbar, S0, S1, idx, b, order, 0.5)
+        err = max(err, np.abs(out - _textbook(Q, K, V, 0.5)).max())
+    return err
+
+
+def convergence_slopes(orc, seed=8):
+    """log-log slopes of the error vs dense as the in-block key spread eps shrinks."""
+    r = _rng(seed)
+    B, H, N, d, b = 1, 1, 64, 8, 8
+    nB = N // b
+    c = r.standard_normal((nB, d))
+    z = r.standard_normal((N, d))
+    Q = r.standard_normal((B, H, N, d))
+    V = r.standard_normal((B, H, N, d))
+    idx = np.zeros((1, 1, nB, 1), dtype=np.int32)
+    epss = [0.4, 0.2, 0.1, 0.05]
+    errs = {0: [], 1: []}
+    for eps in epss:
+        K = (np.repeat(c, b, axis=0) + eps * z)[None, None]
+        kbar, S0, S1 = orc.block_stats(K, V, b)
+        ref = _textbook(Q, K, V, 0.5)
+        for order in (0, 1):
+            out = orc.attention(Q, K, V, kbar, S0, S1, idx, b, order, 0.5)
+            errs[order].append(np.abs(out - ref).max())
+    le = np.log(epss)
+    return {o: float(np.polyfit(le, np.log(errs[o]), 1)[0]) for o in (0, 1)}
+
+
+def pin_order0_pseudo_tokens(orc, seed=9):
+    """No critical block, order 0: softmax over pseudo-tokens (kbar_j, S0_j/n_j) with a
+    log-count bias ln n_j (textbook softmax attention over pooled tokens)."""
+    r = _rng(seed)
+    B, H, N, d, b = 1, 1, 30, 5, 7          # counts 7,7,7,7,2
+    Q, K, V = (r.standard_normal((B, H, N, d)) for _ in range(3))
+    kbar, S0, S1 = orc.block_stats(K, V, b)
+    nB = -(-N // b)
+    idx = np.zeros((1, 1, nB, 0), dtype=np.int32)
+    out = orc.attention(Q, K, V, kbar, S0, S1, idx, b, 0, 0.9)
+    counts = np.array([min(N, (j + 1) * b) - j * b for j in range(nB)], dtype=float)
+    z = 0.9 * Q[0, 0] @ kbar[0, 0].T + np.log(counts)[None, :]
+    ref = softmax(z, axis=-1) @ (S0[0, 0] / counts[:, None])
+    return np.abs(out[0, 0] - ref).max()
+
+
+def pin_first_order_key_form(orc, seed=10):
+    """Order-1 output from a second formulation: S1_j^T x = sum_n (x.(k_n - kbar_j)) v_n,
+    i.e. each non-critical key gets weight e^{x.kbar}(1 + x.(k - kbar))."""
+    r = _rng(seed)
+    B, H, N, d, b = 1, 2, 40, 6, 8
+    Q, K, V = (r.standard_normal((B, H, N, d)) for _ in range(3))
+    kbar, S0, S1 = orc.block_stats(K, V, b)
+    nB = N // b
+    idx = np.stack([np.sort(r.choice(nB, 2, replace=False)) for _ in range(B * H * nB)])
+    idx = idx.reshape(B, H, nB, 2).astype(np.int32)
+    scale = 0.6
+    out = orc.attention(Q, K, V, kbar, S0, S1, idx, b, 1, scale)
+    err = 0.0
+    for h in range(H):
+        for i in range(nB):
+            crit = set(idx[0, h, i].tolist())
+            for t in range(i * b, i * b + b):
+                x = scale * Q[0, h, t]
+                wts, vals = [], []
+                for j in range(nB):
+                    kb = K[0, h, j * b:j * b + b].mean(axis=0)
+                    for n in range(j * b, j * b + b):
+                        if j in crit:
+                            wts.append(math.exp(x @ K[0, h, n]))
+                        else:
+                            wts.append(math.exp(x @ kb) * (1.0 + x @ (K[0, h, n] - kb)))
+                        vals.append(V[0, h, n])
+                # the denominator of a non-critical block is n_j e^{x.kbar}: the
+                # first-order weights sum to that exactly
+                ref = np.array(wts) @ np.array(vals) / sum(wts)
+                err = max(err, np.abs(out[0, h, t] - ref).max())
+    return err
+
+
+def pin_linear_in_values(orc, seed=11):
+    r = _rng(seed)
+    B, H, N, d, b = 1, 1, 32, 4, 8
+    Q, K, V1, V2 = (r.standard_normal((B, H, N, d)) for _ in range(4))
+    idx = np.array([[[[1], [0], [3], [2]]]], dtype=np.int32)
+
+    def run(V):
+        kb, s0, s1 = orc.block_stats(K, V, b)
+        return orc.attention(Q, K, V, kb, s0, s1, idx, b, 1, 0.5)
+    return np.abs(run(2.0 * V1 - 3.0 * V2) - (2.0 * run(V1) - 3.0 * run(V2))).max()
+
+
+def pin_permutation_in_block(orc, seed=12):
+    """Permuting (k, v) pairs inside a non-critical block leaves the output unchanged."""
+    r = _rng(seed)
+    B, H, N, d, b = 1, 1, 32, 4, 8
+    Q, K, V = (r.standard_normal((B, H, N, d)) for _ in range(3))
+    idx = np.zeros((1, 1, 4, 1), dtype=np.int32)
+    perm = np.arange(N)
+    perm[16:24] = 16 + r.permutation(8)
+    outs = []
+    for P in (np.arange(N), perm):
+        Kp, Vp = K[:, :, P], V[:, :, P]
+        kb, s0, s1 = orc.block_stats(Kp, Vp, b)
+        outs.append(orc.attention(Q, Kp, Vp, kb, s0, s1, idx, b, 1, 0.5))
+    return np.abs(outs[0] - outs[1]).max()
+
+
+def pin_order0_convex(orc, seed=13):
+    """Order 0 is a convex combination of exact values and block mean values:
+    returns the largest violation of min <= o <= max (per coordinate)."""
+    r = _rng(seed)
+    B, H, N, d, b = 1, 1, 40, 4, 8
+    Q, K, V = (r.standard_normal((B, H, N, d)) * 2 for _ in range(3))
+    kb, s0, s1 = orc.block_stats(K, V, b)
+    idx = np.array([[[[0], [1], [2], [3], [4]]]], dtype=np.int32)
+    out = orc.attention(Q, K, V, kb, s0, s1, idx, b, 0, 1.0)
+    pool = np.concatenate([V[0, 0], s0[0, 0] / b], axis=0)
+    lo, hi = pool.min(axis=0), pool.max(axis=0)
+    return float(max(0.0, (lo - out[0, 0]).max(), (out[0, 0] - hi).max()))
+
+
+def pin_worked_example(orc, case):
+    """Scalar (d = 1) worked example expanded by hand (tests/golden/worked_example.json)."""
+    q, k, v = (np.array(case[n], dtype=float) for n in ("q", "k", "v"))
+    b, scale = case["block"], case["scale"]
+    crit = case["critical"]                  # one list per query block
+    N = len(q)
+    Q, K, V = (a.reshape(1, 1, N, 1) for a in (q, k, v))
+    kb, s0, s1 = orc.block_stats(K, V, b)
+    idx = np.array(crit, dtype=np.int32).reshape(1, 1, len(crit), -1)
+    err = 0.0
+    for order in (0, 1):
+        out = orc.attention(Q, K, V, kb, s0, s1, idx, b, order, scale)
+        for t in range(N):
+            x = scale * q[t]
+            num = den = 0.0
+            for j in range(-(-N // b)):
+                toks = range(j * b, min(j * b + b, N))
+                if j in crit[t // b]:
+                    for n in toks:
+                        num += math.exp(x * k[n]) * v[n]
+                        den += math.exp(x * k[n])
+                else:
+                    kbar = sum(k[n] for n in toks) / len(toks)
+                    vsum = sum(v[n] for n in toks)
+                    first = sum((k[n] - kbar) * v[n] for n in toks)
+                    a = math.exp(x * kbar)
+                    num += a * (vsum + (order * first * x))
+                    den += a * len(toks)
+            err = max(err, abs(out[0, 0, t, 0] - num / den))
+    return err

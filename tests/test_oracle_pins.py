@@ -1,0 +1,103 @@
+"""The CPU oracle against what the method and the mathematics fix (no GPU).
+
+Also plants plausible mistakes in copies of the oracle (source mutations, on
+the CPU) and checks that at least one pin catches each of them.
+"""
+import json
+import os
+import types
+
+import numpy as np
+import pytest
+
+import oracle
+from tests import oracle_pins as P
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ORACLE_SRC = os.path.join(os.path.dirname(HERE), "oracle", "pisa.py")
+EXAMPLE = json.load(open(os.path.join(HERE, "golden", "worked_example.json")))
+
+TOL = 1e-10
+
+
+def _pins(orc):
+    """name -> (value, passes?) for every pin."""
+    out = {}
+    for name, fn, ok in [
+        ("stats_bruteforce", P.pin_stats_bruteforce, lambda e: e < TOL),
+        ("stats_covariance", P.pin_stats_covariance, lambda e: e < TOL),
+        ("stats_constant_values", P.pin_stats_constant_values, lambda e: e < TOL),
+        ("select_bruteforce", P.pin_select_bruteforce, lambda e: e == 0),
+        ("select_ties", P.pin_select_ties, lambda e: e == 0),
+        ("all_selected_is_dense", P.pin_all_selected_is_dense, lambda e: e < TOL),
+        ("block_one_is_exact", P.pin_block_one_is_exact, lambda e: e < TOL),
+        ("identical_keys_exact", P.pin_identical_keys_exact, lambda e: e < TOL),
+        ("order0_pseudo_tokens", P.pin_order0_pseudo_tokens, lambda e: e < TOL),
+        ("first_order_key_form", P.pin_first_order_key_form, lambda e: e < TOL),
+        ("linear_in_values", P.pin_linear_in_values, lambda e: e < TOL),
+        ("permutation_in_block", P.pin_permutation_in_block, lambda e: e < TOL),
+        ("order0_convex", P.pin_order0_convex, lambda e: e <= 1e-12),
+        ("worked_example", lambda o: P.pin_worked_example(o, EXAMPLE), lambda e: e < TOL),
+    ]:
+        try:
+            v = fn(orc)
+            out[name] = (v, bool(ok(v)))
+        except Exception as exc:  # a mutant may crash a pin: that counts as caught
+            out[name] = (repr(exc), False)
+    slopes = P.convergence_slopes(orc)
+    out["convergence_order0"] = (slopes[0], 0.8 < slopes[0] < 1.3)
+    out["convergence_order1"] = (slopes[1], 1.7 < slopes[1] < 2.4)
+    return out
+
+
+@pytest.fixture(scope="module")
+def real_pins():
+    return _pins(oracle)
+
+
+@pytest.mark.parametrize("name", [
+    "stats_bruteforce", "stats_covariance", "stats_constant_values", "select_bruteforce",
+    "select_ties", "all_selected_is_dense", "block_one_is_exact", "identical_keys_exact",
+    "order0_pseudo_tokens", "first_order_key_form", "linear_in_values",
+    "permutation_in_block", "order0_convex", "worked_example",
+    "convergence_order0", "convergence_order1"])
+def test_pin(real_pins, name):
+    value, ok = real_pins[name]
+    assert ok, f"{name}: {value}"
+
+
+def test_near_tie_flag():
+    """Two centroids whose scores differ by 1e-7 relative straddle the k-th place."""
+    Q = np.ones((1, 1, 16, 2))
+    kbar = np.array([[[[3.0, 0.0], [1.0, 0.0], [1.0 + 1e-7, 0.0], [0.0, 0.0]]]])
+    idx, near, _ = oracle.select(Q, kbar, 4, 2)
+    assert list(idx[0, 0, 0]) == [0, 2] and near[0, 0, 0]
+    idx, near, _ = oracle.select(Q, kbar, 4, 1)
+    assert list(idx[0, 0, 0]) == [0] and not near[0, 0, 0]
+
+
+MUTATIONS = {
+    "S1 transposed in stats": ("np.swapaxes(centred, -1, -2), Vj", "np.swapaxes(Vj, -1, -2), centred"),
+    "count dropped from denominator": ("alpha @ counts[rest]", "alpha.sum(axis=1)"),
+    "ties to the higher index": ("np.lexsort((cols, -row))", "np.lexsort((-cols, -row))"),
+    "lowest scores selected": ("np.lexsort((cols, -row))", "np.lexsort((cols, row))"),
+    "scale missing from alpha": ("z_ap = X @ kbar", "z_ap = Q[b, h, s_i:e_i] @ kbar"),
+    "first-order sign flipped": ("num = num + np.einsum", "num = num - np.einsum"),
+    "ragged centroid over b": ("Kj.sum(axis=2) / (e - s)", "Kj.sum(axis=2) / block"),
+    "S1 transposed in attention": ('"ta,jac->tjc"', '"ta,jca->tjc"'),
+    "value mean instead of sum": ("S0[:, :, j] = Vj.sum(axis=2)", "S0[:, :, j] = Vj.mean(axis=2)"),
+    "pooled query over wrong rows": ("Q[:, :, s:e, :].sum(axis=2) / (e - s)",
+                                     "Q[:, :, s:s + 1, :].sum(axis=2)"),
+    "exact keys from the wrong block": ("for t in range(*bounds[j])]", "for t in range(*bounds[(j + 1) % nB])]"),
+}
+
+
+@pytest.mark.parametrize("label", list(MUTATIONS))
+def test_planted_mistake_is_caught(label):
+    old, new = MUTATIONS[label]
+    src = open(ORACLE_SRC).read()
+    assert src.count(old) >= 1, f"mutation anchor not found: {old}"
+    mod = types.ModuleType("oracle_mutant")
+    exec(compile(src.replace(old, new), "oracle_mutant", "exec"), mod.__dict__)
+    failed = [n for n, (_, ok) in _pins(mod).items() if not ok]
+    assert failed, f"no pin caught: {label}"
