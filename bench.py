@@ -1,0 +1,370 @@
+"""Benchmark of the PISA hot path on B200: stats -> select -> attention.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload video] [--kernel fused|simt]
+
+One step = one pass of the whole path (block statistics, block selection,
+fused attention) over one batch of the named workload, inputs already resident
+in HBM. Default workload "video": B=1, H=24, N=32768 (8x64x64 latent grid),
+d=128, block 64, top-k 64 of 512 blocks (12.5% exact), order 1, seeded
+synthetic smooth tokens. Inputs (Q, K, V: 604 MB) are larger than L2, so no
+flush is needed between steps.
+
+N > 1 (torchrun, one process per GPU): every rank runs its own batch (weak
+scaling); the heads and batches are independent, so there is no collective in
+the data path. Timing: barrier + synchronize on both sides of the K timed
+steps, CUDA events on the launching stream, max over ranks.
+
+--impl reference times the CPU oracle (NumPy fp64) on a bounded sample of the
+same workload on this host's cores; it is the reported baseline, not a target.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+from block_sparse_attention_pisa_b200 import roofline as R  # noqa: E402
+
+METRIC = "ms/call and effective TFLOP/s at N=32K,H=24,d=128,12.5% kept; tensor-pipe % of peak"
+UNIT = "TFLOP/s"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+def _workload_desc(wl):
+    return (f"{wl.name}: B={wl.B} H={wl.H} N={wl.N} d={wl.d} block={wl.block} "
+            f"topk={wl.topk}/{wl.nB} ({100.0 * wl.topk / wl.nB:.1f}% exact) order={wl.order} "
+            f"scale={wl.scale:.6g}")
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled in the background."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.lines = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _physical_gpu(local: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    parts = [p for p in vis.split(",") if p.strip()]
+    if parts and parts[min(local, len(parts) - 1)].strip().isdigit():
+        return int(parts[min(local, len(parts) - 1)])
+    return local
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle baseline (the only place bench.py runs oracle/)
+# ----------------------------------------------------------------------------
+def oracle_sample(wl, budget_s: float = 15.0, min_blocks: int = 2):
+    """Time the oracle (stats + select + attention) on one head and as many query
+    blocks as fit in ``budget_s``; returns (TFLOP/s, seconds, description, threads)."""
+    import oracle
+    q, k, v = W.make_inputs(wl.with_(B=1), heads=[0])
+    Qf, Kf, Vf = (W.bf16_bits_to_f32(a).astype(np.float64) for a in (q, k, v))
+    t0 = time.perf_counter()
+    kbar, S0, S1 = oracle.block_stats(Kf, Vf, wl.block, wl.order)
+    idx, _, _ = oracle.select(Qf, kbar, wl.block, wl.topk)
+    t_pre = time.perf_counter() - t0
+    # query blocks spread over the sequence, run until the budget is spent
+    order = np.random.default_rng(0).permutation(wl.nB)
+    done, t1 = 0, time.perf_counter()
+    while done < wl.nB and (done < min_blocks or time.perf_counter() - t1 < budget_s):
+        oracle.attention(Qf, Kf, Vf, kbar, S0, S1, idx, wl.block, wl.order, wl.scale,
+                         query_blocks=[int(order[done])])
+        done += 1
+    t_attn = time.perf_counter() - t1
+    frac_q = done / wl.nB
+    flops = (R.attention_flops(1, 1, wl.N, wl.d, wl.block, wl.topk, wl.order) * frac_q
+             + R.stats_flops(1, 1, wl.N, wl.d, wl.block, wl.order)
+             + R.select_flops(1, 1, wl.N, wl.d, wl.block))
+    secs = t_pre + t_attn
+    threads = _blas_threads()
+    desc = (f"oracle fp64 on head 0 of {wl.name}: full stats + select, attention on {done} of "
+            f"{wl.nB} query blocks ({t_attn:.1f} s); algorithmic flops of that sample / time")
+    return flops / secs / 1e12, secs, desc, threads
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def run_reference(args):
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    wl = W.get(args.workload)
+    per_step = []
+    for i in range(args.warmup + args.steps):
+        tf, secs, desc, thr = oracle_sample(wl, budget_s=args.ref_budget, min_blocks=1)
+        if i >= args.warmup:
+            per_step.append((tf, secs))
+    tf = statistics.mean(t for t, _ in per_step)
+    full_ms = R.step_flops(wl.B, wl.H, wl.N, wl.d, wl.block, wl.topk, wl.order) / (tf * 1e12) * 1e3
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tf, "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": full_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": _config(wl, ws),
+        "cpu_baseline": {"value": tf, "unit": UNIT, "cores": thr, "kind": "oracle", "sample": desc},
+        "e2e": {"value": tf, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "note": "ms_per_step extrapolates the sampled oracle throughput to one full step",
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _config(wl, ws):
+    return {"workload": _workload_desc(wl), "global_batch": wl.B * ws, "seq_len": wl.N,
+            "heads": wl.H, "head_dim": wl.d, "block": wl.block, "topk": wl.topk,
+            "keep": wl.topk / wl.nB, "order": wl.order,
+            "l2": "inputs larger than L2 (Q+K+V %.0f MB per GPU), no flush" % (3 * wl.B * wl.H * wl.N * wl.d * 2 / 1e6),
+            "parallelism": f"dp{ws} (independent batches per GPU, no collective)"}
+
+
+# ----------------------------------------------------------------------------
+# our path
+# ----------------------------------------------------------------------------
+def run_ours(args):
+    import torch
+    import block_sparse_attention_pisa_b200 as P
+
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    wl = W.get(args.workload)
+    q, k, v = W.make_inputs(wl, batch_offset=rank * wl.B)
+    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
+    Q, K, V = to_dev(q), to_dev(k), to_dev(v)
+    nB = wl.nB
+    kbar = torch.empty((wl.B, wl.H, nB, wl.d), device=dev, dtype=torch.float32)
+    S0 = torch.empty_like(kbar)
+    S1 = torch.empty((wl.B, wl.H, nB, wl.d, wl.d), device=dev, dtype=torch.bfloat16) if wl.order else None
+    idx = torch.empty((wl.B, wl.H, nB, wl.topk), device=dev, dtype=torch.int32)
+    O = torch.empty_like(Q)
+    attn = P.attention if args.kernel == "fused" else P.attention_simt
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        P.block_stats(K, V, wl.block, wl.order, out=(kbar, S0, S1))
+        if ev is not None:
+            ev[1].record(stream)
+        P.select(Q, kbar, wl.block, wl.topk, out=idx)
+        if ev is not None:
+            ev[2].record(stream)
+        attn(Q, K, V, kbar, S0, S1, idx, wl.block, wl.order, wl.scale, out=O)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    P.device_error()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    sampler = ClockSampler(_physical_gpu(local)).start() if rank == 0 else None
+    time.sleep(0.3 if sampler else 0)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    clocks = sampler.stop() if sampler else None
+    P.device_error()
+    ms_total = start.elapsed_time(end)
+    t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+    if pg:
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    k_ms = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
+            for i, n in enumerate(("stats", "select", "attention"))}
+
+    flops_step = R.step_flops(wl.B, wl.H, wl.N, wl.d, wl.block, wl.topk, wl.order)
+    value = flops_step * ws / (ms_step * 1e-3) / 1e12
+    att_flops = R.attention_flops(wl.B, wl.H, wl.N, wl.d, wl.block, wl.topk, wl.order)
+    att_tf = att_flops / (k_ms["attention"] * 1e-3) / 1e12
+    dense_tf = R.dense_flops(wl.B, wl.H, wl.N, wl.d) / (k_ms["attention"] * 1e-3) / 1e12
+    st_gbs = R.stats_bytes(wl.B, wl.H, wl.N, wl.d, wl.block, wl.order) / (k_ms["stats"] * 1e-3) / 1e9
+    se_gbs = R.select_bytes(wl.B, wl.H, wl.N, wl.d, wl.block, wl.topk) / (k_ms["select"] * 1e-3) / 1e9
+    pk = _peaks()
+    peak = pk["bf16_sus"]
+
+    # end to end through the public host API: pinned host Q, K, V in, O out
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in (q, k, v))
+        for _ in range(2):
+            P.pisa_host(hq, hk, hv, wl.block, wl.topk, wl.order, wl.scale, device=dev)
+        n_e2e = max(2, min(args.steps, 5))
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            P.pisa_host(hq, hk, hv, wl.block, wl.topk, wl.order, wl.scale, device=dev)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        wall = (time.perf_counter() - t0) * 1e3 / n_e2e
+        ms_e2e = max(e0.elapsed_time(e1) / n_e2e, wall)
+        te = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
+        if pg:
+            pg.all_reduce(te, op=pg.ReduceOp.MAX)
+        ms_e2e = float(te.item())
+        nbytes = 3 * Q.numel() * 2
+        e2e = {"value": flops_step * ws / (ms_e2e * 1e-3) / 1e12, "unit": UNIT,
+               "ms_per_step": ms_e2e, "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": O.numel() * 2}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        tf, secs, desc, thr = oracle_sample(wl, budget_s=args.ref_budget)
+        cpu = {"value": tf, "unit": UNIT, "cores": thr, "kind": "oracle", "sample": desc}
+
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": _config(wl, ws),
+        "roofline": {"bound": "tensor", "kernel": "attention", "achieved": att_tf, "peak": peak,
+                     "unit": "TFLOP/s", "frac": att_tf / peak, "traffic": args.traffic,
+                     "peak_source": f"{pk['source']} bf16 sustained",
+                     "algorithmic_flops_per_launch": att_flops},
+        "kernels_ms": k_ms,
+        "attention_effective_tflops": att_tf,
+        "attention_dense_equivalent_tflops": dense_tf,
+        "stats_gbs": st_gbs, "stats_hbm_frac": st_gbs / pk["hbm"],
+        "select_gbs": se_gbs, "select_hbm_frac": se_gbs / pk["hbm"],
+        "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": 3 * args.steps, "clocks": clocks,
+        "attention_kernel": args.kernel,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="video", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--kernel", choices=["fused", "simt"], default="fused")
+    ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of oracle work per sample")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="DRAM bytes per attention launch from an ncu capture of the current kernel")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,183 @@
+"""PISA piecewise sparse attention for NVIDIA B200 (sm_100a).
+
+A thin ctypes binding over the C ABI in ``include/pisa.h`` (``libpisa.so``,
+built in-tree by ``python -m block_sparse_attention_pisa_b200.build``). The
+binding only marshals arguments: it reads shapes and device pointers from
+torch tensors, allocates outputs with torch, and passes torch's current CUDA
+stream. Every step of the computation runs in the library's CUDA kernels;
+there is no CPU or PyTorch fallback -- if the library is missing or the
+device is not a B200 the calls raise.
+
+Method: "PISA: Piecewise Sparse Attention Is Wiser for Efficient Diffusion
+Transformers" (explainer of arXiv 2602.01077 on gist.science), technical
+summary section 2.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "PisaError", "Shape", "lib", "block_stats", "select", "attention", "attention_simt",
+    "pisa", "pisa_host", "device_error", "num_blocks", "LIB_PATH", "SYMBOLS",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpisa.so")
+
+# entry points declared in include/pisa.h
+SYMBOLS = (
+    "pisa_block_stats", "pisa_select", "pisa_attention", "pisa_attention_simt",
+    "pisa_device_error", "pisa_status_string", "pisa_last_error", "pisa_version",
+)
+
+STATUS = {0: "PISA_OK", 1: "PISA_ERR_INVALID_ARG", 2: "PISA_ERR_UNSUPPORTED",
+          3: "PISA_ERR_CUDA", 4: "PISA_ERR_TIMEOUT"}
+
+
+class PisaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32),
+                ("d", ctypes.c_int32), ("block", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded ``libpisa.so`` (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing: build it with `python -m block_sparse_attention_pisa_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
+    L.pisa_block_stats.argtypes = [vp, vp, Shape, i32, vp, vp, vp, vp]
+    L.pisa_select.argtypes = [vp, vp, Shape, i32, vp, vp]
+    attn = [vp, vp, vp, vp, vp, vp, vp, Shape, i32, i32, f32, vp, vp]
+    L.pisa_attention.argtypes = attn
+    L.pisa_attention_simt.argtypes = attn
+    L.pisa_device_error.argtypes = [vp]
+    L.pisa_status_string.argtypes = [ctypes.c_int]
+    L.pisa_status_string.restype = ctypes.c_char_p
+    L.pisa_last_error.argtypes = []
+    L.pisa_last_error.restype = ctypes.c_char_p
+    L.pisa_version.argtypes = []
+    for name in ("pisa_block_stats", "pisa_select", "pisa_attention", "pisa_attention_simt",
+                 "pisa_device_error", "pisa_version"):
+        getattr(L, name).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def _check(status: int):
+    if status != 0:
+        raise PisaError(status, lib().pisa_last_error().decode())
+
+
+def num_blocks(N: int, block: int) -> int:
+    return -(-N // block)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(t):
+    import torch
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _shape(x, block: int) -> Shape:
+    if x.dim() != 4:
+        raise ValueError("expected a [B, H, N, d] tensor")
+    if not x.is_contiguous():
+        raise ValueError("tensors must be contiguous [B, H, N, d]")
+    B, H, N, d = x.shape
+    return Shape(B, H, N, d, block)
+
+
+def block_stats(K, V, block: int, order: int = 1, out=None):
+    """kbar (fp32), S0 (fp32), S1 (bf16, None at order 0) of every key/value block.
+    ``out`` = (kbar, S0, S1) preallocated outputs (optional)."""
+    import torch
+    s = _shape(K, block)
+    nB = num_blocks(s.N, block)
+    if out is not None:
+        kbar, S0, S1 = out
+    else:
+        kbar = torch.empty((s.B, s.H, nB, s.d), device=K.device, dtype=torch.float32)
+        S0 = torch.empty_like(kbar)
+        S1 = (torch.empty((s.B, s.H, nB, s.d, s.d), device=K.device, dtype=torch.bfloat16)
+              if order == 1 else None)
+    _check(lib().pisa_block_stats(_ptr(K), _ptr(V), s, order, _ptr(kbar), _ptr(S0), _ptr(S1),
+                                  _stream(K)))
+    return kbar, S0, S1
+
+
+def select(Q, kbar, block: int, topk: int, out=None):
+    """int32 [B, H, nB, topk]: critical blocks of every query block (ascending)."""
+    import torch
+    s = _shape(Q, block)
+    nB = num_blocks(s.N, block)
+    idx = (torch.empty((s.B, s.H, nB, topk), device=Q.device, dtype=torch.int32)
+           if out is None else out)
+    _check(lib().pisa_select(_ptr(Q), _ptr(kbar), s, topk, _ptr(idx), _stream(Q)))
+    return idx
+
+
+def _attention(fn, Q, K, V, kbar, S0, S1, idx, block, order, scale, out=None):
+    import torch
+    s = _shape(Q, block)
+    O = torch.empty_like(Q) if out is None else out
+    topk = int(idx.shape[-1])
+    _check(fn(_ptr(Q), _ptr(K), _ptr(V), _ptr(kbar), _ptr(S0), _ptr(S1), _ptr(idx), s, topk,
+              order, float(scale), _ptr(O), _stream(Q)))
+    return O
+
+
+def attention(Q, K, V, kbar, S0, S1, idx, block: int, order: int, scale: float, out=None):
+    """Fused exact + Taylor attention; bf16 [B, H, N, d]."""
+    return _attention(lib().pisa_attention, Q, K, V, kbar, S0, S1, idx, block, order, scale, out)
+
+
+def attention_simt(Q, K, V, kbar, S0, S1, idx, block: int, order: int, scale: float, out=None):
+    """The same operation on the plain CUDA-core cross-check kernel."""
+    return _attention(lib().pisa_attention_simt, Q, K, V, kbar, S0, S1, idx, block, order, scale, out)
+
+
+def pisa(Q, K, V, block: int, topk: int, order: int = 1, scale: float | None = None):
+    """The whole path on device tensors: stats -> select -> attention. Returns (O, idx)."""
+    if scale is None:
+        scale = Q.shape[-1] ** -0.5
+    kbar, S0, S1 = block_stats(K, V, block, order)
+    idx = select(Q, kbar, block, topk)
+    return attention(Q, K, V, kbar, S0, S1, idx, block, order, scale), idx
+
+
+def pisa_host(Q, K, V, block: int, topk: int, order: int = 1, scale: float | None = None,
+              device="cuda"):
+    """The whole path on HOST tensors: copies Q, K, V to the device, runs it, and copies
+    the output back (pinned host memory gives asynchronous copies). Returns O on the host."""
+    import torch
+    dq = Q.to(device, non_blocking=True)
+    dk = K.to(device, non_blocking=True)
+    dv = V.to(device, non_blocking=True)
+    O, _ = pisa(dq, dk, dv, block, topk, order, scale)
+    out = torch.empty(O.shape, dtype=O.dtype, pin_memory=Q.is_pinned())
+    out.copy_(O, non_blocking=True)
+    torch.cuda.current_stream(O.device).synchronize()
+    return out
+
+
+def device_error(stream_tensor=None):
+    """Synchronise the current stream and raise if a kernel flagged the device error word."""
+    import torch
+    st = torch.cuda.current_stream().cuda_stream if stream_tensor is None else _stream(stream_tensor).value
+    _check(lib().pisa_device_error(ctypes.c_void_p(st)))

@@ -1,0 +1,307 @@
+// C ABI of the PISA kernels: argument validation, device checks and launches.
+// The entry points and their contracts are declared in include/pisa.h.
+#include <cstdarg>
+#include <cstdio>
+#include <cmath>
+#include <mutex>
+#include <string>
+
+#include "../../include/pisa.h"
+#include "common.cuh"
+#include "stats.cuh"
+#include "select.cuh"
+#include "attention_simt.cuh"
+#include "attention_tc.cuh"
+
+using pisa::bf16;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+pisa_status_t fail(pisa_status_t s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+pisa_status_t ok() { return PISA_OK; }
+
+#define PISA_TRY(expr)                        \
+  do {                                        \
+    pisa_status_t _s = (expr);                \
+    if (_s != PISA_OK) return _s;             \
+  } while (0)
+
+inline int64_t num_blocks(const pisa_shape_t& s) { return (int64_t(s.N) + s.block - 1) / s.block; }
+
+// Shape sanity. Sets *empty for B*H*N == 0 (nothing to do, nothing touched).
+pisa_status_t check_shape(const pisa_shape_t& s, bool* empty) {
+  *empty = false;
+  if (s.B < 0 || s.H < 0 || s.N < 0)
+    return fail(PISA_ERR_INVALID_ARG, "negative shape (B=%d H=%d N=%d)", s.B, s.H, s.N);
+  if (s.d <= 0 || s.block <= 0)
+    return fail(PISA_ERR_INVALID_ARG, "d and block must be positive (d=%d block=%d)", s.d, s.block);
+  if (int64_t(s.B) * s.H * s.N == 0) {
+    *empty = true;
+    return ok();
+  }
+  return ok();
+}
+
+pisa_status_t check_support(const pisa_shape_t& s) {
+  if (s.d != 64 && s.d != 128) return fail(PISA_ERR_UNSUPPORTED, "head dimension d=%d (supported: 64, 128)", s.d);
+  if (s.block != 64 && s.block != 128)
+    return fail(PISA_ERR_UNSUPPORTED, "block=%d (supported: 64, 128)", s.block);
+  if (num_blocks(s) > PISA_MAX_BLOCKS)
+    return fail(PISA_ERR_UNSUPPORTED, "nB=%lld exceeds PISA_MAX_BLOCKS=%d", (long long)num_blocks(s),
+                PISA_MAX_BLOCKS);
+  if (int64_t(s.B) * s.H > 65535)
+    return fail(PISA_ERR_UNSUPPORTED, "B*H=%lld exceeds 65535", (long long)(int64_t(s.B) * s.H));
+  return ok();
+}
+
+pisa_status_t check_ptr(const void* p, const char* name) {
+  if (p == nullptr) return fail(PISA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (reinterpret_cast<uintptr_t>(p) & 15u) return fail(PISA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return ok();
+}
+
+pisa_status_t check_order(int32_t order) {
+  if (order != 0 && order != 1) return fail(PISA_ERR_INVALID_ARG, "order=%d (must be 0 or 1)", order);
+  return ok();
+}
+
+pisa_status_t check_topk(const pisa_shape_t& s, int32_t topk) {
+  if (topk < 1 || topk > num_blocks(s))
+    return fail(PISA_ERR_INVALID_ARG, "topk=%d outside [1, nB=%lld]", topk, (long long)num_blocks(s));
+  return ok();
+}
+
+// Compute capability 10.0 (B200 / GB200) on the current device; cached per device.
+pisa_status_t check_device(int* sm_count) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(PISA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  static std::mutex mu;
+  static int cached_ok[64] = {0};
+  static int cached_sms[64] = {0};
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev >= 0 && dev < 64 && cached_ok[dev]) {
+    *sm_count = cached_sms[dev];
+    return ok();
+  }
+  int major = 0, minor = 0, sms = 0;
+  if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return fail(PISA_ERR_CUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
+  if (major != 10 || minor != 0)
+    return fail(PISA_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a only", dev, major,
+                minor);
+  if (dev >= 0 && dev < 64) {
+    cached_ok[dev] = 1;
+    cached_sms[dev] = sms;
+  }
+  *sm_count = sms;
+  return ok();
+}
+
+pisa_status_t check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(PISA_ERR_CUDA, "%s launch: %s", what, cudaGetErrorString(e));
+  return ok();
+}
+
+template <typename Kernel>
+pisa_status_t set_smem(Kernel k, size_t bytes) {
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
+  if (e != cudaSuccess) return fail(PISA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+template <int D, int BLK>
+pisa_status_t launch_stats(const pisa_shape_t& s, const bf16* K, const bf16* V, int order, float* kbar,
+                           float* S0, bf16* S1, cudaStream_t st) {
+  using C = pisa::StatsCfg<D, BLK>;
+  auto k = pisa::stats_kernel<D, BLK>;
+  PISA_TRY(set_smem(k, C::kSmem));
+  const int nB = int(num_blocks(s));
+  dim3 grid(nB, s.B * s.H);
+  k<<<grid, C::kThreads, C::kSmem, st>>>(K, V, s.N, nB, order, kbar, S0, S1);
+  return check_launch("stats_kernel");
+}
+
+template <int D>
+pisa_status_t launch_select(const pisa_shape_t& s, const bf16* Q, const float* kbar, int topk, int32_t* idx,
+                            cudaStream_t st) {
+  auto k = pisa::select_kernel<D>;
+  const int nB = int(num_blocks(s));
+  const size_t smem = pisa::select_smem_bytes(D, nB);
+  PISA_TRY(set_smem(k, smem));
+  dim3 grid((nB + pisa::kSelectQB - 1) / pisa::kSelectQB, s.B * s.H);
+  k<<<grid, pisa::kSelectThreads, smem, st>>>(Q, kbar, s.N, nB, s.block, topk, idx);
+  return check_launch("select_kernel");
+}
+
+template <int D>
+pisa_status_t launch_attention_simt(const pisa_shape_t& s, const bf16* Q, const bf16* K, const bf16* V,
+                                    const float* kbar, const float* S0, const bf16* S1, const int32_t* idx,
+                                    int topk, int order, float scale, bf16* O, cudaStream_t st) {
+  auto k = pisa::attention_simt_kernel<D>;
+  const size_t smem = pisa::SimtCfg<D>::smem_bytes();
+  PISA_TRY(set_smem(k, smem));
+  const int nB = int(num_blocks(s));
+  dim3 grid(nB, s.B * s.H);
+  k<<<grid, s.block, smem, st>>>(Q, K, V, kbar, S0, S1, idx, s.N, nB, s.block, topk, order, scale, O);
+  return check_launch("attention_simt_kernel");
+}
+
+struct AttnArgs {
+  const void* Q;
+  const void* K;
+  const void* V;
+  const float* kbar;
+  const float* S0;
+  const void* S1;
+  const int32_t* idx;
+  int32_t topk;
+  int32_t order;
+  float scale;
+  void* O;
+};
+
+pisa_status_t validate_attention(const pisa_shape_t& shape, const AttnArgs& a, bool* empty) {
+  PISA_TRY(check_shape(shape, empty));
+  if (*empty) return ok();
+  PISA_TRY(check_ptr(a.Q, "Q"));
+  PISA_TRY(check_ptr(a.K, "K"));
+  PISA_TRY(check_ptr(a.V, "V"));
+  PISA_TRY(check_ptr(a.kbar, "kbar"));
+  PISA_TRY(check_ptr(a.S0, "S0"));
+  PISA_TRY(check_ptr(a.idx, "idx"));
+  PISA_TRY(check_ptr(a.O, "O"));
+  PISA_TRY(check_order(a.order));
+  if (a.order == 1) PISA_TRY(check_ptr(a.S1, "S1"));
+  PISA_TRY(check_topk(shape, a.topk));
+  if (!std::isfinite(a.scale) || !(a.scale > 0.f))
+    return fail(PISA_ERR_INVALID_ARG, "scale=%g (must be finite and > 0)", double(a.scale));
+  return check_support(shape);
+}
+
+}  // namespace
+
+extern "C" {
+
+pisa_status_t pisa_block_stats(const void* K, const void* V, pisa_shape_t shape, int32_t order, float* kbar,
+                               float* S0, void* S1, void* stream) {
+  bool empty = false;
+  PISA_TRY(check_shape(shape, &empty));
+  if (empty) return ok();
+  PISA_TRY(check_ptr(K, "K"));
+  PISA_TRY(check_ptr(V, "V"));
+  PISA_TRY(check_ptr(kbar, "kbar"));
+  PISA_TRY(check_ptr(S0, "S0"));
+  PISA_TRY(check_order(order));
+  if (order == 1) PISA_TRY(check_ptr(S1, "S1"));
+  PISA_TRY(check_support(shape));
+  int sms = 0;
+  PISA_TRY(check_device(&sms));
+  auto st = static_cast<cudaStream_t>(stream);
+  auto k = static_cast<const bf16*>(K);
+  auto v = static_cast<const bf16*>(V);
+  auto s1 = static_cast<bf16*>(S1);
+  if (shape.d == 128 && shape.block == 64) return launch_stats<128, 64>(shape, k, v, order, kbar, S0, s1, st);
+  if (shape.d == 128 && shape.block == 128) return launch_stats<128, 128>(shape, k, v, order, kbar, S0, s1, st);
+  if (shape.d == 64 && shape.block == 64) return launch_stats<64, 64>(shape, k, v, order, kbar, S0, s1, st);
+  return launch_stats<64, 128>(shape, k, v, order, kbar, S0, s1, st);
+}
+
+pisa_status_t pisa_select(const void* Q, const float* kbar, pisa_shape_t shape, int32_t topk, int32_t* idx,
+                          void* stream) {
+  bool empty = false;
+  PISA_TRY(check_shape(shape, &empty));
+  if (empty) return ok();
+  PISA_TRY(check_ptr(Q, "Q"));
+  PISA_TRY(check_ptr(kbar, "kbar"));
+  PISA_TRY(check_ptr(idx, "idx"));
+  PISA_TRY(check_topk(shape, topk));
+  PISA_TRY(check_support(shape));
+  int sms = 0;
+  PISA_TRY(check_device(&sms));
+  auto st = static_cast<cudaStream_t>(stream);
+  auto q = static_cast<const bf16*>(Q);
+  if (shape.d == 128) return launch_select<128>(shape, q, kbar, topk, idx, st);
+  return launch_select<64>(shape, q, kbar, topk, idx, st);
+}
+
+pisa_status_t pisa_attention(const void* Q, const void* K, const void* V, const float* kbar, const float* S0,
+                             const void* S1, const int32_t* idx, pisa_shape_t shape, int32_t topk, int32_t order,
+                             float scale, void* O, void* stream) {
+  AttnArgs a{Q, K, V, kbar, S0, S1, idx, topk, order, scale, O};
+  bool empty = false;
+  PISA_TRY(validate_attention(shape, a, &empty));
+  if (empty) return ok();
+  int sms = 0;
+  PISA_TRY(check_device(&sms));
+  auto st = static_cast<cudaStream_t>(stream);
+  auto q = static_cast<const bf16*>(Q);
+  auto k = static_cast<const bf16*>(K);
+  auto v = static_cast<const bf16*>(V);
+  auto s1 = static_cast<const bf16*>(S1);
+  auto o = static_cast<bf16*>(O);
+  if (shape.d == 128) return launch_attention_simt<128>(shape, q, k, v, kbar, S0, s1, idx, topk, order, scale, o, st);
+  return launch_attention_simt<64>(shape, q, k, v, kbar, S0, s1, idx, topk, order, scale, o, st);
+}
+
+pisa_status_t pisa_attention_simt(const void* Q, const void* K, const void* V, const float* kbar,
+                                  const float* S0, const void* S1, const int32_t* idx, pisa_shape_t shape,
+                                  int32_t topk, int32_t order, float scale, void* O, void* stream) {
+  AttnArgs a{Q, K, V, kbar, S0, S1, idx, topk, order, scale, O};
+  bool empty = false;
+  PISA_TRY(validate_attention(shape, a, &empty));
+  if (empty) return ok();
+  int sms = 0;
+  PISA_TRY(check_device(&sms));
+  auto st = static_cast<cudaStream_t>(stream);
+  auto q = static_cast<const bf16*>(Q);
+  auto k = static_cast<const bf16*>(K);
+  auto v = static_cast<const bf16*>(V);
+  auto s1 = static_cast<const bf16*>(S1);
+  auto o = static_cast<bf16*>(O);
+  if (shape.d == 128) return launch_attention_simt<128>(shape, q, k, v, kbar, S0, s1, idx, topk, order, scale, o, st);
+  return launch_attention_simt<64>(shape, q, k, v, kbar, S0, s1, idx, topk, order, scale, o, st);
+}
+
+pisa_status_t pisa_device_error(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(PISA_ERR_CUDA, "cudaStreamSynchronize: %s", cudaGetErrorString(e));
+  unsigned word = 0, zero = 0;
+  if ((e = cudaMemcpyFromSymbol(&word, pisa::g_pisa_error, sizeof(word))) != cudaSuccess ||
+      (e = cudaMemcpyToSymbol(pisa::g_pisa_error, &zero, sizeof(zero))) != cudaSuccess)
+    return fail(PISA_ERR_CUDA, "device error word: %s", cudaGetErrorString(e));
+  if (word & pisa::kErrTimeout) return fail(PISA_ERR_TIMEOUT, "a bounded device wait ran out (word=0x%x)", word);
+  if (word & pisa::kErrBadIndex) return fail(PISA_ERR_INVALID_ARG, "idx held an out-of-range block (word=0x%x)", word);
+  return ok();
+}
+
+const char* pisa_status_string(pisa_status_t status) {
+  switch (status) {
+    case PISA_OK: return "PISA_OK";
+    case PISA_ERR_INVALID_ARG: return "PISA_ERR_INVALID_ARG: invalid argument";
+    case PISA_ERR_UNSUPPORTED: return "PISA_ERR_UNSUPPORTED: shape or device not supported";
+    case PISA_ERR_CUDA: return "PISA_ERR_CUDA: CUDA call failed";
+    case PISA_ERR_TIMEOUT: return "PISA_ERR_TIMEOUT: bounded device wait ran out";
+  }
+  return "unknown pisa_status_t";
+}
+
+const char* pisa_last_error(void) { return g_last_error.c_str(); }
+
+int32_t pisa_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,185 @@
+// Block statistics: kbar (centroid), S0 (value sum), S1 (first-order matrix).
+//
+// PISA explainer ("PISA: Piecewise Sparse Attention Is Wiser for Efficient
+// Diffusion Transformers"), technical summary section 2, "Hardware
+// implementation": the precompute step forms the block centroids and value sums
+// before the fused kernel runs. S1_j = sum_n (k_n - kbar_j) v_n^T is the
+// first-order Taylor matrix of block j.
+//
+// One CTA per (block j, head). K_j and V_j are streamed once from HBM with
+// 16-byte coalesced loads into padded shared memory; the column sums are
+// reduced with warp shuffles and a small shared-memory pass. S1 is formed as
+// K_j^T V_j on the tensor cores (fp32 accumulation over bf16 inputs, so the
+// products are exact) minus kbar_j S0_j^T in fp32, rounded once to bf16, staged
+// in shared memory and written with coalesced 16-byte stores.
+//
+// The kernel is HBM-bound (K, V in; S1 out). The d x b x d contraction is ~32
+// flop/byte, below the tensor ridge, so the warp-level mma.sync path keeps it
+// under the memory time.
+#pragma once
+
+#include "common.cuh"
+
+namespace pisa {
+
+template <int D, int BLK>
+struct StatsCfg {
+  static constexpr int kThreads = 256;
+  static constexpr int kLd = D + 8;             // padded smem row (elements): conflict-free ldmatrix
+  static constexpr int kChunks = D / 8;         // 16-byte chunks per row
+  static constexpr int kRowStep = kThreads / kChunks;
+  static constexpr int kTileElems = BLK * kLd;  // one of sK / sV
+  static constexpr size_t kSmem = size_t(2) * kTileElems * sizeof(bf16)  // sK, sV (S1 staging reuses both)
+                                  + size_t(8) * 2 * D * sizeof(float)    // per-warp partial sums
+                                  + size_t(2) * D * sizeof(float);       // kbar, S0
+  static_assert(2 * kTileElems >= D * kLd, "S1 staging must fit in the K/V tiles");
+};
+
+template <int D, int BLK>
+__global__ void __launch_bounds__(256)
+stats_kernel(const bf16* __restrict__ K, const bf16* __restrict__ V, int N, int nB, int order,
+             float* __restrict__ kbar, float* __restrict__ S0, bf16* __restrict__ S1) {
+  using C = StatsCfg<D, BLK>;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  bf16* sK = reinterpret_cast<bf16*>(smem_raw);
+  bf16* sV = sK + C::kTileElems;
+  float* sPart = reinterpret_cast<float*>(sV + C::kTileElems);  // [8 warps][2][D]
+  float* sKbar = sPart + 8 * 2 * D;
+  float* sS0 = sKbar + D;
+
+  const int j = blockIdx.x;
+  const size_t bh = blockIdx.y;
+  const int start = j * BLK;
+  const int n = min(BLK, N - start);
+  const bf16* gK = K + (bh * size_t(N) + start) * D;
+  const bf16* gV = V + (bh * size_t(N) + start) * D;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int ch = tid % C::kChunks;
+  const int r0 = tid / C::kChunks;
+
+  // ---- stream K_j, V_j once (rows >= n are zero-filled) and sum columns ----
+  float ks[8], vs[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) ks[e] = vs[e] = 0.f;
+#pragma unroll
+  for (int r = r0; r < BLK; r += C::kRowStep) {
+    uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
+    if (r < n) {
+      kv = ldg_stream_v4(gK + size_t(r) * D + ch * 8);
+      vv = ldg_stream_v4(gV + size_t(r) * D + ch * 8);
+    }
+    *reinterpret_cast<uint4*>(sK + r * C::kLd + ch * 8) = kv;
+    *reinterpret_cast<uint4*>(sV + r * C::kLd + ch * 8) = vv;
+    const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+    const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      ks[2 * e] += bf16_lo(kw[e]);
+      ks[2 * e + 1] += bf16_hi(kw[e]);
+      vs[2 * e] += bf16_lo(vw[e]);
+      vs[2 * e + 1] += bf16_hi(vw[e]);
+    }
+  }
+  // lanes holding the same chunk index sit kChunks apart inside the warp
+#pragma unroll
+  for (int off = C::kChunks; off < 32; off <<= 1) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      ks[e] += __shfl_xor_sync(0xffffffffu, ks[e], off);
+      vs[e] += __shfl_xor_sync(0xffffffffu, vs[e], off);
+    }
+  }
+  if (lane < C::kChunks) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      sPart[(warp * 2 + 0) * D + ch * 8 + e] = ks[e];
+      sPart[(warp * 2 + 1) * D + ch * 8 + e] = vs[e];
+    }
+  }
+  __syncthreads();
+  if (tid < 2 * D) {
+    const int which = tid / D, col = tid % D;
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) s += sPart[(w * 2 + which) * D + col];
+    const size_t o = (bh * size_t(nB) + j) * D + col;
+    if (which == 0) {
+      const float kb = s / float(n);
+      sKbar[col] = kb;
+      kbar[o] = kb;
+    } else {
+      sS0[col] = s;
+      S0[o] = s;
+    }
+  }
+  if (order == 0) return;
+  __syncthreads();
+
+  // ---- S1 = K^T V - kbar S0^T : M = D (key dim a), N = D (value dim c), K = BLK tokens ----
+  constexpr int TM = D / 4, TN = D / 2;      // warp tile (8 warps as 4 x 2)
+  constexpr int MT = TM / 16, NT = TN / 8;
+  const int a_base = (warp >> 1) * TM;
+  const int c_base = (warp & 1) * TN;
+  float acc[MT][NT][4];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+
+  const uint32_t sK_u = smem_u32(sK), sV_u = smem_u32(sV);
+#pragma unroll
+  for (int kt = 0; kt < BLK / 16; ++kt) {
+    uint32_t af[MT][4];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      // A[a][n] = K[n][a]: transposed 8x8 loads from rows n, columns a
+      const int row = kt * 16 + (lane & 7) + ((lane >> 4) << 3);
+      const int col = a_base + mt * 16 + (((lane >> 3) & 1) << 3);
+      ldsm_x4_trans(sK_u + (row * C::kLd + col) * 2, af[mt][0], af[mt][1], af[mt][2], af[mt][3]);
+    }
+#pragma unroll
+    for (int np = 0; np < NT / 2; ++np) {
+      // B[n][c] = V[n][c]: two n8 tiles per x4 load
+      const int row = kt * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+      const int col = c_base + np * 16 + ((lane >> 4) << 3);
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_trans(sV_u + (row * C::kLd + col) * 2, b0, b1, b2, b3);
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        mma_bf16_16816(acc[mt][2 * np], af[mt], b0, b1);
+        mma_bf16_16816(acc[mt][2 * np + 1], af[mt], b2, b3);
+      }
+    }
+  }
+  __syncthreads();  // all warps are done reading sK / sV: reuse them as the S1 staging tile
+
+  bf16* sOut = sK;  // [D][kLd]
+  const int g = lane >> 2, t4 = lane & 3;
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int a = a_base + mt * 16 + g;
+      const int c = c_base + nt * 8 + 2 * t4;
+      const float k0 = sKbar[a], k1 = sKbar[a + 8];
+      const float s0 = sS0[c], s1 = sS0[c + 1];
+      *reinterpret_cast<uint32_t*>(sOut + a * C::kLd + c) =
+          pack_bf16x2(acc[mt][nt][0] - k0 * s0, acc[mt][nt][1] - k0 * s1);
+      *reinterpret_cast<uint32_t*>(sOut + (a + 8) * C::kLd + c) =
+          pack_bf16x2(acc[mt][nt][2] - k1 * s0, acc[mt][nt][3] - k1 * s1);
+    }
+  }
+  __syncthreads();
+  bf16* gS1 = S1 + (bh * size_t(nB) + j) * D * D;
+#pragma unroll 4
+  for (int q = tid; q < D * C::kChunks; q += C::kThreads) {
+    const int a = q / C::kChunks, c8 = q % C::kChunks;
+    *reinterpret_cast<uint4*>(gS1 + size_t(a) * D + c8 * 8) =
+        *reinterpret_cast<const uint4*>(sOut + a * C::kLd + c8 * 8);
+  }
+}
+
+}  // namespace pisa

@@ -1,0 +1,64 @@
+"""Algorithmic work of each kernel (what PISA must do, not the dense work it avoids).
+
+Per-unit figures:
+
+* attention: 4*b*d flops per (query, critical block) -- QK^T and PV --
+  plus 4*d per (query, non-critical block) -- x.kbar and alpha*S0 -- plus,
+  at order 1, 2*d*d per (query, non-critical block) -- S1^T x. Ragged blocks
+  count at their mean size N / nB.
+* stats: bytes = K and V read (2*N*d*2 per head) + kbar and S0 written
+  (2*nB*d*4) + S1 written (nB*d*d*2 at order 1); flops = 2*n*d*d per block
+  for K^T V.
+* select: bytes = Q read (N*d*2) + kbar read (nB*d*4) + idx written
+  (nB*k*4); flops = 2*d per (query block, key block) pooled score.
+* dense-equivalent attention flops: 4*N*N*d per head.
+"""
+from __future__ import annotations
+
+
+def num_blocks(N: int, block: int) -> int:
+    return -(-N // block)
+
+
+def attention_flops(B, H, N, d, block, topk, order) -> float:
+    nB = num_blocks(N, block)
+    mean_n = N / nB
+    rest = nB - topk
+    per_q = 4.0 * mean_n * d * topk + 4.0 * d * rest + (2.0 * d * d * rest if order >= 1 else 0.0)
+    return float(B * H * N * per_q)
+
+
+def attention_bytes(B, H, N, d, block, topk, order) -> float:
+    """Compulsory HBM traffic of one attention call (each operand once)."""
+    nB = num_blocks(N, block)
+    qkvo = 4 * N * d * 2
+    stats = 2 * nB * d * 4 + (nB * d * d * 2 if order >= 1 else 0)
+    return float(B * H * (qkvo + stats + nB * topk * 4))
+
+
+def dense_flops(B, H, N, d) -> float:
+    return 4.0 * B * H * N * N * d
+
+
+def stats_bytes(B, H, N, d, block, order) -> float:
+    nB = num_blocks(N, block)
+    return float(B * H * (2 * N * d * 2 + 2 * nB * d * 4 + (nB * d * d * 2 if order >= 1 else 0)))
+
+
+def stats_flops(B, H, N, d, block, order) -> float:
+    return float(B * H * 2.0 * N * d * d) if order >= 1 else 0.0
+
+
+def select_bytes(B, H, N, d, block, topk) -> float:
+    nB = num_blocks(N, block)
+    return float(B * H * (N * d * 2 + nB * d * 4 + nB * topk * 4))
+
+
+def select_flops(B, H, N, d, block) -> float:
+    nB = num_blocks(N, block)
+    return float(B * H * 2.0 * nB * nB * d)
+
+
+def step_flops(B, H, N, d, block, topk, order) -> float:
+    return (attention_flops(B, H, N, d, block, topk, order) + stats_flops(B, H, N, d, block, order)
+            + select_flops(B, H, N, d, block))

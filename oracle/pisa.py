@@ -159,9 +159,9 @@ def attention(Q, K, V, kbar, S0, S1, idx, block: int, order: int, scale: float,
             num = w @ V[b, h, keys] + alpha @ S0[b, h, rest]
             den = w.sum(axis=1) + alpha @ counts[rest]
             if order >= 1 and rest:
-                # S1_j^T x_t for every (t, j): first[t, j, c] = sum_a x[t, a] S1_j[a, c]
-                first = np.einsum("ta,jac->tjc", X, S1[b, h, rest])
-                num = num + np.einsum("tj,tjc->tc", alpha, first)
+                # S1_j^T x_t for every (j, t): first[j, t, c] = sum_a x[t, a] S1_j[a, c]
+                first = np.matmul(X[None], S1[b, h, rest])
+                num = num + np.einsum("tj,jtc->tc", alpha, first)
             O[b, h, s_i:e_i] = num / den[:, None]
     return O
 

@@ -1,0 +1,53 @@
+"""Helpers shared by the GPU parity tests: moving generated inputs to the
+device, running the oracle on the same bf16-rounded values, and the error
+measures with the tolerances that the outputs must meet."""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+import workloads as W
+
+# Output tolerances: max abs error and L1-relative error sum|o - o*| / sum|o*|.
+MAX_ABS = 1e-2
+MEAN_REL = 5e-3
+
+
+def to_device(bits: np.ndarray):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def to_f64(bits: np.ndarray) -> np.ndarray:
+    return W.bf16_bits_to_f32(bits).astype(np.float64)
+
+
+def bf16_to_f64(t) -> np.ndarray:
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def errors(out: np.ndarray, ref: np.ndarray):
+    diff = np.abs(out - ref)
+    return float(diff.max()), float(diff.sum() / np.abs(ref).sum())
+
+
+def assert_close(out, ref, what=""):
+    mx, rel = errors(out, ref)
+    assert mx <= MAX_ABS and rel <= MEAN_REL, f"{what}: max abs {mx:.3e}, mean rel {rel:.3e}"
+    return mx, rel
+
+
+def compare_idx(gpu_idx: np.ndarray, ref_idx: np.ndarray, near: np.ndarray):
+    """Rows must match exactly unless the oracle recorded a near-tie there.
+    Returns (mismatched rows, of which near-ties)."""
+    bad = np.any(gpu_idx != ref_idx, axis=-1)
+    return int(bad.sum()), int((bad & near).sum()), bad
+
+
+def oracle_pipeline(Qf, Kf, Vf, wl: W.Workload, query_blocks=None):
+    """Oracle stats -> select -> attention on fp64 copies of the inputs."""
+    kbar, S0, S1 = oracle.block_stats(Kf, Vf, wl.block, wl.order)
+    idx, near, _ = oracle.select(Qf, kbar, wl.block, wl.topk)
+    O = oracle.attention(Qf, Kf, Vf, kbar, S0, S1, idx, wl.block, wl.order, wl.scale,
+                         query_blocks=query_blocks)
+    return dict(kbar=kbar, S0=S0, S1=S1, idx=idx, near=near, O=O)

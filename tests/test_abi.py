@@ -1,0 +1,131 @@
+"""The C-ABI library on the CPU: it loads, exports every entry point that
+include/pisa.h declares, and rejects bad arguments on the host before any
+launch. Nothing here launches a kernel."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_attention_pisa_b200 as P
+from block_sparse_attention_pisa_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pisa.h")
+
+OK, INVALID, UNSUPPORTED, CUDA_ERR = 0, 1, 2, 3
+FAKE = 0x7f0000100000          # 16-byte aligned, never dereferenced (validation stops first)
+MISALIGNED = FAKE + 4
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return P.lib()
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^\S.*?\b(pisa_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_binding_symbols():
+    assert _declared() == sorted(P.SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in _declared():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for code in range(5):
+        assert L.pisa_status_string(code)
+    assert L.pisa_version() >= 100
+
+
+def shape(B=1, H=2, N=256, d=128, block=64):
+    return P.Shape(B, H, N, d, block)
+
+
+def vp(x):
+    return ctypes.c_void_p(x)
+
+
+def stats(L, s=None, K=FAKE, V=FAKE, order=1, kbar=FAKE, S0=FAKE, S1=FAKE):
+    return L.pisa_block_stats(vp(K), vp(V), s or shape(), order, vp(kbar), vp(S0), vp(S1), None)
+
+
+def sel(L, s=None, Q=FAKE, kbar=FAKE, topk=2, idx=FAKE):
+    return L.pisa_select(vp(Q), vp(kbar), s or shape(), topk, vp(idx), None)
+
+
+def attn(L, s=None, topk=2, order=1, scale=0.125, fn="pisa_attention", **ptrs):
+    p = {k: FAKE for k in ("Q", "K", "V", "kbar", "S0", "S1", "idx", "O")}
+    p.update(ptrs)
+    return getattr(L, fn)(vp(p["Q"]), vp(p["K"]), vp(p["V"]), vp(p["kbar"]), vp(p["S0"]),
+                          vp(p["S1"]), vp(p["idx"]), s or shape(), topk, order, scale,
+                          vp(p["O"]), None)
+
+
+def test_null_and_misaligned_pointers(L):
+    assert stats(L, K=0) == INVALID
+    assert b"K is NULL" in L.pisa_last_error()
+    assert stats(L, V=MISALIGNED) == INVALID
+    assert b"16-byte" in L.pisa_last_error()
+    assert stats(L, S1=0) == INVALID            # order 1 needs S1
+    assert sel(L, idx=0) == INVALID
+    for name in ("Q", "K", "V", "kbar", "S0", "S1", "idx", "O"):
+        assert attn(L, **{name: 0}) == INVALID, name
+        assert attn(L, **{name: MISALIGNED}) == INVALID, name
+        assert attn(L, fn="pisa_attention_simt", **{name: 0}) == INVALID, name
+
+
+def test_bad_scalars(L):
+    assert stats(L, order=2) == INVALID
+    assert sel(L, topk=0) == INVALID
+    assert sel(L, topk=5) == INVALID            # nB = 4
+    assert attn(L, topk=0) == INVALID
+    assert attn(L, order=-1) == INVALID
+    for sc in (0.0, -1.0, float("nan"), float("inf")):
+        assert attn(L, scale=sc) == INVALID, sc
+    assert attn(L, s=shape(N=-1)) == INVALID
+    assert attn(L, s=shape(d=0)) == INVALID
+
+
+def test_unsupported_shapes(L):
+    assert stats(L, s=shape(d=96)) == UNSUPPORTED
+    assert stats(L, s=shape(block=32)) == UNSUPPORTED
+    assert sel(L, s=shape(N=64 * 2049), topk=4) == UNSUPPORTED   # nB > PISA_MAX_BLOCKS
+    assert attn(L, s=shape(B=300, H=300)) == UNSUPPORTED
+
+
+def test_order0_needs_no_S1(L):
+    # with S1 = NULL at order 0 validation passes and only the device check remains
+    st = stats(L, order=0, S1=0)
+    assert st in (OK, CUDA_ERR, UNSUPPORTED)
+    if st != OK:
+        assert b"cuda" in L.pisa_last_error().lower() or b"sm_" in L.pisa_last_error()
+
+
+def test_empty_problem_touches_nothing(L):
+    # B*H*N == 0: OK with NULL pointers, no launch
+    assert stats(L, s=shape(N=0), K=0, V=0, kbar=0, S0=0, S1=0) == OK
+    assert sel(L, s=shape(H=0), Q=0, kbar=0, idx=0, topk=0) == OK
+    assert attn(L, s=shape(B=0), Q=0, K=0, V=0, kbar=0, S0=0, S1=0, idx=0, O=0) == OK
+
+
+def test_valid_call_without_gpu_reports_cuda_error(L):
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("fake pointers must never reach a real device")
+    assert stats(L) == CUDA_ERR
+    assert sel(L) == CUDA_ERR
+    assert attn(L) == CUDA_ERR
+
+
+def test_binding_raises_on_missing_library(tmp_path, monkeypatch):
+    monkeypatch.setattr(P, "LIB_PATH", str(tmp_path / "libpisa.so"))
+    monkeypatch.setattr(P, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        P.lib()

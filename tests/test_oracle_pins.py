@@ -84,7 +84,8 @@ MUTATIONS = {
     "scale missing from alpha": ("z_ap = X @ kbar", "z_ap = Q[b, h, s_i:e_i] @ kbar"),
     "first-order sign flipped": ("num = num + np.einsum", "num = num - np.einsum"),
     "ragged centroid over b": ("Kj.sum(axis=2) / (e - s)", "Kj.sum(axis=2) / block"),
-    "S1 transposed in attention": ('"ta,jac->tjc"', '"ta,jca->tjc"'),
+    "S1 transposed in attention": ("np.matmul(X[None], S1[b, h, rest])",
+                                   "np.matmul(X[None], np.swapaxes(S1[b, h, rest], -1, -2))"),
     "value mean instead of sum": ("S0[:, :, j] = Vj.sum(axis=2)", "S0[:, :, j] = Vj.mean(axis=2)"),
     "pooled query over wrong rows": ("Q[:, :, s:e, :].sum(axis=2) / (e - s)",
                                      "Q[:, :, s:s + 1, :].sum(axis=2)"),

@@ -30,8 +30,10 @@ GPU receives the bf16 bits and the oracle the same values upcast to fp64.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import dataclasses
 import math
+import os
 
 import numpy as np
 
@@ -172,21 +174,31 @@ def make_head(wl: Workload, b: int, h: int, tensor: str, coords=None) -> np.ndar
     return to_bf16_bits(x)
 
 
-def make_inputs(wl: Workload, heads=None):
+def make_inputs(wl: Workload, heads=None, batch_offset: int = 0):
     """Q, K, V as bf16 bits, each uint16 [B, H, N, d] (or [B, len(heads), N, d]).
 
     ``heads`` selects a subset of (batch-independent) head indices; the values
-    of a head do not depend on which other heads are generated.
+    of a head do not depend on which other heads are generated. ``batch_offset``
+    shifts the batch indices (one process per GPU draws its own batch).
     """
     heads = list(range(wl.H)) if heads is None else list(heads)
     coords = grid_of(wl) if wl.kind != "normal" else None
-    out = []
-    for t in ("q", "k", "v"):
-        arr = np.empty((wl.B, len(heads), wl.N, wl.d), dtype=np.uint16)
-        for b in range(wl.B):
-            for hi, h in enumerate(heads):
-                arr[b, hi] = make_head(wl, b, h, t, coords)
-        out.append(arr)
+    out = [np.empty((wl.B, len(heads), wl.N, wl.d), dtype=np.uint16) for _ in range(3)]
+    jobs = [(ti, t, b, hi, h) for ti, t in enumerate(("q", "k", "v"))
+            for b in range(wl.B) for hi, h in enumerate(heads)]
+
+    def fill(job):
+        ti, t, b, hi, h = job
+        out[ti][b, hi] = make_head(wl, b + batch_offset, h, t, coords)
+
+    # every slice has its own seed, so the result does not depend on the thread schedule
+    workers = min(len(jobs), max(1, min(16, os.cpu_count() or 1)))
+    if workers > 1:
+        with concurrent.futures.ThreadPoolExecutor(workers) as ex:
+            list(ex.map(fill, jobs))
+    else:
+        for job in jobs:
+            fill(job)
     return tuple(out)
 
 
