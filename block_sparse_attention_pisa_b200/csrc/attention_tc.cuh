@@ -1,3 +1,661 @@
-// Fused tensor-core PISA attention (tcgen05 / TMEM / TMA) -- see below.
+// Fused PISA attention on the 5th-generation tensor cores (tcgen05 / TMEM / TMA).
+//
+// PISA explainer ("PISA: Piecewise Sparse Attention Is Wiser for Efficient
+// Diffusion Transformers"), technical summary section 2: "Core algorithm"
+// (o_t = N_t / D_t; exact term over the critical blocks S_i; zeroth-order term
+// alpha_{t,j} S0_j with alpha = exp(x.kbar_j); a first-order term in the
+// numerator) and "Hardware implementation" (a fused FlashAttention-style
+// online softmax with an exact stage over the selected blocks and an
+// approximate stage over the pooled block statistics). The first-order term is
+// the per-block Taylor term alpha_{t,j} S1_j^T x_t with S1_j = sum (k - kbar_j) v^T.
+//
+// One CTA computes a tile of 128 query rows of one head (two query blocks at
+// b = 64, one at b = 128). Warp roles:
+//   warp 0      TMA producer: K_j, V_j of the exact blocks, then S1_j of the
+//               approximated blocks, through a ring of 32 KB shared-memory stages;
+//   warp 1      MMA issuer (one thread): all tcgen05.mma of the tile;
+//   warps 2-3   build the block lists, then convert fp32 kbar / S0 chunks of 64
+//               blocks into bf16 swizzled shared-memory operands;
+//   warps 4-7   one thread per query row (= TMEM lane): online softmax, the
+//               Taylor weights and the tensor-memory operands.
+// Tensor memory (512 columns): O accumulator (D cols), the tile's queries Q as
+// the A operand of QK^T and Q kbar^T (D/2 cols), then either the two exact
+// score buffers S (P overwrites its own S) or, in the approximate stage, two
+// pooled-score buffers Sbar (the bf16 alpha operand overwrites its own Sbar)
+// and a ring of three A_j = (alpha_j * scale) (.) q operands.
+//
+// Exact stage, per block j in the union of the tile's selections:
+//   S = Q K_j^T (TS-MMA), P = exp(x.k - m) (zero for rows whose query block
+//   did not select j and for keys past N), O += P V_j (TS-MMA, V MN-major).
+// Approximate stage, per chunk of 64 key blocks:
+//   Sbar = Q Kbar_c^T, alpha = exp(x.kbar - m) (zero for blocks a row's own
+//   query block selected), O += alpha S0_c (one MMA for the zeroth order), and
+//   for every block j of the chunk that some row approximates, O += A_j S1_j
+//   (TS-MMA, S1 MN-major): the first-order term as one long-K GEMM.
+// Denominator: sum of P plus sum n_j alpha_j, kept in fp32 registers.
+// One running row maximum covers both stages; the accumulator is rescaled only
+// when the maximum grows by more than 2^8 (exact by construction, rare).
 #pragma once
-#include "common.cuh"
+
+#include "tc_ptx.cuh"
+
+namespace pisa {
+
+struct TcParams {
+  const bf16* Q;
+  const float* kbar;
+  const float* S0;
+  const int32_t* idx;
+  bf16* O;
+  int N;
+  int nB;
+  int topk;
+  int order;
+  float scale;
+};
+
+template <int D, int BLK>
+struct TcCfg {
+  static constexpr int kThreads = 256;
+  static constexpr int NS = (D == 128) ? 4 : 8;             // TMA ring stages
+  static constexpr int STAGE = (D == 128) ? 32768 : 16384;  // bytes per stage
+  static constexpr int CHUNK = 64;                          // key blocks per approximate chunk
+  static constexpr int CV_HALF = CHUNK * D * 2;             // bf16 kbar (or S0) chunk
+  static constexpr int CV_STAGE = 2 * CV_HALF;
+  static constexpr int NA = 3;                              // A_j ring depth
+  static constexpr int MAXB = 2048;
+  // tensor-memory columns
+  static constexpr int O_COL = 0;
+  static constexpr int Q_COL = D;
+  static constexpr int R_COL = D + D / 2;
+  static constexpr int A_COL0 = R_COL + 128;
+  static constexpr int A_COLS = D / 2;
+  static constexpr int TMEM_COLS = 512;
+  static_assert(R_COL + 2 * BLK <= TMEM_COLS, "exact score buffers exceed TMEM");
+  static_assert(A_COL0 + NA * A_COLS <= TMEM_COLS, "operand ring exceeds TMEM");
+  static_assert(STAGE >= BLK * D * 2 && STAGE >= D * D * 2, "stage too small");
+  // barriers
+  static constexpr int B_FULL = 0, B_EMPTY = NS, B_CVF = 2 * NS, B_CVE = B_CVF + 2, B_Q = B_CVE + 2;
+  static constexpr int B_SF = B_Q + 1, B_PF = B_SF + 2, B_PV = B_PF + 2, B_SBF = B_PV + 2;
+  static constexpr int B_A0F = B_SBF + 2, B_SBE = B_A0F + 2, B_AF = B_SBE + 2, B_AE = B_AF + NA;
+  static constexpr int B_OSYNC = B_AE + NA, B_ODONE = B_OSYNC + 1, NBARS = B_ODONE + 1;
+  // shared memory (offsets from a 1024-byte aligned base)
+  static constexpr int OFF_RING = 0;
+  static constexpr int OFF_CV = OFF_RING + NS * STAGE;
+  static constexpr int OFF_EXACT = OFF_CV + 2 * CV_STAGE;
+  static constexpr int OFF_APPROX = OFF_EXACT + 2 * MAXB;
+  static constexpr int OFF_CHUNK = OFF_APPROX + 2 * MAXB;
+  static constexpr int OFF_MASK = OFF_CHUNK + 4 * (MAXB / CHUNK + 1 + 3);
+  static constexpr int OFF_BAR = OFF_MASK + 2 * (MAXB / 32) * 4;
+  static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
+  static constexpr int SMEM = OFF_MISC + 64 + 1024;  // + alignment slack
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+};
+
+namespace tc {
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t hmul2_bf16(uint32_t a, uint32_t b) {
+  __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&a);
+  __nv_bfloat162 y = *reinterpret_cast<__nv_bfloat162*>(&b);
+  __nv_bfloat162 z = __hmul2(x, y);
+  return *reinterpret_cast<uint32_t*>(&z);
+}
+
+// bounded wait that ignores the abort flag: used only to drain copies / MMAs
+// already in flight before the CTA releases its shared and tensor memory
+__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitCycles) {
+      flag_error(kErrTimeout);
+      return;
+    }
+  }
+}
+
+// scale one TMEM row of D fp32 columns by f (warp-collective)
+template <int D>
+__device__ __forceinline__ void rescale_row(uint32_t taddr, float f) {
+#pragma unroll
+  for (int ch = 0; ch < D / 16; ++ch) {
+    uint32_t o[16];
+    tmem_ld16(taddr + ch * 16, o);
+    tmem_wait_ld(o);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+    tmem_st16(taddr + ch * 16, o);
+  }
+  tmem_wait_st();
+}
+
+}  // namespace tc
+
+template <int D, int BLK>
+__global__ void __launch_bounds__(256, 1)
+attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    const __grid_constant__ CUtensorMap tmS1, const TcParams p) {
+  using C = TcCfg<D, BLK>;
+  using namespace tc;
+  extern __shared__ __align__(16) uint8_t tc_smem_raw[];
+  const uint32_t raw_u = smem_u32(tc_smem_raw);
+  const uint32_t base_u = (raw_u + 1023u) & ~1023u;  // 128-byte swizzled tiles need 1024-byte alignment
+  uint8_t* base = tc_smem_raw + (base_u - raw_u);
+  int16_t* exact_list = reinterpret_cast<int16_t*>(base + C::OFF_EXACT);
+  int16_t* approx_list = reinterpret_cast<int16_t*>(base + C::OFF_APPROX);
+  int* chunk_off = reinterpret_cast<int*>(base + C::OFF_CHUNK);
+  uint32_t* mask = reinterpret_cast<uint32_t*>(base + C::OFF_MASK);  // [2][MAXB/32]
+  int* misc = reinterpret_cast<int*>(base + C::OFF_MISC);              // tmem, abort, n_exact, n_approx
+  volatile int* abort_flag = misc + 1;
+  const uint32_t bar0 = base_u + C::OFF_BAR;
+#define BAR(i) (bar0 + 8u * uint32_t(i))
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int N = p.N, nB = p.nB;
+  const int nW = (nB + 31) >> 5;
+  const int nC = (nB + C::CHUNK - 1) / C::CHUNK;
+  constexpr bool kTwo = (BLK == 64);  // two query blocks per 128-row tile
+  const int i0 = kTwo ? 2 * tile : tile;
+
+  // ------------------------------------------------------------- prologue
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(BAR(C::B_FULL + s), 1);
+      mbar_init(BAR(C::B_EMPTY + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(BAR(C::B_CVF + s), 64);
+      mbar_init(BAR(C::B_CVE + s), 1);
+      mbar_init(BAR(C::B_SF + s), 1);
+      mbar_init(BAR(C::B_PF + s), 128);
+      mbar_init(BAR(C::B_PV + s), 1);
+      mbar_init(BAR(C::B_SBF + s), 1);
+      mbar_init(BAR(C::B_A0F + s), 128);
+      mbar_init(BAR(C::B_SBE + s), 1);
+    }
+    for (int s = 0; s < C::NA; ++s) {
+      mbar_init(BAR(C::B_AF + s), 128);
+      mbar_init(BAR(C::B_AE + s), 1);
+    }
+    mbar_init(BAR(C::B_Q), 128);
+    mbar_init(BAR(C::B_OSYNC), 1);
+    mbar_init(BAR(C::B_ODONE), 1);
+    misc[1] = 0;
+    mbar_init_fence();
+  }
+  if (warp == 2) {
+    tmem_alloc(base_u + C::OFF_MISC, C::TMEM_COLS);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (warp == 3) {
+    // critical-block bitmasks of the tile's query block(s)
+    for (int w = lane; w < 2 * (C::MAXB / 32); w += 32) mask[w] = 0u;
+    __syncwarp();
+    for (int q = 0; q < (kTwo ? 2 : 1); ++q) {
+      const int i = i0 + q;
+      if (i >= nB) continue;
+      const int32_t* row = p.idx + (size_t(bh) * nB + i) * p.topk;
+      for (int e = lane; e < p.topk; e += 32) {
+        const int j = row[e];
+        if (j >= 0 && j < nB) atomicOr(&mask[q * (C::MAXB / 32) + (j >> 5)], 1u << (j & 31));
+        else flag_error(kErrBadIndex);
+      }
+    }
+    __syncwarp();
+    if (kTwo && i0 + 1 >= nB)  // no second query block: its (padding) rows follow the first
+      for (int w = lane; w < nW; w += 32) mask[C::MAXB / 32 + w] = mask[w];
+    __syncwarp();
+    const uint32_t* m0 = mask;
+    const uint32_t* m1 = kTwo ? mask + C::MAXB / 32 : mask;
+    // exact list = union of the selections; approximate list = blocks that some
+    // row does not take exactly; both ascending; chunk_off[c] = first approximate
+    // entry of chunk c
+    int ne = 0, na = 0;
+    for (int wb = 0; wb < nW; wb += 32) {
+      const int w = wb + lane;
+      uint32_t u = 0, a = 0;
+      if (w < nW) {
+        const uint32_t valid = (w == nW - 1 && (nB & 31)) ? ((1u << (nB & 31)) - 1u) : 0xffffffffu;
+        u = (m0[w] | m1[w]) & valid;
+        a = ~(m0[w] & m1[w]) & valid;
+      }
+      const int pu = __popc(u), pa = __popc(a);
+      int xu = pu, xa = pa;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int tu = __shfl_up_sync(0xffffffffu, xu, off);
+        const int ta = __shfl_up_sync(0xffffffffu, xa, off);
+        if (lane >= off) {
+          xu += tu;
+          xa += ta;
+        }
+      }
+      int eu = ne + xu - pu, ea = na + xa - pa;
+      if (w < nW && (w & 1) == 0) chunk_off[w >> 1] = ea;
+      while (u) {
+        const int bit = __ffs(u) - 1;
+        u &= u - 1;
+        exact_list[eu++] = int16_t(w * 32 + bit);
+      }
+      while (a) {
+        const int bit = __ffs(a) - 1;
+        a &= a - 1;
+        approx_list[ea++] = int16_t(w * 32 + bit);
+      }
+      ne += __shfl_sync(0xffffffffu, xu, 31);
+      na += __shfl_sync(0xffffffffu, xa, 31);
+    }
+    if (lane == 0) {
+      chunk_off[nC] = na;
+      misc[2] = ne;
+      misc[3] = na;
+    }
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = uint32_t(misc[0]);
+  const int n_exact = misc[2];
+  const int n_approx = misc[3];
+
+  if (warp == 0) {
+    // ----------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int item = 0;
+      bool ok = true;
+      for (int e = 0; e < n_exact && ok; ++e) {
+        const int j = exact_list[e];
+        for (int kv = 0; kv < 2; ++kv, ++item) {
+          const int s = item % C::NS;
+          if (!(ok = wait_bounded(BAR(C::B_EMPTY + s), ((item / C::NS) & 1) ^ 1, abort_flag))) break;
+          const uint32_t dst = base_u + C::OFF_RING + s * C::STAGE;
+          mbar_arrive_expect_tx(BAR(C::B_FULL + s), BLK * D * 2);
+#pragma unroll
+          for (int pn = 0; pn < D / 64; ++pn)
+            tma_load_3d(dst + pn * BLK * 128, kv ? &tmV : &tmK, BAR(C::B_FULL + s), pn * 64, j * BLK, bh);
+        }
+      }
+      if (p.order == 1) {
+        for (int a = 0; a < n_approx && ok; ++a, ++item) {
+          const int j = approx_list[a];
+          const int s = item % C::NS;
+          if (!(ok = wait_bounded(BAR(C::B_EMPTY + s), ((item / C::NS) & 1) ^ 1, abort_flag))) break;
+          const uint32_t dst = base_u + C::OFF_RING + s * C::STAGE;
+          mbar_arrive_expect_tx(BAR(C::B_FULL + s), D * D * 2);
+#pragma unroll
+          for (int pn = 0; pn < D / 64; ++pn)
+            tma_load_3d(dst + pn * D * 128, &tmS1, BAR(C::B_FULL + s), pn * 64, 0, bh * nB + j);
+        }
+      }
+      // no copy may still be in flight when the CTA exits
+      for (int it = item > C::NS ? item - C::NS : 0; it < item; ++it)
+        wait_drain(BAR(C::B_FULL + it % C::NS), (it / C::NS) & 1);
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(128, BLK, false);  // S = Q K^T
+      constexpr uint32_t idSB = idesc_bf16(128, 64, false);  // Sbar = Q Kbar^T
+      constexpr uint32_t idO = idesc_bf16(128, D, true);     // O += {P V, alpha S0, A S1}
+      uint32_t o_acc = 0;
+      bool ok = wait_bounded(BAR(C::B_Q), 0, abort_flag);
+      tc_fence_after();
+      auto pv = [&](int e) -> bool {
+        const int b = e & 1;
+        if (!wait_bounded(BAR(C::B_PF + b), (e >> 1) & 1, abort_flag)) return false;
+        const int it = 2 * e + 1, s = it % C::NS;
+        if (!wait_bounded(BAR(C::B_FULL + s), (it / C::NS) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t vb = base_u + C::OFF_RING + s * C::STAGE;
+#pragma unroll
+        for (int k = 0; k < BLK / 16; ++k)
+          umma_ts(tmem + C::O_COL, tmem + C::R_COL + b * BLK + k * 8,
+                  sdesc_sw128(vb + k * 2048, BLK * 128, 1024), idO, (o_acc | uint32_t(k)) ? 1u : 0u);
+        o_acc = 1;
+        umma_commit(BAR(C::B_EMPTY + s));
+        umma_commit(BAR(C::B_PV + b));
+        return true;
+      };
+      for (int e = 0; e < n_exact && ok; ++e) {
+        const int b = e & 1;
+        if (e >= 2 && !(ok = wait_bounded(BAR(C::B_PV + b), ((e - 2) >> 1) & 1, abort_flag))) break;
+        const int it = 2 * e, s = it % C::NS;
+        if (!(ok = wait_bounded(BAR(C::B_FULL + s), (it / C::NS) & 1, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t kb = base_u + C::OFF_RING + s * C::STAGE;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k)
+          umma_ts(tmem + C::R_COL + b * BLK, tmem + C::Q_COL + k * 8,
+                  sdesc_sw128(kb + (k >> 2) * (BLK * 128) + (k & 3) * 32, 16, 1024), idS, k ? 1u : 0u);
+        umma_commit(BAR(C::B_EMPTY + s));
+        umma_commit(BAR(C::B_SF + b));
+        if (e >= 1) ok = pv(e - 1);
+      }
+      if (ok && n_exact > 0) ok = pv(n_exact - 1);
+      umma_commit(BAR(C::B_OSYNC));  // completion 0: end of the exact stage
+
+      if (ok && n_approx > 0) {
+        // the pooled-score buffers reuse the exact score buffers
+        ok = wait_bounded(BAR(C::B_PV + ((n_exact - 1) & 1)), ((n_exact - 1) >> 1) & 1, abort_flag);
+        auto sbar = [&](int c) -> bool {
+          const int b = c & 1;
+          if (!wait_bounded(BAR(C::B_CVF + b), (c >> 1) & 1, abort_flag)) return false;
+          if (c >= 2 && !wait_bounded(BAR(C::B_SBE + b), ((c - 2) >> 1) & 1, abort_flag)) return false;
+          tc_fence_after();
+          const uint32_t kb = base_u + C::OFF_CV + b * C::CV_STAGE;
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k)
+            umma_ts(tmem + C::R_COL + b * 64, tmem + C::Q_COL + k * 8,
+                    sdesc_sw128(kb + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024), idSB, k ? 1u : 0u);
+          umma_commit(BAR(C::B_SBF + b));
+          return true;
+        };
+        if (ok) ok = sbar(0);
+        int a = 0;
+        for (int c = 0; c < nC && ok; ++c) {
+          const int b = c & 1;
+          if (!(ok = wait_bounded(BAR(C::B_A0F + b), (c >> 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          const uint32_t sb = base_u + C::OFF_CV + b * C::CV_STAGE + C::CV_HALF;
+#pragma unroll
+          for (int k = 0; k < C::CHUNK / 16; ++k)
+            umma_ts(tmem + C::O_COL, tmem + C::R_COL + b * 64 + k * 8, sdesc_sw128(sb + k * 2048, 8192, 1024), idO,
+                    (o_acc | uint32_t(k)) ? 1u : 0u);
+          o_acc = 1;
+          umma_commit(BAR(C::B_SBE + b));
+          umma_commit(BAR(C::B_CVE + b));
+          if (c + 1 < nC && !(ok = sbar(c + 1))) break;
+          if (p.order == 1) {
+            const int a_end = chunk_off[c + 1];
+            for (; a < a_end; ++a) {
+              const int slot = a % C::NA;
+              if (!(ok = wait_bounded(BAR(C::B_AF + slot), (a / C::NA) & 1, abort_flag))) break;
+              const int it = 2 * n_exact + a, s = it % C::NS;
+              if (!(ok = wait_bounded(BAR(C::B_FULL + s), (it / C::NS) & 1, abort_flag))) break;
+              tc_fence_after();
+              const uint32_t s1 = base_u + C::OFF_RING + s * C::STAGE;
+#pragma unroll
+              for (int k = 0; k < D / 16; ++k)
+                umma_ts(tmem + C::O_COL, tmem + C::A_COL0 + slot * C::A_COLS + k * 8,
+                        sdesc_sw128(s1 + k * 2048, D * 128, 1024), idO, 1u);
+              umma_commit(BAR(C::B_EMPTY + s));
+              umma_commit(BAR(C::B_AE + slot));
+            }
+          }
+          umma_commit(BAR(C::B_OSYNC));  // completion c + 1: end of chunk c
+        }
+      }
+      umma_commit(BAR(C::B_ODONE));
+      wait_drain(BAR(C::B_ODONE), 0);  // nothing of ours may run on after the CTA frees TMEM
+    }
+  } else if (warp < 4) {
+    // ----------------------------------------------------------- kbar / S0 converter
+    if (n_approx > 0) {
+      const int ct = threadIdx.x - 64;
+      for (int c = 0; c < nC; ++c) {
+        const int s = c & 1;
+        if (!wait_bounded(BAR(C::B_CVE + s), ((c >> 1) & 1) ^ 1, abort_flag)) break;
+        uint8_t* dk = base + C::OFF_CV + s * C::CV_STAGE;
+        uint8_t* ds = dk + C::CV_HALF;
+        const float* gk = p.kbar + (size_t(bh) * nB + size_t(c) * C::CHUNK) * D;
+        const float* gs = p.S0 + (size_t(bh) * nB + size_t(c) * C::CHUNK) * D;
+        // [64 blocks][D] row-major, 128-byte rows per 64-column panel, 16-byte
+        // chunks swizzled by (row % 8): the K-major (kbar) and MN-major (S0) UMMA
+        // operand layouts coincide for this row = block, column = d storage
+        for (int q = ct; q < C::CHUNK * (D / 8); q += 64) {
+          const int r = q / (D / 8), c16 = q % (D / 8);
+          uint4 kv = make_uint4(0, 0, 0, 0), sv = make_uint4(0, 0, 0, 0);
+          if (c * C::CHUNK + r < nB) {
+            const float4 k0 = __ldg(reinterpret_cast<const float4*>(gk + r * D + c16 * 8));
+            const float4 k1 = __ldg(reinterpret_cast<const float4*>(gk + r * D + c16 * 8 + 4));
+            const float4 s0 = __ldg(reinterpret_cast<const float4*>(gs + r * D + c16 * 8));
+            const float4 s1 = __ldg(reinterpret_cast<const float4*>(gs + r * D + c16 * 8 + 4));
+            kv = make_uint4(pack_bf16x2(k0.x, k0.y), pack_bf16x2(k0.z, k0.w), pack_bf16x2(k1.x, k1.y),
+                            pack_bf16x2(k1.z, k1.w));
+            sv = make_uint4(pack_bf16x2(s0.x, s0.y), pack_bf16x2(s0.z, s0.w), pack_bf16x2(s1.x, s1.y),
+                            pack_bf16x2(s1.z, s1.w));
+          }
+          const int off = (c16 >> 3) * (C::CHUNK * 128) + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
+          *reinterpret_cast<uint4*>(dk + off) = kv;
+          *reinterpret_cast<uint4*>(ds + off) = sv;
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(BAR(C::B_CVF + s));
+      }
+    }
+  } else {
+    // ----------------------------------------------------------- row threads
+    const int r = threadIdx.x - 128;                         // row in tile = TMEM lane
+    const uint32_t lrow = uint32_t((warp & 3) * 32) << 16;   // this warp's TMEM lane quarter
+    const int grow = tile * 128 + r;
+    const bool valid = grow < N;
+    const uint32_t* mymask = (kTwo && r >= 64) ? mask + C::MAXB / 32 : mask;
+    bool ok = true;
+
+    // queries -> TMEM (the A operand of Q K^T and Q Kbar^T)
+    {
+      const uint4* src = reinterpret_cast<const uint4*>(p.Q + (size_t(bh) * N + (valid ? grow : 0)) * D);
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t t[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 v = valid ? __ldg(src + ch * 4 + i) : make_uint4(0, 0, 0, 0);
+          t[4 * i] = v.x;
+          t[4 * i + 1] = v.y;
+          t[4 * i + 2] = v.z;
+          t[4 * i + 3] = v.w;
+        }
+        tmem_st16(tmem + lrow + C::Q_COL + ch * 16, t);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(BAR(C::B_Q));
+    }
+
+    const float sl2 = p.scale * 1.4426950408889634f;  // exponents in base 2
+    float m = -INFINITY, l = 0.f;
+
+    // ------------------------------------------------ exact stage
+    for (int e = 0; e < n_exact; ++e) {
+      const int j = exact_list[e], b = e & 1;
+      const bool sel = (mymask[j >> 5] >> (j & 31)) & 1u;  // uniform per warp
+      const int nj = min(BLK, N - j * BLK);
+      ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SF + b), (e >> 1) & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t sa = tmem + lrow + C::R_COL + b * BLK;
+      uint32_t s[BLK];
+#pragma unroll
+      for (int ch = 0; ch < BLK / 16; ++ch) tmem_ld16(sa + ch * 16, *reinterpret_cast<uint32_t(*)[16]>(&s[ch * 16]));
+#pragma unroll
+      for (int ch = 0; ch < BLK / 16; ++ch) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&s[ch * 16]));
+      float mx = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < BLK; ++k) {
+        const float v = (sel && k < nj) ? __uint_as_float(s[k]) * sl2 : -INFINITY;
+        s[k] = __float_as_uint(v);
+        mx = fmaxf(mx, v);
+      }
+      const bool grow_max = mx > m + 8.f;          // false for rows that did not select j
+      const bool need_o = grow_max && m != -INFINITY;
+      if (__any_sync(0xffffffffu, need_o)) {
+        if (e >= 1) {
+          ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_PV + ((e - 1) & 1)), ((e - 1) >> 1) & 1, abort_flag));
+          if (!ok) break;
+        }
+        tc_fence_after();
+        const float f = need_o ? ex2(m - mx) : 1.f;
+        rescale_row<D>(tmem + lrow + C::O_COL, f);
+        l *= f;
+      }
+      if (grow_max) m = mx;
+      float rs = 0.f;
+#pragma unroll
+      for (int ch = 0; ch < BLK / 32; ++ch) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          // rows whose query block did not select j take no exact weight (m may
+          // still be -inf for them, so no exponential is evaluated)
+          const float p0 = sel ? ex2(__uint_as_float(s[ch * 32 + 2 * i]) - m) : 0.f;
+          const float p1 = sel ? ex2(__uint_as_float(s[ch * 32 + 2 * i + 1]) - m) : 0.f;
+          rs += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(sa + ch * 16, pk);
+      }
+      l += rs;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(BAR(C::B_PF + b));
+    }
+
+    // ------------------------------------------------ approximate stage
+    if (ok && n_approx > 0) {
+      // every exact-stage MMA is done: the operand ring may reuse their columns
+      ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_OSYNC), 0, abort_flag));
+      uint32_t q[D / 2];
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch)
+          tmem_ld16(tmem + lrow + C::Q_COL + ch * 16, *reinterpret_cast<uint32_t(*)[16]>(&q[ch * 16]));
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&q[ch * 16]));
+      }
+      const uint32_t* m1 = kTwo ? mask + C::MAXB / 32 : mask;
+      const int nlast = N - (nB - 1) * BLK;
+      int a = 0;
+      for (int c = 0; c < nC && ok; ++c) {
+        const int b = c & 1;
+        ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SBF + b), (c >> 1) & 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t sa = tmem + lrow + C::R_COL + b * 64;
+        uint32_t sv[64];
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) tmem_ld16(sa + ch * 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[ch * 16]));
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&sv[ch * 16]));
+        const int w0 = 2 * c, w1 = 2 * c + 1;
+        const uint32_t my0 = mymask[w0], my1 = w1 < nW ? mymask[w1] : 0xffffffffu;
+        const int kmax = nB - c * C::CHUNK;  // blocks of this chunk that exist
+        float mx = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < 64; ++k) {
+          const bool mine = k < kmax && !(((k < 32 ? my0 >> k : my1 >> (k - 32)) & 1u));
+          const float v = mine ? __uint_as_float(sv[k]) * sl2 : -INFINITY;
+          sv[k] = __float_as_uint(v);
+          mx = fmaxf(mx, v);
+        }
+        const bool need_o = mx > m + 8.f;
+        if (__any_sync(0xffffffffu, need_o)) {
+          ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_OSYNC), c & 1, abort_flag));
+          if (!ok) break;
+          tc_fence_after();
+          const float f = need_o ? ex2(m - mx) : 1.f;
+          rescale_row<D>(tmem + lrow + C::O_COL, f);
+          l *= f;
+          if (need_o) m = mx;
+        }
+        float ls = 0.f;
+        uint32_t a0[32];
+#pragma unroll
+        for (int k = 0; k < 64; k += 2) {
+          const float x0 = ex2(__uint_as_float(sv[k]) - m);
+          const float x1 = ex2(__uint_as_float(sv[k + 1]) - m);
+          sv[k] = __float_as_uint(x0);
+          sv[k + 1] = __float_as_uint(x1);
+          const float n0 = (c * C::CHUNK + k == nB - 1) ? float(nlast) : float(BLK);
+          const float n1 = (c * C::CHUNK + k + 1 == nB - 1) ? float(nlast) : float(BLK);
+          ls = fmaf(n0, x0, ls);
+          ls = fmaf(n1, x1, ls);
+          a0[k >> 1] = pack_bf16x2(x0, x1);
+        }
+        l += ls;
+        tmem_st16(sa, *reinterpret_cast<uint32_t(*)[16]>(&a0[0]));
+        tmem_st16(sa + 16, *reinterpret_cast<uint32_t(*)[16]>(&a0[16]));
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(BAR(C::B_A0F + b));
+
+        if (p.order == 1) {
+          // blocks of this chunk that some row of the tile approximates (CTA-uniform)
+          const uint32_t am0 = ~(mask[w0] & m1[w0]);
+          const uint32_t am1 = w1 < nW ? ~(mask[w1] & m1[w1]) : 0u;
+#pragma unroll
+          for (int k = 0; k < 64; ++k) {
+            const bool listed = k < kmax && (((k < 32 ? am0 >> k : am1 >> (k - 32)) & 1u));
+            if (!listed) continue;
+            const int slot = a % C::NA;
+            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_AE + slot), ((a / C::NA) & 1) ^ 1, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            const float coef = __uint_as_float(sv[k]) * p.scale;  // zero where the row's block is exact
+            const __nv_bfloat162 c2 = __floats2bfloat162_rn(coef, coef);
+            const uint32_t cw = *reinterpret_cast<const uint32_t*>(&c2);
+            const uint32_t aa = tmem + lrow + C::A_COL0 + slot * C::A_COLS;
+#pragma unroll
+            for (int ch = 0; ch < D / 32; ++ch) {
+              uint32_t t[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) t[i] = hmul2_bf16(q[ch * 16 + i], cw);
+              tmem_st16(aa + ch * 16, t);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(BAR(C::B_AF + slot));
+            ++a;
+          }
+        }
+      }
+    }
+
+    // ------------------------------------------------ epilogue
+    if (ok) {
+      ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_ODONE), 0, abort_flag));
+      if (ok) {
+        tc_fence_after();
+        const float inv = 1.f / l;
+        bf16* dst = p.O + (size_t(bh) * N + (valid ? grow : 0)) * D;
+#pragma unroll
+        for (int ch = 0; ch < D / 16; ++ch) {
+          uint32_t o[16];
+          tmem_ld16(tmem + lrow + C::O_COL + ch * 16, o);
+          tmem_wait_ld(o);
+          uint4 w0, w1;
+          w0.x = pack_bf16x2(__uint_as_float(o[0]) * inv, __uint_as_float(o[1]) * inv);
+          w0.y = pack_bf16x2(__uint_as_float(o[2]) * inv, __uint_as_float(o[3]) * inv);
+          w0.z = pack_bf16x2(__uint_as_float(o[4]) * inv, __uint_as_float(o[5]) * inv);
+          w0.w = pack_bf16x2(__uint_as_float(o[6]) * inv, __uint_as_float(o[7]) * inv);
+          w1.x = pack_bf16x2(__uint_as_float(o[8]) * inv, __uint_as_float(o[9]) * inv);
+          w1.y = pack_bf16x2(__uint_as_float(o[10]) * inv, __uint_as_float(o[11]) * inv);
+          w1.z = pack_bf16x2(__uint_as_float(o[12]) * inv, __uint_as_float(o[13]) * inv);
+          w1.w = pack_bf16x2(__uint_as_float(o[14]) * inv, __uint_as_float(o[15]) * inv);
+          if (valid) {
+            reinterpret_cast<uint4*>(dst + ch * 16)[0] = w0;
+            reinterpret_cast<uint4*>(dst + ch * 16)[1] = w1;
+          }
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------- teardown
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+#undef BAR
+}
+
+}  // namespace pisa

@@ -6,6 +6,8 @@
 #include <mutex>
 #include <string>
 
+#include <cudaTypedefs.h>
+
 #include "../../include/pisa.h"
 #include "common.cuh"
 #include "stats.cuh"
@@ -161,6 +163,56 @@ pisa_status_t launch_attention_simt(const pisa_shape_t& s, const bf16* Q, const 
   return check_launch("attention_simt_kernel");
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link)
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// 3-D bf16 tensor [d2][d1][d0] (d0 innermost), box {64, box1, 1}, 128-byte swizzle,
+// out-of-range rows read as zero
+pisa_status_t make_map(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box1) {
+  auto fn = encode_fn();
+  if (!fn) return fail(PISA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {64, box1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PISA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return ok();
+}
+
+template <int D, int BLK>
+pisa_status_t launch_attention_tc(const pisa_shape_t& s, const bf16* Q, const bf16* K, const bf16* V,
+                                  const float* kbar, const float* S0, const bf16* S1, const int32_t* idx, int topk,
+                                  int order, float scale, bf16* O, cudaStream_t st) {
+  using C = pisa::TcCfg<D, BLK>;
+  const int nB = int(num_blocks(s));
+  const uint64_t BH = uint64_t(s.B) * s.H;
+  CUtensorMap mK, mV, mS1;
+  PISA_TRY(make_map(&mK, K, D, uint64_t(s.N), BH, BLK));
+  PISA_TRY(make_map(&mV, V, D, uint64_t(s.N), BH, BLK));
+  if (order == 1) PISA_TRY(make_map(&mS1, S1, D, D, BH * nB, D));
+  else mS1 = mK;  // never read at order 0
+  auto k = pisa::attention_tc_kernel<D, BLK>;
+  PISA_TRY(set_smem(k, C::SMEM));
+  pisa::TcParams p{Q, kbar, S0, idx, O, s.N, nB, topk, order, scale};
+  dim3 grid((s.N + 127) / 128, unsigned(BH));
+  k<<<grid, C::kThreads, C::SMEM, st>>>(mK, mV, mS1, p);
+  return check_launch("attention_tc_kernel");
+}
+
 struct AttnArgs {
   const void* Q;
   const void* K;
@@ -254,8 +306,13 @@ pisa_status_t pisa_attention(const void* Q, const void* K, const void* V, const 
   auto v = static_cast<const bf16*>(V);
   auto s1 = static_cast<const bf16*>(S1);
   auto o = static_cast<bf16*>(O);
-  if (shape.d == 128) return launch_attention_simt<128>(shape, q, k, v, kbar, S0, s1, idx, topk, order, scale, o, st);
-  return launch_attention_simt<64>(shape, q, k, v, kbar, S0, s1, idx, topk, order, scale, o, st);
+  if (shape.d == 128 && shape.block == 64)
+    return launch_attention_tc<128, 64>(shape, q, k, v, kbar, S0, s1, idx, topk, order, scale, o, st);
+  if (shape.d == 128 && shape.block == 128)
+    return launch_attention_tc<128, 128>(shape, q, k, v, kbar, S0, s1, idx, topk, order, scale, o, st);
+  if (shape.d == 64 && shape.block == 64)
+    return launch_attention_tc<64, 64>(shape, q, k, v, kbar, S0, s1, idx, topk, order, scale, o, st);
+  return launch_attention_tc<64, 128>(shape, q, k, v, kbar, S0, s1, idx, topk, order, scale, o, st);
 }
 
 pisa_status_t pisa_attention_simt(const void* Q, const void* K, const void* V, const float* kbar,
