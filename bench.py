@@ -176,10 +176,12 @@ def run_reference(args):
     ws, rank, _ = _dist()
     if rank != 0:
         return 0
-    wl = W.get(args.workload)
+    wl = _workload(args)
     per_step = []
+    # the whole reference run is kept to about 150 s of oracle work
+    budget = max(0.5, min(args.ref_budget, 150.0 / (args.warmup + args.steps)))
     for i in range(args.warmup + args.steps):
-        tf, secs, desc, thr = oracle_sample(wl, budget_s=args.ref_budget, min_blocks=1)
+        tf, secs, desc, thr = oracle_sample(wl, budget_s=budget, min_blocks=1)
         if i >= args.warmup:
             per_step.append((tf, secs))
     tf = statistics.mean(t for t, _ in per_step)
@@ -195,6 +197,42 @@ def run_reference(args):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def rank_batch_offset(wl, rank: int) -> int:
+    """Each rank draws its own batch (weak scaling: heads and batches are independent)."""
+    return rank * wl.B
+
+
+def max_over_ranks(value: float, pg, device) -> float:
+    """The job's time is the slowest rank's time."""
+    import torch
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    if pg is not None:
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(flops_per_rank_step: float, world: int, ms_per_step: float) -> float:
+    """Whole-job TFLOP/s: the work of every rank over the slowest rank's step time."""
+    return flops_per_rank_step * world / (ms_per_step * 1e-3) / 1e12
+
+
+def _captured_traffic(wl):
+    """DRAM bytes per attention launch from the committed ncu capture, or None when the
+    kernel sources changed since that capture (or the workload is not the captured one)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "attention_tc_traffic.json")
+    if not os.path.exists(path) or wl.name != "video" or wl.H != W.get("video").H:
+        return None
+    d = json.load(open(path))
+    h = hashlib.sha256(b"".join(open(os.path.join(ROOT, s), "rb").read() for s in d["sources"])).hexdigest()
+    return d["dram_bytes_per_full_launch"] if h == d["sources_sha256"] else None
+
+
+def _workload(args):
+    wl = W.get(args.workload)
+    return wl.with_(H=args.heads) if args.heads else wl
 
 
 def _config(wl, ws):
@@ -221,8 +259,8 @@ def run_ours(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         pg = dist
-    wl = W.get(args.workload)
-    q, k, v = W.make_inputs(wl, batch_offset=rank * wl.B)
+    wl = _workload(args)
+    q, k, v = W.make_inputs(wl, batch_offset=rank_batch_offset(wl, rank))
     to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
     Q, K, V = to_dev(q), to_dev(k), to_dev(v)
     nB = wl.nB
@@ -267,17 +305,13 @@ def run_ours(args):
         pg.barrier()
     clocks = sampler.stop() if sampler else None
     P.device_error()
-    ms_total = start.elapsed_time(end)
-    t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-    if pg:
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-    ms_total = float(t.item())
+    ms_total = max_over_ranks(start.elapsed_time(end), pg, dev)
     ms_step = ms_total / args.steps
     k_ms = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
             for i, n in enumerate(("stats", "select", "attention"))}
 
     flops_step = R.step_flops(wl.B, wl.H, wl.N, wl.d, wl.block, wl.topk, wl.order)
-    value = flops_step * ws / (ms_step * 1e-3) / 1e12
+    value = job_throughput(flops_step, ws, ms_step)
     att_flops = R.attention_flops(wl.B, wl.H, wl.N, wl.d, wl.block, wl.topk, wl.order)
     att_tf = att_flops / (k_ms["attention"] * 1e-3) / 1e12
     dense_tf = R.dense_flops(wl.B, wl.H, wl.N, wl.d) / (k_ms["attention"] * 1e-3) / 1e12
@@ -305,13 +339,9 @@ def run_ours(args):
         e1.record(stream)
         torch.cuda.synchronize()
         wall = (time.perf_counter() - t0) * 1e3 / n_e2e
-        ms_e2e = max(e0.elapsed_time(e1) / n_e2e, wall)
-        te = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
-        if pg:
-            pg.all_reduce(te, op=pg.ReduceOp.MAX)
-        ms_e2e = float(te.item())
+        ms_e2e = max_over_ranks(max(e0.elapsed_time(e1) / n_e2e, wall), pg, dev)
         nbytes = 3 * Q.numel() * 2
-        e2e = {"value": flops_step * ws / (ms_e2e * 1e-3) / 1e12, "unit": UNIT,
+        e2e = {"value": job_throughput(flops_step, ws, ms_e2e), "unit": UNIT,
                "ms_per_step": ms_e2e, "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": O.numel() * 2}
 
     cpu = None
@@ -330,7 +360,9 @@ def run_ours(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": _config(wl, ws),
         "roofline": {"bound": "tensor", "kernel": "attention", "achieved": att_tf, "peak": peak,
-                     "unit": "TFLOP/s", "frac": att_tf / peak, "traffic": args.traffic,
+                     "unit": "TFLOP/s", "frac": att_tf / peak,
+                     "traffic": args.traffic if args.traffic is not None else _captured_traffic(wl),
+                     "algorithmic_bytes_per_launch": R.attention_bytes(wl.B, wl.H, wl.N, wl.d, wl.block, wl.topk, wl.order),
                      "peak_source": f"{pk['source']} bf16 sustained",
                      "algorithmic_flops_per_launch": att_flops},
         "kernels_ms": k_ms,
@@ -356,6 +388,7 @@ def main(argv=None):
     ap.add_argument("--ref-budget", type=float, default=15.0, help="seconds of oracle work per sample")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per attention launch from an ncu capture of the current kernel")
+    ap.add_argument("--heads", type=int, default=None, help="override the workload's head count")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

@@ -1,0 +1,31 @@
+"""Algorithmic work counts used by the benchmark's roofline (CPU)."""
+import pytest
+
+from block_sparse_attention_pisa_b200 import roofline as R
+
+
+def test_video_attention_flops():
+    # N=32768, H=24, d=128, b=64, k=64 of 512, order 1: 1.649 exact + 0.180 order-0 +
+    # 11.545 order-1 TFLOP
+    exact = 24 * 32768 * 4 * 64 * 128 * 64
+    zero = 24 * 32768 * 4 * 128 * 448
+    first = 24 * 32768 * 2 * 128 * 128 * 448
+    assert R.attention_flops(1, 24, 32768, 128, 64, 64, 1) == pytest.approx(exact + zero + first)
+    assert R.attention_flops(1, 24, 32768, 128, 64, 64, 1) / 1e12 == pytest.approx(13.37, abs=0.01)
+    assert R.attention_flops(1, 24, 32768, 128, 64, 64, 0) == pytest.approx(exact + zero)
+
+
+def test_all_selected_equals_dense():
+    assert R.attention_flops(1, 16, 16384, 64, 128, 128, 1) == pytest.approx(R.dense_flops(1, 16, 16384, 64))
+
+
+def test_stats_and_select_bytes():
+    # K, V read (2 x 201 MB) + kbar, S0 (2 x 6.3 MB) + S1 (403 MB) = 818 MB
+    assert R.stats_bytes(1, 24, 32768, 128, 64, 1) / 1e6 == pytest.approx(818.0, abs=1.0)
+    assert R.select_bytes(1, 24, 32768, 128, 64, 64) / 1e6 == pytest.approx(211.0, abs=1.0)
+
+
+def test_ragged_counts_real_tokens():
+    # long workload: 75600 tokens in 591 blocks of <= 128
+    f = R.attention_flops(1, 40, 75600, 128, 128, 60, 1)
+    assert f / 1e12 == pytest.approx(65.33, abs=0.05)
