@@ -588,18 +588,20 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         mbar_arrive(BAR(C::B_A0F + b));
 
         if (p.order == 1) {
-          // blocks of this chunk that some row of the tile approximates (CTA-uniform)
-          const uint32_t am0 = ~(mask[w0] & m1[w0]);
-          const uint32_t am1 = w1 < nW ? ~(mask[w1] & m1[w1]) : 0u;
-#pragma unroll
-          for (int k = 0; k < 64; ++k) {
-            const bool listed = k < kmax && (((k < 32 ? am0 >> k : am1 >> (k - 32)) & 1u));
-            if (!listed) continue;
+          // One runtime iteration per block of this chunk that some row of the tile
+          // approximates (kept rolled: an unrolled copy of this loop is large enough to
+          // evict the MMA-issuing warp's instructions). The row's alpha comes from the
+          // packed bf16 operand a0 (zero where the row's own block is exact).
+          const int a_end = chunk_off[c + 1];
+#pragma unroll 1
+          for (; a < a_end; ++a) {
+            const int k = approx_list[a] - c * C::CHUNK;
             const int slot = a % C::NA;
             ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_AE + slot), ((a / C::NA) & 1) ^ 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            const float coef = __uint_as_float(sv[k]) * p.scale;  // zero where the row's block is exact
+            const uint32_t w = a0[k >> 1];
+            const float coef = ((k & 1) ? bf16_hi(w) : bf16_lo(w)) * p.scale;
             const __nv_bfloat162 c2 = __floats2bfloat162_rn(coef, coef);
             const uint32_t cw = *reinterpret_cast<const uint32_t*>(&c2);
             const uint32_t aa = tmem + lrow + C::A_COL0 + slot * C::A_COLS;
@@ -613,7 +615,6 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(BAR(C::B_AF + slot));
-            ++a;
           }
         }
       }
