@@ -11,30 +11,38 @@
 //
 // One CTA computes a tile of 128 query rows of one head (two query blocks at
 // b = 64, one at b = 128). Warp roles:
-//   warp 0      TMA producer: K_j, V_j of the exact blocks, then S1_j of the
-//               approximated blocks, through a ring of 32 KB shared-memory stages;
-//   warp 1      MMA issuer (one thread): all tcgen05.mma of the tile;
-//   warps 2-3   build the block lists, then convert fp32 kbar / S0 chunks of 64
+//   warp 0      TMA producer: K_j and V_j of the exact blocks, then S1_j of the
+//               approximated blocks, through a ring of shared-memory stages;
+//   warp 1      MMA issuer (one thread): every tcgen05.mma of the tile;
+//   warps 2-3   build the block lists, then convert fp32 kbar / S0 chunks of 32
 //               blocks into bf16 swizzled shared-memory operands;
 //   warps 4-7   one thread per query row (= TMEM lane): online softmax, the
 //               Taylor weights and the tensor-memory operands.
-// Tensor memory (512 columns): O accumulator (D cols), the tile's queries Q as
-// the A operand of QK^T and Q kbar^T (D/2 cols), then either the two exact
-// score buffers S (P overwrites its own S) or, in the approximate stage, two
-// pooled-score buffers Sbar (the bf16 alpha operand overwrites its own Sbar)
-// and a ring of three A_j = (alpha_j * scale) (.) q operands.
+// Tensor memory (512 columns): O accumulator (D), the tile's queries Q (D/2; the A
+// operand of Q K^T and Q Kbar^T), then either a ring of exact score buffers S
+// (P overwrites its own S) or, in the approximate stage, two pooled-score buffers
+// Sbar (the bf16 alpha operand overwrites its own Sbar) and four A_j =
+// (alpha_j * scale) (.) q operand slots used in pairs.
 //
 // Exact stage, per block j in the union of the tile's selections:
 //   S = Q K_j^T (TS-MMA), P = exp(x.k - m) (zero for rows whose query block
 //   did not select j and for keys past N), O += P V_j (TS-MMA, V MN-major).
-// Approximate stage, per chunk of 64 key blocks:
+// Approximate stage, per chunk of 32 key blocks that some row approximates:
 //   Sbar = Q Kbar_c^T, alpha = exp(x.kbar - m) (zero for blocks a row's own
-//   query block selected), O += alpha S0_c (one MMA for the zeroth order), and
-//   for every block j of the chunk that some row approximates, O += A_j S1_j
-//   (TS-MMA, S1 MN-major): the first-order term as one long-K GEMM.
-// Denominator: sum of P plus sum n_j alpha_j, kept in fp32 registers.
-// One running row maximum covers both stages; the accumulator is rescaled only
-// when the maximum grows by more than 2^8 (exact by construction, rare).
+//   query block selected), O += alpha S0_c (zeroth order), and, two blocks per
+//   hand-off, O += A_j S1_j (TS-MMA, S1 MN-major): the first-order term as one
+//   long-K GEMM.
+// Denominator: sum of P plus sum n_j alpha_j, kept in fp32 registers. One running
+// row maximum covers both stages; the accumulator is rescaled only when the
+// maximum grows by more than 2^8 (exact by construction, rare).
+//
+// Synchronisation: the MMA thread polls its barriers with the non-suspending
+// mbarrier probe, and waits once per exact block (K_j and V_j land on one
+// barrier) and once per pair of approximated blocks (both S1 tiles on one
+// barrier, both A operands on another): every wait it makes costs tensor-pipe
+// time, so there are few of them. Every wait is bounded by clock64; on timeout a
+// CTA raises the device error word, drains its copies and MMAs, frees TMEM and
+// exits.
 #pragma once
 
 #include "tc_ptx.cuh"
@@ -57,38 +65,56 @@ struct TcParams {
 template <int D, int BLK>
 struct TcCfg {
   static constexpr int kThreads = 256;
-  static constexpr int NS = (D == 128) ? 4 : 8;             // TMA ring stages
+  static constexpr int NS = (D == 128) ? 5 : 10;            // TMA stages
   static constexpr int STAGE = (D == 128) ? 32768 : 16384;  // bytes per stage
-  static constexpr int CHUNK = 64;                          // key blocks per approximate chunk
+  static constexpr int NTF = NS;                            // landed-copy barriers (one per load unit)
+  static constexpr int CHUNK = 32;                          // key blocks per approximate chunk
   static constexpr int CV_HALF = CHUNK * D * 2;             // bf16 kbar (or S0) chunk
   static constexpr int CV_STAGE = 2 * CV_HALF;
-  static constexpr int NA = 3;                              // A_j ring depth
+  static constexpr int GROUP = 2;                           // approximated blocks per hand-off
+  static constexpr int NA = 2 * GROUP;                      // A operand slots (two groups)
+  static constexpr int NSB = (BLK == 64) ? 4 : 2;           // exact score buffers
   static constexpr int MAXB = 2048;
+  static constexpr int MAXC = MAXB / CHUNK;
   // tensor-memory columns
   static constexpr int O_COL = 0;
   static constexpr int Q_COL = D;
   static constexpr int R_COL = D + D / 2;
-  static constexpr int A_COL0 = R_COL + 128;
+  static constexpr int A_COL0 = R_COL + 2 * CHUNK;
   static constexpr int A_COLS = D / 2;
   static constexpr int TMEM_COLS = 512;
-  static_assert(R_COL + 2 * BLK <= TMEM_COLS, "exact score buffers exceed TMEM");
+  static_assert(R_COL + NSB * BLK <= TMEM_COLS, "exact score buffers exceed TMEM");
   static_assert(A_COL0 + NA * A_COLS <= TMEM_COLS, "operand ring exceeds TMEM");
   static_assert(STAGE >= BLK * D * 2 && STAGE >= D * D * 2, "stage too small");
   // barriers
-  static constexpr int B_FULL = 0, B_EMPTY = NS, B_CVF = 2 * NS, B_CVE = B_CVF + 2, B_Q = B_CVE + 2;
-  static constexpr int B_SF = B_Q + 1, B_PF = B_SF + 2, B_PV = B_PF + 2, B_SBF = B_PV + 2;
-  static constexpr int B_A0F = B_SBF + 2, B_SBE = B_A0F + 2, B_AF = B_SBE + 2, B_AE = B_AF + NA;
-  static constexpr int B_OSYNC = B_AE + NA, B_ODONE = B_OSYNC + 1, NBARS = B_ODONE + 1;
+  static constexpr int B_SE = 0;                  // [NS]  stage consumed (MMA commit)
+  static constexpr int B_TF = B_SE + NS;          // [NTF] copies of a load unit landed
+  static constexpr int B_Q = B_TF + NTF;          //       queries in TMEM (128 rows)
+  static constexpr int B_SF = B_Q + 1;            // [NSB] S ready (commit)
+  static constexpr int B_PF = B_SF + NSB;         // [NSB] P written (128 rows)
+  static constexpr int B_PV = B_PF + NSB;         // [NSB] P V done (commit)
+  static constexpr int B_CVF = B_PV + NSB;        // [2]   kbar / S0 chunk converted (64)
+  static constexpr int B_CVE = B_CVF + 2;         // [2]   chunk operands consumed (commit)
+  static constexpr int B_SBF = B_CVE + 2;         // [2]   Sbar ready (commit)
+  static constexpr int B_A0F = B_SBF + 2;         // [2]   alpha operand written (128)
+  static constexpr int B_SBE = B_A0F + 2;         // [2]   alpha MMA done (commit)
+  static constexpr int B_GA = B_SBE + 2;          // [2]   a pair of A_j written (128)
+  static constexpr int B_AE = B_GA + 2;           // [2]   a pair of A_j consumed (commit)
+  static constexpr int B_OSYNC = B_AE + 2;        //       end of the exact stage / of a chunk (commit)
+  static constexpr int B_ODONE = B_OSYNC + 1;     //       all MMAs done (commit)
+  static constexpr int NBARS = B_ODONE + 1;
   // shared memory (offsets from a 1024-byte aligned base)
   static constexpr int OFF_RING = 0;
   static constexpr int OFF_CV = OFF_RING + NS * STAGE;
-  static constexpr int OFF_EXACT = OFF_CV + 2 * CV_STAGE;
-  static constexpr int OFF_APPROX = OFF_EXACT + 2 * MAXB;
-  static constexpr int OFF_CHUNK = OFF_APPROX + 2 * MAXB;
-  static constexpr int OFF_MASK = OFF_CHUNK + 4 * (MAXB / CHUNK + 1 + 3);
+  static constexpr int OFF_EXACT = OFF_CV + 2 * CV_STAGE;   // int16[MAXB]
+  static constexpr int OFF_APPROX = OFF_EXACT + 2 * MAXB;   // int16[MAXB]
+  static constexpr int OFF_ACTIVE = OFF_APPROX + 2 * MAXB;  // int16[MAXC]
+  static constexpr int OFF_CHUNK = OFF_ACTIVE + 2 * MAXC;   // int32[MAXC + 1]
+  static constexpr int OFF_MASK = OFF_CHUNK + 4 * (MAXC + 4);
   static constexpr int OFF_BAR = OFF_MASK + 2 * (MAXB / 32) * 4;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
   static constexpr int SMEM = OFF_MISC + 64 + 1024;  // + alignment slack
+  static_assert(OFF_BAR % 8 == 0, "barrier alignment");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
@@ -148,9 +174,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   uint8_t* base = tc_smem_raw + (base_u - raw_u);
   int16_t* exact_list = reinterpret_cast<int16_t*>(base + C::OFF_EXACT);
   int16_t* approx_list = reinterpret_cast<int16_t*>(base + C::OFF_APPROX);
+  int16_t* active = reinterpret_cast<int16_t*>(base + C::OFF_ACTIVE);
   int* chunk_off = reinterpret_cast<int*>(base + C::OFF_CHUNK);
   uint32_t* mask = reinterpret_cast<uint32_t*>(base + C::OFF_MASK);  // [2][MAXB/32]
-  int* misc = reinterpret_cast<int*>(base + C::OFF_MISC);              // tmem, abort, n_exact, n_approx
+  int* misc = reinterpret_cast<int*>(base + C::OFF_MISC);  // tmem, abort, n_exact, n_approx, n_active
   volatile int* abort_flag = misc + 1;
   const uint32_t bar0 = base_u + C::OFF_BAR;
 #define BAR(i) (bar0 + 8u * uint32_t(i))
@@ -159,29 +186,27 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   const int tile = blockIdx.x;
   const int bh = blockIdx.y;
   const int N = p.N, nB = p.nB;
-  const int nW = (nB + 31) >> 5;
-  const int nC = (nB + C::CHUNK - 1) / C::CHUNK;
-  constexpr bool kTwo = (BLK == 64);  // two query blocks per 128-row tile
+  const int nW = (nB + 31) >> 5;  // mask words; one chunk per word (CHUNK == 32)
+  constexpr bool kTwo = (BLK == 64);
   const int i0 = kTwo ? 2 * tile : tile;
+  static_assert(C::CHUNK == 32, "chunk == mask word");
 
   // ------------------------------------------------------------- prologue
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::NS; ++s) {
-      mbar_init(BAR(C::B_FULL + s), 1);
-      mbar_init(BAR(C::B_EMPTY + s), 1);
+    for (int s = 0; s < C::NS; ++s) mbar_init(BAR(C::B_SE + s), 1);
+    for (int s = 0; s < C::NTF; ++s) mbar_init(BAR(C::B_TF + s), 1);
+    for (int s = 0; s < C::NSB; ++s) {
+      mbar_init(BAR(C::B_SF + s), 1);
+      mbar_init(BAR(C::B_PF + s), 128);
+      mbar_init(BAR(C::B_PV + s), 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(BAR(C::B_CVF + s), 64);
       mbar_init(BAR(C::B_CVE + s), 1);
-      mbar_init(BAR(C::B_SF + s), 1);
-      mbar_init(BAR(C::B_PF + s), 128);
-      mbar_init(BAR(C::B_PV + s), 1);
       mbar_init(BAR(C::B_SBF + s), 1);
       mbar_init(BAR(C::B_A0F + s), 128);
       mbar_init(BAR(C::B_SBE + s), 1);
-    }
-    for (int s = 0; s < C::NA; ++s) {
-      mbar_init(BAR(C::B_AF + s), 128);
+      mbar_init(BAR(C::B_GA + s), 128);
       mbar_init(BAR(C::B_AE + s), 1);
     }
     mbar_init(BAR(C::B_Q), 128);
@@ -215,10 +240,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     __syncwarp();
     const uint32_t* m0 = mask;
     const uint32_t* m1 = kTwo ? mask + C::MAXB / 32 : mask;
-    // exact list = union of the selections; approximate list = blocks that some
-    // row does not take exactly; both ascending; chunk_off[c] = first approximate
-    // entry of chunk c
-    int ne = 0, na = 0;
+    // exact list = union of the selections; approximate list = blocks that some row
+    // does not take exactly; active chunks = chunks holding approximate blocks;
+    // chunk_off[c] = first approximate entry of chunk c. All ascending.
+    const unsigned lt = (1u << lane) - 1u;
+    int ne = 0, na = 0, nac = 0;
     for (int wb = 0; wb < nW; wb += 32) {
       const int w = wb + lane;
       uint32_t u = 0, a = 0;
@@ -239,7 +265,9 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         }
       }
       int eu = ne + xu - pu, ea = na + xa - pa;
-      if (w < nW && (w & 1) == 0) chunk_off[w >> 1] = ea;
+      if (w < nW) chunk_off[w] = ea;
+      const unsigned act = __ballot_sync(0xffffffffu, a != 0u);
+      if (a != 0u) active[nac + __popc(act & lt)] = int16_t(w);
       while (u) {
         const int bit = __ffs(u) - 1;
         u &= u - 1;
@@ -252,144 +280,162 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       }
       ne += __shfl_sync(0xffffffffu, xu, 31);
       na += __shfl_sync(0xffffffffu, xa, 31);
+      nac += __popc(act);
     }
     if (lane == 0) {
-      chunk_off[nC] = na;
+      chunk_off[nW] = na;
       misc[2] = ne;
       misc[3] = na;
+      misc[4] = nac;
     }
   }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = uint32_t(misc[0]);
   const int n_exact = misc[2];
-  const int n_approx = misc[3];
+  const int n_active = misc[4];
 
   if (warp == 0) {
     // ----------------------------------------------------------- TMA producer
     if (lane == 0) {
-      int item = 0;
+      int t = 0, u = 0;  // tiles issued, load units issued
       bool ok = true;
-      for (int e = 0; e < n_exact && ok; ++e) {
+      for (int e = 0; e < n_exact && ok; ++e, ++u) {
         const int j = exact_list[e];
-        for (int kv = 0; kv < 2; ++kv, ++item) {
-          const int s = item % C::NS;
-          if (!(ok = wait_bounded(BAR(C::B_EMPTY + s), ((item / C::NS) & 1) ^ 1, abort_flag))) break;
-          const uint32_t dst = base_u + C::OFF_RING + s * C::STAGE;
-          mbar_arrive_expect_tx(BAR(C::B_FULL + s), BLK * D * 2);
+        for (int q = 0; q < 2 && ok; ++q)
+          ok = wait_bounded(BAR(C::B_SE + (t + q) % C::NS), (((t + q) / C::NS) & 1) ^ 1, abort_flag);
+        if (!ok) break;
+        const uint32_t tf = BAR(C::B_TF + u % C::NTF);
+        mbar_arrive_expect_tx(tf, 2 * BLK * D * 2);
+        for (int kv = 0; kv < 2; ++kv, ++t) {
+          const uint32_t dst = base_u + C::OFF_RING + (t % C::NS) * C::STAGE;
 #pragma unroll
           for (int pn = 0; pn < D / 64; ++pn)
-            tma_load_3d(dst + pn * BLK * 128, kv ? &tmV : &tmK, BAR(C::B_FULL + s), pn * 64, j * BLK, bh);
+            tma_load_3d(dst + pn * BLK * 128, kv ? &tmV : &tmK, tf, pn * 64, j * BLK, bh);
         }
       }
       if (p.order == 1) {
-        for (int a = 0; a < n_approx && ok; ++a, ++item) {
-          const int j = approx_list[a];
-          const int s = item % C::NS;
-          if (!(ok = wait_bounded(BAR(C::B_EMPTY + s), ((item / C::NS) & 1) ^ 1, abort_flag))) break;
-          const uint32_t dst = base_u + C::OFF_RING + s * C::STAGE;
-          mbar_arrive_expect_tx(BAR(C::B_FULL + s), D * D * 2);
+        for (int ac = 0; ac < n_active && ok; ++ac) {
+          const int c = active[ac];
+          const int a_end = chunk_off[c + 1];
+          for (int a = chunk_off[c]; a < a_end && ok; a += C::GROUP, ++u) {
+            const int n = min(C::GROUP, a_end - a);
+            for (int q = 0; q < n && ok; ++q)
+              ok = wait_bounded(BAR(C::B_SE + (t + q) % C::NS), (((t + q) / C::NS) & 1) ^ 1, abort_flag);
+            if (!ok) break;
+            const uint32_t tf = BAR(C::B_TF + u % C::NTF);
+            mbar_arrive_expect_tx(tf, n * D * D * 2);
+            for (int q = 0; q < n; ++q, ++t) {
+              const uint32_t dst = base_u + C::OFF_RING + (t % C::NS) * C::STAGE;
+              const int j = approx_list[a + q];
 #pragma unroll
-          for (int pn = 0; pn < D / 64; ++pn)
-            tma_load_3d(dst + pn * D * 128, &tmS1, BAR(C::B_FULL + s), pn * 64, 0, bh * nB + j);
+              for (int pn = 0; pn < D / 64; ++pn)
+                tma_load_3d(dst + pn * D * 128, &tmS1, tf, pn * 64, 0, bh * nB + j);
+            }
+          }
         }
       }
-      // no copy may still be in flight when the CTA exits
-      for (int it = item > C::NS ? item - C::NS : 0; it < item; ++it)
-        wait_drain(BAR(C::B_FULL + it % C::NS), (it / C::NS) & 1);
+      // no copy may still be in flight when the CTA exits (each load unit's barrier
+      // completes from its copies alone)
+      for (int v = u > C::NTF ? u - C::NTF : 0; v < u; ++v) wait_drain(BAR(C::B_TF + v % C::NTF), (v / C::NTF) & 1);
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(128, BLK, false);  // S = Q K^T
-      constexpr uint32_t idSB = idesc_bf16(128, 64, false);  // Sbar = Q Kbar^T
-      constexpr uint32_t idO = idesc_bf16(128, D, true);     // O += {P V, alpha S0, A S1}
+      constexpr uint32_t idS = idesc_bf16(128, BLK, false);        // S = Q K^T
+      constexpr uint32_t idSB = idesc_bf16(128, C::CHUNK, false);  // Sbar = Q Kbar^T
+      constexpr uint32_t idO = idesc_bf16(128, D, true);           // O += {P V, alpha S0, A S1}
       uint32_t o_acc = 0;
-      bool ok = wait_bounded(BAR(C::B_Q), 0, abort_flag);
+      bool ok = wait_poll(BAR(C::B_Q), 0, abort_flag);
       tc_fence_after();
       auto pv = [&](int e) -> bool {
-        const int b = e & 1;
-        if (!wait_bounded(BAR(C::B_PF + b), (e >> 1) & 1, abort_flag)) return false;
-        const int it = 2 * e + 1, s = it % C::NS;
-        if (!wait_bounded(BAR(C::B_FULL + s), (it / C::NS) & 1, abort_flag)) return false;
+        const int sb = e % C::NSB;
+        if (!wait_poll(BAR(C::B_PF + sb), (e / C::NSB) & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t vb = base_u + C::OFF_RING + s * C::STAGE;
+        const int sv = (2 * e + 1) % C::NS;
+        const uint32_t vb = base_u + C::OFF_RING + sv * C::STAGE;
 #pragma unroll
         for (int k = 0; k < BLK / 16; ++k)
-          umma_ts(tmem + C::O_COL, tmem + C::R_COL + b * BLK + k * 8,
-                  sdesc_sw128(vb + k * 2048, BLK * 128, 1024), idO, (o_acc | uint32_t(k)) ? 1u : 0u);
+          umma_ts(tmem + C::O_COL, tmem + C::R_COL + sb * BLK + k * 8, sdesc_sw128(vb + k * 2048, BLK * 128, 1024),
+                  idO, (o_acc | uint32_t(k)) ? 1u : 0u);
         o_acc = 1;
-        umma_commit(BAR(C::B_EMPTY + s));
-        umma_commit(BAR(C::B_PV + b));
+        umma_commit(BAR(C::B_SE + sv));
+        umma_commit(BAR(C::B_PV + sb));
         return true;
       };
       for (int e = 0; e < n_exact && ok; ++e) {
-        const int b = e & 1;
-        if (e >= 2 && !(ok = wait_bounded(BAR(C::B_PV + b), ((e - 2) >> 1) & 1, abort_flag))) break;
-        const int it = 2 * e, s = it % C::NS;
-        if (!(ok = wait_bounded(BAR(C::B_FULL + s), (it / C::NS) & 1, abort_flag))) break;
+        const int sb = e % C::NSB;
+        if (e >= C::NSB && !(ok = wait_poll(BAR(C::B_PV + sb), ((e - C::NSB) / C::NSB) & 1, abort_flag))) break;
+        if (!(ok = wait_poll(BAR(C::B_TF + e % C::NTF), (e / C::NTF) & 1, abort_flag))) break;
         tc_fence_after();
-        const uint32_t kb = base_u + C::OFF_RING + s * C::STAGE;
+        const int sk = (2 * e) % C::NS;
+        const uint32_t kb = base_u + C::OFF_RING + sk * C::STAGE;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          umma_ts(tmem + C::R_COL + b * BLK, tmem + C::Q_COL + k * 8,
+          umma_ts(tmem + C::R_COL + sb * BLK, tmem + C::Q_COL + k * 8,
                   sdesc_sw128(kb + (k >> 2) * (BLK * 128) + (k & 3) * 32, 16, 1024), idS, k ? 1u : 0u);
-        umma_commit(BAR(C::B_EMPTY + s));
-        umma_commit(BAR(C::B_SF + b));
+        umma_commit(BAR(C::B_SE + sk));
+        umma_commit(BAR(C::B_SF + sb));
         if (e >= 1) ok = pv(e - 1);
       }
       if (ok && n_exact > 0) ok = pv(n_exact - 1);
       umma_commit(BAR(C::B_OSYNC));  // completion 0: end of the exact stage
 
-      if (ok && n_approx > 0) {
-        // the pooled-score buffers reuse the exact score buffers
-        ok = wait_bounded(BAR(C::B_PV + ((n_exact - 1) & 1)), ((n_exact - 1) >> 1) & 1, abort_flag);
-        auto sbar = [&](int c) -> bool {
-          const int b = c & 1;
-          if (!wait_bounded(BAR(C::B_CVF + b), (c >> 1) & 1, abort_flag)) return false;
-          if (c >= 2 && !wait_bounded(BAR(C::B_SBE + b), ((c - 2) >> 1) & 1, abort_flag)) return false;
+      if (ok && n_active > 0) {
+        // the pooled-score and operand columns reuse the exact score buffers
+        ok = wait_poll(BAR(C::B_PV + (n_exact - 1) % C::NSB), ((n_exact - 1) / C::NSB) & 1, abort_flag);
+        auto sbar = [&](int ac) -> bool {
+          const int b = ac & 1;
+          if (!wait_poll(BAR(C::B_CVF + b), (ac >> 1) & 1, abort_flag)) return false;
+          if (ac >= 2 && !wait_poll(BAR(C::B_SBE + b), ((ac - 2) >> 1) & 1, abort_flag)) return false;
           tc_fence_after();
           const uint32_t kb = base_u + C::OFF_CV + b * C::CV_STAGE;
 #pragma unroll
           for (int k = 0; k < D / 16; ++k)
-            umma_ts(tmem + C::R_COL + b * 64, tmem + C::Q_COL + k * 8,
-                    sdesc_sw128(kb + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024), idSB, k ? 1u : 0u);
+            umma_ts(tmem + C::R_COL + b * C::CHUNK, tmem + C::Q_COL + k * 8,
+                    sdesc_sw128(kb + (k >> 2) * (C::CHUNK * 128) + (k & 3) * 32, 16, 1024), idSB, k ? 1u : 0u);
           umma_commit(BAR(C::B_SBF + b));
           return true;
         };
         if (ok) ok = sbar(0);
-        int a = 0;
-        for (int c = 0; c < nC && ok; ++c) {
-          const int b = c & 1;
-          if (!(ok = wait_bounded(BAR(C::B_A0F + b), (c >> 1) & 1, abort_flag))) break;
+        int g = 0;               // pair (hand-off) counter
+        int t = 2 * n_exact;     // tile counter
+        int u = n_exact;         // load-unit counter
+        for (int ac = 0; ac < n_active && ok; ++ac) {
+          const int c = active[ac];
+          const int b = ac & 1;
+          if (!(ok = wait_poll(BAR(C::B_A0F + b), (ac >> 1) & 1, abort_flag))) break;
           tc_fence_after();
           const uint32_t sb = base_u + C::OFF_CV + b * C::CV_STAGE + C::CV_HALF;
 #pragma unroll
           for (int k = 0; k < C::CHUNK / 16; ++k)
-            umma_ts(tmem + C::O_COL, tmem + C::R_COL + b * 64 + k * 8, sdesc_sw128(sb + k * 2048, 8192, 1024), idO,
-                    (o_acc | uint32_t(k)) ? 1u : 0u);
+            umma_ts(tmem + C::O_COL, tmem + C::R_COL + b * C::CHUNK + k * 8,
+                    sdesc_sw128(sb + k * 2048, C::CHUNK * 128, 1024), idO, (o_acc | uint32_t(k)) ? 1u : 0u);
           o_acc = 1;
           umma_commit(BAR(C::B_SBE + b));
           umma_commit(BAR(C::B_CVE + b));
-          if (c + 1 < nC && !(ok = sbar(c + 1))) break;
+          if (ac + 1 < n_active && !(ok = sbar(ac + 1))) break;
           if (p.order == 1) {
             const int a_end = chunk_off[c + 1];
-            for (; a < a_end; ++a) {
-              const int slot = a % C::NA;
-              if (!(ok = wait_bounded(BAR(C::B_AF + slot), (a / C::NA) & 1, abort_flag))) break;
-              const int it = 2 * n_exact + a, s = it % C::NS;
-              if (!(ok = wait_bounded(BAR(C::B_FULL + s), (it / C::NS) & 1, abort_flag))) break;
+            for (int a = chunk_off[c]; a < a_end; a += C::GROUP, ++g, ++u) {
+              const int n = min(C::GROUP, a_end - a);
+              const int gs = g & 1;
+              if (!(ok = wait_poll(BAR(C::B_GA + gs), (g >> 1) & 1, abort_flag))) break;
+              if (!(ok = wait_poll(BAR(C::B_TF + u % C::NTF), (u / C::NTF) & 1, abort_flag))) break;
               tc_fence_after();
-              const uint32_t s1 = base_u + C::OFF_RING + s * C::STAGE;
+              for (int q = 0; q < n; ++q, ++t) {
+                const int s = t % C::NS;
+                const uint32_t s1 = base_u + C::OFF_RING + s * C::STAGE;
+                const uint32_t aa = tmem + C::A_COL0 + (gs * C::GROUP + q) * C::A_COLS;
 #pragma unroll
-              for (int k = 0; k < D / 16; ++k)
-                umma_ts(tmem + C::O_COL, tmem + C::A_COL0 + slot * C::A_COLS + k * 8,
-                        sdesc_sw128(s1 + k * 2048, D * 128, 1024), idO, 1u);
-              umma_commit(BAR(C::B_EMPTY + s));
-              umma_commit(BAR(C::B_AE + slot));
+                for (int k = 0; k < D / 16; ++k)
+                  umma_ts(tmem + C::O_COL, aa + k * 8, sdesc_sw128(s1 + k * 2048, D * 128, 1024), idO, 1u);
+                umma_commit(BAR(C::B_SE + s));
+              }
+              umma_commit(BAR(C::B_AE + gs));
             }
           }
-          umma_commit(BAR(C::B_OSYNC));  // completion c + 1: end of chunk c
+          umma_commit(BAR(C::B_OSYNC));  // completion ac + 1: end of active chunk ac
         }
       }
       umma_commit(BAR(C::B_ODONE));
@@ -397,38 +443,37 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     }
   } else if (warp < 4) {
     // ----------------------------------------------------------- kbar / S0 converter
-    if (n_approx > 0) {
-      const int ct = threadIdx.x - 64;
-      for (int c = 0; c < nC; ++c) {
-        const int s = c & 1;
-        if (!wait_bounded(BAR(C::B_CVE + s), ((c >> 1) & 1) ^ 1, abort_flag)) break;
-        uint8_t* dk = base + C::OFF_CV + s * C::CV_STAGE;
-        uint8_t* ds = dk + C::CV_HALF;
-        const float* gk = p.kbar + (size_t(bh) * nB + size_t(c) * C::CHUNK) * D;
-        const float* gs = p.S0 + (size_t(bh) * nB + size_t(c) * C::CHUNK) * D;
-        // [64 blocks][D] row-major, 128-byte rows per 64-column panel, 16-byte
-        // chunks swizzled by (row % 8): the K-major (kbar) and MN-major (S0) UMMA
-        // operand layouts coincide for this row = block, column = d storage
-        for (int q = ct; q < C::CHUNK * (D / 8); q += 64) {
-          const int r = q / (D / 8), c16 = q % (D / 8);
-          uint4 kv = make_uint4(0, 0, 0, 0), sv = make_uint4(0, 0, 0, 0);
-          if (c * C::CHUNK + r < nB) {
-            const float4 k0 = __ldg(reinterpret_cast<const float4*>(gk + r * D + c16 * 8));
-            const float4 k1 = __ldg(reinterpret_cast<const float4*>(gk + r * D + c16 * 8 + 4));
-            const float4 s0 = __ldg(reinterpret_cast<const float4*>(gs + r * D + c16 * 8));
-            const float4 s1 = __ldg(reinterpret_cast<const float4*>(gs + r * D + c16 * 8 + 4));
-            kv = make_uint4(pack_bf16x2(k0.x, k0.y), pack_bf16x2(k0.z, k0.w), pack_bf16x2(k1.x, k1.y),
-                            pack_bf16x2(k1.z, k1.w));
-            sv = make_uint4(pack_bf16x2(s0.x, s0.y), pack_bf16x2(s0.z, s0.w), pack_bf16x2(s1.x, s1.y),
-                            pack_bf16x2(s1.z, s1.w));
-          }
-          const int off = (c16 >> 3) * (C::CHUNK * 128) + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
-          *reinterpret_cast<uint4*>(dk + off) = kv;
-          *reinterpret_cast<uint4*>(ds + off) = sv;
+    const int ct = threadIdx.x - 64;
+    for (int ac = 0; ac < n_active; ++ac) {
+      const int c = active[ac];
+      const int s = ac & 1;
+      if (!wait_bounded(BAR(C::B_CVE + s), ((ac >> 1) & 1) ^ 1, abort_flag)) break;
+      uint8_t* dk = base + C::OFF_CV + s * C::CV_STAGE;
+      uint8_t* ds = dk + C::CV_HALF;
+      const float* gk = p.kbar + (size_t(bh) * nB + size_t(c) * C::CHUNK) * D;
+      const float* gs = p.S0 + (size_t(bh) * nB + size_t(c) * C::CHUNK) * D;
+      // [CHUNK blocks][D] row-major, 128-byte rows per 64-column panel, 16-byte
+      // chunks swizzled by (row % 8): the K-major (kbar) and MN-major (S0) UMMA
+      // operand layouts coincide for this row = block, column = d storage
+      for (int q = ct; q < C::CHUNK * (D / 8); q += 64) {
+        const int r = q / (D / 8), c16 = q % (D / 8);
+        uint4 kv = make_uint4(0, 0, 0, 0), sv = make_uint4(0, 0, 0, 0);
+        if (c * C::CHUNK + r < nB) {
+          const float4 k0 = __ldg(reinterpret_cast<const float4*>(gk + r * D + c16 * 8));
+          const float4 k1 = __ldg(reinterpret_cast<const float4*>(gk + r * D + c16 * 8 + 4));
+          const float4 s0 = __ldg(reinterpret_cast<const float4*>(gs + r * D + c16 * 8));
+          const float4 s1 = __ldg(reinterpret_cast<const float4*>(gs + r * D + c16 * 8 + 4));
+          kv = make_uint4(pack_bf16x2(k0.x, k0.y), pack_bf16x2(k0.z, k0.w), pack_bf16x2(k1.x, k1.y),
+                          pack_bf16x2(k1.z, k1.w));
+          sv = make_uint4(pack_bf16x2(s0.x, s0.y), pack_bf16x2(s0.z, s0.w), pack_bf16x2(s1.x, s1.y),
+                          pack_bf16x2(s1.z, s1.w));
         }
-        fence_proxy_async_smem();
-        mbar_arrive(BAR(C::B_CVF + s));
+        const int off = (c16 >> 3) * (C::CHUNK * 128) + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
+        *reinterpret_cast<uint4*>(dk + off) = kv;
+        *reinterpret_cast<uint4*>(ds + off) = sv;
       }
+      fence_proxy_async_smem();
+      mbar_arrive(BAR(C::B_CVF + s));
     }
   } else {
     // ----------------------------------------------------------- row threads
@@ -465,13 +510,13 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
 
     // ------------------------------------------------ exact stage
     for (int e = 0; e < n_exact; ++e) {
-      const int j = exact_list[e], b = e & 1;
+      const int j = exact_list[e], sb = e % C::NSB;
       const bool sel = (mymask[j >> 5] >> (j & 31)) & 1u;  // uniform per warp
       const int nj = min(BLK, N - j * BLK);
-      ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SF + b), (e >> 1) & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SF + sb), (e / C::NSB) & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      const uint32_t sa = tmem + lrow + C::R_COL + b * BLK;
+      const uint32_t sa = tmem + lrow + C::R_COL + sb * BLK;
       uint32_t s[BLK];
 #pragma unroll
       for (int ch = 0; ch < BLK / 16; ++ch) tmem_ld16(sa + ch * 16, *reinterpret_cast<uint32_t(*)[16]>(&s[ch * 16]));
@@ -488,7 +533,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       const bool need_o = grow_max && m != -INFINITY;
       if (__any_sync(0xffffffffu, need_o)) {
         if (e >= 1) {
-          ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_PV + ((e - 1) & 1)), ((e - 1) >> 1) & 1, abort_flag));
+          ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_PV + (e - 1) % C::NSB), ((e - 1) / C::NSB) & 1,
+                                                    abort_flag));
           if (!ok) break;
         }
         tc_fence_after();
@@ -515,12 +561,12 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       l += rs;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(BAR(C::B_PF + b));
+      mbar_arrive(BAR(C::B_PF + sb));
     }
 
     // ------------------------------------------------ approximate stage
-    if (ok && n_approx > 0) {
-      // every exact-stage MMA is done: the operand ring may reuse their columns
+    if (ok && n_active > 0) {
+      // every exact-stage MMA is done: the operand slots may reuse their columns
       ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_OSYNC), 0, abort_flag));
       uint32_t q[D / 2];
       if (ok) {
@@ -531,34 +577,33 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
 #pragma unroll
         for (int ch = 0; ch < D / 32; ++ch) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&q[ch * 16]));
       }
-      const uint32_t* m1 = kTwo ? mask + C::MAXB / 32 : mask;
       const int nlast = N - (nB - 1) * BLK;
-      int a = 0;
-      for (int c = 0; c < nC && ok; ++c) {
-        const int b = c & 1;
-        ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SBF + b), (c >> 1) & 1, abort_flag));
+      int g = 0;
+      for (int ac = 0; ac < n_active && ok; ++ac) {
+        const int c = active[ac];
+        const int b = ac & 1;
+        ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SBF + b), (ac >> 1) & 1, abort_flag));
         if (!ok) break;
         tc_fence_after();
-        const uint32_t sa = tmem + lrow + C::R_COL + b * 64;
-        uint32_t sv[64];
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) tmem_ld16(sa + ch * 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[ch * 16]));
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&sv[ch * 16]));
-        const int w0 = 2 * c, w1 = 2 * c + 1;
-        const uint32_t my0 = mymask[w0], my1 = w1 < nW ? mymask[w1] : 0xffffffffu;
+        const uint32_t sa = tmem + lrow + C::R_COL + b * C::CHUNK;
+        uint32_t sv[C::CHUNK];
+        tmem_ld16(sa, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
+        tmem_ld16(sa + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
+        tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
+        tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
+        const uint32_t myw = mymask[c];
         const int kmax = nB - c * C::CHUNK;  // blocks of this chunk that exist
         float mx = -INFINITY;
 #pragma unroll
-        for (int k = 0; k < 64; ++k) {
-          const bool mine = k < kmax && !(((k < 32 ? my0 >> k : my1 >> (k - 32)) & 1u));
+        for (int k = 0; k < C::CHUNK; ++k) {
+          const bool mine = k < kmax && !((myw >> k) & 1u);
           const float v = mine ? __uint_as_float(sv[k]) * sl2 : -INFINITY;
           sv[k] = __float_as_uint(v);
           mx = fmaxf(mx, v);
         }
         const bool need_o = mx > m + 8.f;
         if (__any_sync(0xffffffffu, need_o)) {
-          ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_OSYNC), c & 1, abort_flag));
+          ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_OSYNC), ac & 1, abort_flag));
           if (!ok) break;
           tc_fence_after();
           const float f = need_o ? ex2(m - mx) : 1.f;
@@ -567,13 +612,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           if (need_o) m = mx;
         }
         float ls = 0.f;
-        uint32_t a0[32];
+        uint32_t a0[C::CHUNK / 2];
 #pragma unroll
-        for (int k = 0; k < 64; k += 2) {
+        for (int k = 0; k < C::CHUNK; k += 2) {
           const float x0 = ex2(__uint_as_float(sv[k]) - m);
           const float x1 = ex2(__uint_as_float(sv[k + 1]) - m);
-          sv[k] = __float_as_uint(x0);
-          sv[k + 1] = __float_as_uint(x1);
           const float n0 = (c * C::CHUNK + k == nB - 1) ? float(nlast) : float(BLK);
           const float n1 = (c * C::CHUNK + k + 1 == nB - 1) ? float(nlast) : float(BLK);
           ls = fmaf(n0, x0, ls);
@@ -581,40 +624,42 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           a0[k >> 1] = pack_bf16x2(x0, x1);
         }
         l += ls;
-        tmem_st16(sa, *reinterpret_cast<uint32_t(*)[16]>(&a0[0]));
-        tmem_st16(sa + 16, *reinterpret_cast<uint32_t(*)[16]>(&a0[16]));
+        tmem_st16(sa, a0);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(BAR(C::B_A0F + b));
 
         if (p.order == 1) {
-          // One runtime iteration per block of this chunk that some row of the tile
-          // approximates (kept rolled: an unrolled copy of this loop is large enough to
-          // evict the MMA-issuing warp's instructions). The row's alpha comes from the
+          // one runtime iteration per pair of approximated blocks (kept rolled: an
+          // unrolled copy evicts the MMA warp's instructions). alpha comes from the
           // packed bf16 operand a0 (zero where the row's own block is exact).
           const int a_end = chunk_off[c + 1];
 #pragma unroll 1
-          for (; a < a_end; ++a) {
-            const int k = approx_list[a] - c * C::CHUNK;
-            const int slot = a % C::NA;
-            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_AE + slot), ((a / C::NA) & 1) ^ 1, abort_flag));
+          for (int a = chunk_off[c]; a < a_end; a += C::GROUP, ++g) {
+            const int n = min(C::GROUP, a_end - a);
+            const int gs = g & 1;
+            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_AE + gs), ((g >> 1) & 1) ^ 1, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            const uint32_t w = a0[k >> 1];
-            const float coef = ((k & 1) ? bf16_hi(w) : bf16_lo(w)) * p.scale;
-            const __nv_bfloat162 c2 = __floats2bfloat162_rn(coef, coef);
-            const uint32_t cw = *reinterpret_cast<const uint32_t*>(&c2);
-            const uint32_t aa = tmem + lrow + C::A_COL0 + slot * C::A_COLS;
+#pragma unroll 1
+            for (int qq = 0; qq < n; ++qq) {
+              const int k = approx_list[a + qq] - c * C::CHUNK;
+              const uint32_t w = a0[k >> 1];
+              const float coef = ((k & 1) ? bf16_hi(w) : bf16_lo(w)) * p.scale;
+              const __nv_bfloat162 c2 = __floats2bfloat162_rn(coef, coef);
+              const uint32_t cw = *reinterpret_cast<const uint32_t*>(&c2);
+              const uint32_t aa = tmem + lrow + C::A_COL0 + (gs * C::GROUP + qq) * C::A_COLS;
 #pragma unroll
-            for (int ch = 0; ch < D / 32; ++ch) {
-              uint32_t t[16];
+              for (int ch = 0; ch < D / 32; ++ch) {
+                uint32_t t[16];
 #pragma unroll
-              for (int i = 0; i < 16; ++i) t[i] = hmul2_bf16(q[ch * 16 + i], cw);
-              tmem_st16(aa + ch * 16, t);
+                for (int i = 0; i < 16; ++i) t[i] = hmul2_bf16(q[ch * 16 + i], cw);
+                tmem_st16(aa + ch * 16, t);
+              }
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(BAR(C::B_AF + slot));
+            mbar_arrive(BAR(C::B_GA + gs));
           }
         }
       }

@@ -32,6 +32,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-suspending probe of a phase (the MMA-issuing thread polls with it: a thread
+// suspended inside try_wait resumes too late to keep the tensor pipe fed).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Every wait is bounded: after kWaitCycles SM cycles (about a second) the waiter
 // raises the CTA's abort flag and the device error word and gives up; a waiter
 // also gives up as soon as another role has raised the abort flag.
@@ -42,6 +56,21 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      *abort_flag = 1;
+      flag_error(kErrTimeout);
+      return false;
+    }
+  }
+}
+
+// bounded polling wait with the non-suspending probe (same limits as wait_bounded)
+__device__ __forceinline__ bool wait_poll(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_test_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     if (clock64() - t0 > kWaitCycles) {
       *abort_flag = 1;
