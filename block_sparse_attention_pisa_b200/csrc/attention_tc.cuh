@@ -37,10 +37,11 @@
 // maximum grows by more than 2^8 (exact by construction, rare).
 //
 // Synchronisation: the MMA thread polls its barriers with the non-suspending
-// mbarrier probe, and waits once per exact block (K_j and V_j land on one
-// barrier) and once per pair of approximated blocks (both S1 tiles on one
-// barrier, both A operands on another): every wait it makes costs tensor-pipe
-// time, so there are few of them. Every wait is bounded by clock64; on timeout a
+// mbarrier probe and waits as rarely as it can, because every wait it makes costs
+// tensor-pipe time: per exact block once for K_j and V_j (one barrier) and once
+// for P; per pair of approximated blocks once (the row threads signal a pair only
+// after writing both A operands and seeing both S1 tiles land). The exact scores
+// run two blocks ahead of the softmax (b = 64). Every wait is bounded by clock64; on timeout a
 // CTA raises the device error word, drains its copies and MMAs, frees TMEM and
 // exits.
 #pragma once
@@ -124,6 +125,12 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// two non-negative finite floats -> packed bf16x2, rounded to nearest (ties up),
+// with integer ops instead of the conversion unit (which the exponentials share)
+__device__ __forceinline__ uint32_t pack_bf16x2_int(float lo, float hi) {
+  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
 }
 
 __device__ __forceinline__ uint32_t hmul2_bf16(uint32_t a, uint32_t b) {
@@ -363,10 +370,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         umma_commit(BAR(C::B_PV + sb));
         return true;
       };
-      for (int e = 0; e < n_exact && ok; ++e) {
+      // S = Q K_j^T for block e (its buffer was last used by block e - NSB)
+      auto qk = [&](int e) -> bool {
         const int sb = e % C::NSB;
-        if (e >= C::NSB && !(ok = wait_poll(BAR(C::B_PV + sb), ((e - C::NSB) / C::NSB) & 1, abort_flag))) break;
-        if (!(ok = wait_poll(BAR(C::B_TF + e % C::NTF), (e / C::NTF) & 1, abort_flag))) break;
+        if (e >= C::NSB && !wait_poll(BAR(C::B_PV + sb), ((e - C::NSB) / C::NSB) & 1, abort_flag)) return false;
+        if (!wait_poll(BAR(C::B_TF + e % C::NTF), (e / C::NTF) & 1, abort_flag)) return false;
         tc_fence_after();
         const int sk = (2 * e) % C::NS;
         const uint32_t kb = base_u + C::OFF_RING + sk * C::STAGE;
@@ -376,9 +384,15 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                   sdesc_sw128(kb + (k >> 2) * (BLK * 128) + (k & 3) * 32, 16, 1024), idS, k ? 1u : 0u);
         umma_commit(BAR(C::B_SE + sk));
         umma_commit(BAR(C::B_SF + sb));
-        if (e >= 1) ok = pv(e - 1);
+        return true;
+      };
+      // the scores run kLook blocks ahead of the row threads' softmax
+      constexpr int kLook = C::NSB >= 4 ? C::NSB - 2 : 1;
+      for (int e = 0; e < kLook && e < n_exact && ok; ++e) ok = qk(e);
+      for (int e = 0; e < n_exact && ok; ++e) {
+        ok = pv(e);
+        if (ok && e + kLook < n_exact) ok = qk(e + kLook);
       }
-      if (ok && n_exact > 0) ok = pv(n_exact - 1);
       umma_commit(BAR(C::B_OSYNC));  // completion 0: end of the exact stage
 
       if (ok && n_active > 0) {
@@ -420,8 +434,9 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             for (int a = chunk_off[c]; a < a_end; a += C::GROUP, ++g, ++u) {
               const int n = min(C::GROUP, a_end - a);
               const int gs = g & 1;
+              // the row threads signal a pair only after its S1 copies have landed, so one
+              // wait covers both operands
               if (!(ok = wait_poll(BAR(C::B_GA + gs), (g >> 1) & 1, abort_flag))) break;
-              if (!(ok = wait_poll(BAR(C::B_TF + u % C::NTF), (u / C::NTF) & 1, abort_flag))) break;
               tc_fence_after();
               for (int q = 0; q < n; ++q, ++t) {
                 const int s = t % C::NS;
@@ -522,13 +537,18 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       for (int ch = 0; ch < BLK / 16; ++ch) tmem_ld16(sa + ch * 16, *reinterpret_cast<uint32_t(*)[16]>(&s[ch * 16]));
 #pragma unroll
       for (int ch = 0; ch < BLK / 16; ++ch) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&s[ch * 16]));
-      float mx = -INFINITY;
+      // (independent partial maxima: one warp per SMSP cannot hide a serial chain)
+      float mxp[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mxp[i] = -INFINITY;
 #pragma unroll
       for (int k = 0; k < BLK; ++k) {
         const float v = (sel && k < nj) ? __uint_as_float(s[k]) * sl2 : -INFINITY;
         s[k] = __float_as_uint(v);
-        mx = fmaxf(mx, v);
+        mxp[k & 7] = fmaxf(mxp[k & 7], v);
       }
+      const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                             fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
       const bool grow_max = mx > m + 8.f;          // false for rows that did not select j
       const bool need_o = grow_max && m != -INFINITY;
       if (__any_sync(0xffffffffu, need_o)) {
@@ -543,7 +563,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         l *= f;
       }
       if (grow_max) m = mx;
-      float rs = 0.f;
+      float rsp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int ch = 0; ch < BLK / 32; ++ch) {
         uint32_t pk[16];
@@ -553,12 +573,12 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           // still be -inf for them, so no exponential is evaluated)
           const float p0 = sel ? ex2(__uint_as_float(s[ch * 32 + 2 * i]) - m) : 0.f;
           const float p1 = sel ? ex2(__uint_as_float(s[ch * 32 + 2 * i + 1]) - m) : 0.f;
-          rs += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
+          rsp[i & 3] += p0 + p1;
+          pk[i] = pack_bf16x2_int(p0, p1);
         }
         tmem_st16(sa + ch * 16, pk);
       }
-      l += rs;
+      l += (rsp[0] + rsp[1]) + (rsp[2] + rsp[3]);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(BAR(C::B_PF + sb));
@@ -593,14 +613,15 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
         const uint32_t myw = mymask[c];
         const int kmax = nB - c * C::CHUNK;  // blocks of this chunk that exist
-        float mx = -INFINITY;
+        float mxp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int k = 0; k < C::CHUNK; ++k) {
           const bool mine = k < kmax && !((myw >> k) & 1u);
           const float v = mine ? __uint_as_float(sv[k]) * sl2 : -INFINITY;
           sv[k] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
+          mxp[k & 3] = fmaxf(mxp[k & 3], v);
         }
+        const float mx = fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3]));
         const bool need_o = mx > m + 8.f;
         if (__any_sync(0xffffffffu, need_o)) {
           ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_OSYNC), ac & 1, abort_flag));
@@ -611,7 +632,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           l *= f;
           if (need_o) m = mx;
         }
-        float ls = 0.f;
+        float lsp[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t a0[C::CHUNK / 2];
 #pragma unroll
         for (int k = 0; k < C::CHUNK; k += 2) {
@@ -619,11 +640,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           const float x1 = ex2(__uint_as_float(sv[k + 1]) - m);
           const float n0 = (c * C::CHUNK + k == nB - 1) ? float(nlast) : float(BLK);
           const float n1 = (c * C::CHUNK + k + 1 == nB - 1) ? float(nlast) : float(BLK);
-          ls = fmaf(n0, x0, ls);
-          ls = fmaf(n1, x1, ls);
-          a0[k >> 1] = pack_bf16x2(x0, x1);
+          lsp[(k >> 1) & 3] = fmaf(n1, x1, fmaf(n0, x0, lsp[(k >> 1) & 3]));
+          a0[k >> 1] = pack_bf16x2_int(x0, x1);
         }
-        l += ls;
+        l += (lsp[0] + lsp[1]) + (lsp[2] + lsp[3]);
         tmem_st16(sa, a0);
         tmem_wait_st();
         tc_fence_before();
@@ -659,6 +679,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             }
             tmem_wait_st();
             tc_fence_before();
+            // the pair's S1 tiles (load unit n_exact + g) must have landed as well
+            const int u = n_exact + g;
+            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_TF + u % C::NTF), (u / C::NTF) & 1, abort_flag));
+            if (!ok) break;
             mbar_arrive(BAR(C::B_GA + gs));
           }
         }

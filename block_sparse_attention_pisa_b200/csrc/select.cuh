@@ -7,23 +7,25 @@
 // throughout, so that the ranking matches an exact evaluation except at
 // near-ties).
 //
-// One CTA handles kQB consecutive query blocks of one head:
-//   1. pool: stream the kQB query blocks once (16-byte coalesced loads) and
-//      average their rows into qbar (fp32, shared memory);
-//   2. score: one thread per key block j computes kQB dot products against
-//      kbar_j (fp32 FMA, kbar read through the read-only cache; a head's kbar
-//      is shared by all CTAs of that head and stays in L2);
-//   3. top-k: one warp per row finds the k-th largest score key bit by bit
-//      (a count of keys >= candidate per bit), then emits the selected block
-//      indices in ascending order with ballots; among keys equal to the
-//      threshold the lowest indices are taken.
+// One CTA handles kSelectQB consecutive query blocks of one head:
+//   1. pool: stream the query blocks once (16-byte coalesced loads, two row
+//      halves per (block, 16-byte column) pair) and average their rows into
+//      qbar (fp32, shared memory);
+//   2. score: each thread takes two key blocks per pass and forms kSelectQB dot
+//      products against each (fp32 FMA; kbar read through the read-only cache --
+//      a head's kbar is shared by all its CTAs and stays in L2). Scores are
+//      stored as order-preserving uint32 keys;
+//   3. top-k: one warp per row finds the k-th largest key bit by bit (a count of
+//      keys >= candidate per bit, starting below the row's common key prefix),
+//      then emits the selected block indices in ascending order with ballots;
+//      among keys equal to the threshold the lowest indices are taken.
 #pragma once
 
 #include "common.cuh"
 
 namespace pisa {
 
-constexpr int kSelectQB = 16;        // query blocks per CTA
+constexpr int kSelectQB = 8;         // query blocks per CTA
 constexpr int kSelectThreads = 256;
 
 __host__ __device__ constexpr int select_score_ld(int nB) { return ((nB + 31) / 32) * 32 + 4; }
@@ -33,8 +35,9 @@ __global__ void __launch_bounds__(kSelectThreads)
 select_kernel(const bf16* __restrict__ Q, const float* __restrict__ kbar, int N, int nB,
               int block, int topk, int32_t* __restrict__ idx) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  float* sQbar = reinterpret_cast<float*>(smem_raw);  // [kQB][D]
-  float* sScore = sQbar + kSelectQB * D;                // [kQB][ld]
+  float* sQbar = reinterpret_cast<float*>(smem_raw);                    // [QB][D]
+  float* sHalf = sQbar + kSelectQB * D;                                 // [QB][D] second-half row sums
+  uint32_t* sKey = reinterpret_cast<uint32_t*>(sHalf + kSelectQB * D);  // [QB][ld]
   const int ld = select_score_ld(nB);
 
   const size_t bh = blockIdx.y;
@@ -42,20 +45,21 @@ select_kernel(const bf16* __restrict__ Q, const float* __restrict__ kbar, int N,
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int CH = D / 8;
 
-  // ---- 1. pooled queries ----
-  for (int p = tid; p < kSelectQB * CH; p += kSelectThreads) {
-    const int qb = p / CH, ch = p % CH;
+  // ---- 1. pooled queries: item = (query block, 16-byte column, row half) ----
+  for (int p = tid; p < kSelectQB * CH * 2; p += kSelectThreads) {
+    const int half = p / (kSelectQB * CH);
+    const int qb = (p / CH) % kSelectQB, ch = p % CH;
     const int i = i0 + qb;
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-    int n = 0;
     if (i < nB) {
       const int s = i * block;
-      n = min(block, N - s);
+      const int n = min(block, N - s);
+      const int r0 = half ? (n + 1) / 2 : 0, r1 = half ? n : (n + 1) / 2;
       const bf16* src = Q + (bh * size_t(N) + s) * D + ch * 8;
 #pragma unroll 8
-      for (int r = 0; r < n; ++r) {
+      for (int r = r0; r < r1; ++r) {
         const uint4 w = ldg_stream_v4(src + size_t(r) * D);
         const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -65,33 +69,50 @@ select_kernel(const bf16* __restrict__ Q, const float* __restrict__ kbar, int N,
         }
       }
     }
-    const float inv = n > 0 ? 1.f / float(n) : 0.f;
+    float* dst = (half ? sHalf : sQbar) + qb * D + ch * 8;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) sQbar[qb * D + ch * 8 + e] = acc[e] * inv;
+    for (int e = 0; e < 8; ++e) dst[e] = acc[e];
+  }
+  __syncthreads();
+  for (int p = tid; p < kSelectQB * D; p += kSelectThreads) {
+    const int i = i0 + p / D;
+    const int n = i < nB ? min(block, N - i * block) : 1;
+    sQbar[p] = (sQbar[p] + sHalf[p]) * (1.f / float(n));
   }
   __syncthreads();
 
-  // ---- 2. pooled scores: thread per key block ----
+  // ---- 2. pooled scores: each thread two key blocks per pass ----
   const float* kb_head = kbar + bh * size_t(nB) * D;
-  for (int j = tid; j < nB; j += kSelectThreads) {
-    float acc[kSelectQB];
+  for (int j0 = tid; j0 < nB; j0 += 2 * kSelectThreads) {
+    const int j1 = j0 + kSelectThreads;
+    const bool has1 = j1 < nB;
+    float a0[kSelectQB], a1[kSelectQB];
 #pragma unroll
-    for (int q = 0; q < kSelectQB; ++q) acc[q] = 0.f;
-    const float4* krow = reinterpret_cast<const float4*>(kb_head + size_t(j) * D);
+    for (int q = 0; q < kSelectQB; ++q) a0[q] = a1[q] = 0.f;
+    const float4* k0row = reinterpret_cast<const float4*>(kb_head + size_t(j0) * D);
+    const float4* k1row = reinterpret_cast<const float4*>(kb_head + size_t(has1 ? j1 : j0) * D);
 #pragma unroll 4
     for (int a4 = 0; a4 < D / 4; ++a4) {
-      const float4 k = __ldg(krow + a4);
+      const float4 k0 = __ldg(k0row + a4);
+      const float4 k1 = __ldg(k1row + a4);
 #pragma unroll
       for (int q = 0; q < kSelectQB; ++q) {
         const float4 x = reinterpret_cast<const float4*>(sQbar + q * D)[a4];
-        acc[q] = fmaf(x.x, k.x, acc[q]);
-        acc[q] = fmaf(x.y, k.y, acc[q]);
-        acc[q] = fmaf(x.z, k.z, acc[q]);
-        acc[q] = fmaf(x.w, k.w, acc[q]);
+        a0[q] = fmaf(x.x, k0.x, a0[q]);
+        a0[q] = fmaf(x.y, k0.y, a0[q]);
+        a0[q] = fmaf(x.z, k0.z, a0[q]);
+        a0[q] = fmaf(x.w, k0.w, a0[q]);
+        a1[q] = fmaf(x.x, k1.x, a1[q]);
+        a1[q] = fmaf(x.y, k1.y, a1[q]);
+        a1[q] = fmaf(x.z, k1.z, a1[q]);
+        a1[q] = fmaf(x.w, k1.w, a1[q]);
       }
     }
 #pragma unroll
-    for (int q = 0; q < kSelectQB; ++q) sScore[q * ld + j] = acc[q] + 0.f;  // -0 -> +0
+    for (int q = 0; q < kSelectQB; ++q) {
+      sKey[q * ld + j0] = float_order_key(a0[q] + 0.f);  // -0 -> +0
+      if (has1) sKey[q * ld + j1] = float_order_key(a1[q] + 0.f);
+    }
   }
   __syncthreads();
 
@@ -100,24 +121,36 @@ select_kernel(const bf16* __restrict__ Q, const float* __restrict__ kbar, int N,
   for (int q = warp; q < kSelectQB; q += kSelectThreads / 32) {
     const int i = i0 + q;
     if (i >= nB) break;
-    const float* row = sScore + q * ld;
-    uint32_t T = 0;
-    for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t* row = sKey + q * ld;
+    // the k-th largest key lies between the row's extremes: bits above their
+    // first difference are common to every candidate threshold
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    for (int jj = lane; jj < nB; jj += 32) {
+      const uint32_t k = row[jj];
+      kmin = min(kmin, k);
+      kmax = max(kmax, k);
+    }
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    const uint32_t diff = kmin ^ kmax;
+    const int top = diff ? 31 - __clz(diff) : -1;  // highest differing bit
+    uint32_t T = top < 0 ? kmax : (top >= 31 ? 0u : (kmax & ~((2u << top) - 1u)));
+    for (int bit = top; bit >= 0; --bit) {
       const uint32_t cand = T | (1u << bit);
       unsigned cnt = 0;
-      for (int jj = lane; jj < nB; jj += 32) cnt += float_order_key(row[jj]) >= cand;
+      for (int jj = lane; jj < nB; jj += 32) cnt += row[jj] >= cand;
       cnt = __reduce_add_sync(0xffffffffu, cnt);
       if (cnt >= unsigned(topk)) T = cand;
     }
     unsigned gt = 0;
-    for (int jj = lane; jj < nB; jj += 32) gt += float_order_key(row[jj]) > T;
+    for (int jj = lane; jj < nB; jj += 32) gt += row[jj] > T;
     gt = __reduce_add_sync(0xffffffffu, gt);
     const int need_eq = topk - int(gt);
     int32_t* out = idx + (bh * size_t(nB) + i) * topk;
     int written = 0, eq_seen = 0;
     for (int base = 0; base < nB; base += 32) {
       const int jj = base + lane;
-      const uint32_t key = jj < nB ? float_order_key(row[jj]) : 0u;
+      const uint32_t key = jj < nB ? row[jj] : 0u;
       const bool is_gt = jj < nB && key > T;
       const bool is_eq = jj < nB && key == T;
       const unsigned eq_mask = __ballot_sync(0xffffffffu, is_eq);
@@ -131,7 +164,7 @@ select_kernel(const bf16* __restrict__ Q, const float* __restrict__ kbar, int N,
 }
 
 inline size_t select_smem_bytes(int D, int nB) {
-  return size_t(kSelectQB) * D * sizeof(float) + size_t(kSelectQB) * select_score_ld(nB) * sizeof(float);
+  return size_t(2) * kSelectQB * D * sizeof(float) + size_t(kSelectQB) * select_score_ld(nB) * sizeof(uint32_t);
 }
 
 }  // namespace pisa

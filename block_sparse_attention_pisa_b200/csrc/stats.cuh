@@ -10,8 +10,9 @@
 // 16-byte coalesced loads into padded shared memory; the column sums are
 // reduced with warp shuffles and a small shared-memory pass. S1 is formed as
 // K_j^T V_j on the tensor cores (fp32 accumulation over bf16 inputs, so the
-// products are exact) minus kbar_j S0_j^T in fp32, rounded once to bf16, staged
-// in shared memory and written with coalesced 16-byte stores.
+// products are exact) minus kbar_j S0_j^T in fp32, rounded once to bf16 and
+// written with coalesced 16-byte stores from a staging tile, one half of the
+// value dimension at a time (two passes keep 32 accumulators per thread).
 //
 // The kernel is HBM-bound (K, V in; S1 out). The d x b x d contraction is ~32
 // flop/byte, below the tensor ridge, so the warp-level mma.sync path keeps it
@@ -29,21 +30,23 @@ struct StatsCfg {
   static constexpr int kChunks = D / 8;         // 16-byte chunks per row
   static constexpr int kRowStep = kThreads / kChunks;
   static constexpr int kTileElems = BLK * kLd;  // one of sK / sV
-  static constexpr size_t kSmem = size_t(2) * kTileElems * sizeof(bf16)  // sK, sV (S1 staging reuses both)
+  static constexpr int kStageLd = D / 2 + 8;    // padded row of one value-dimension half of S1
+  static constexpr size_t kSmem = size_t(2) * kTileElems * sizeof(bf16)  // sK, sV
+                                  + size_t(D) * kStageLd * sizeof(bf16)  // S1 half staging
                                   + size_t(8) * 2 * D * sizeof(float)    // per-warp partial sums
                                   + size_t(2) * D * sizeof(float);       // kbar, S0
-  static_assert(2 * kTileElems >= D * kLd, "S1 staging must fit in the K/V tiles");
 };
 
 template <int D, int BLK>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 3)
 stats_kernel(const bf16* __restrict__ K, const bf16* __restrict__ V, int N, int nB, int order,
              float* __restrict__ kbar, float* __restrict__ S0, bf16* __restrict__ S1) {
   using C = StatsCfg<D, BLK>;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   bf16* sK = reinterpret_cast<bf16*>(smem_raw);
   bf16* sV = sK + C::kTileElems;
-  float* sPart = reinterpret_cast<float*>(sV + C::kTileElems);  // [8 warps][2][D]
+  bf16* sStage = sV + C::kTileElems;                            // [D][kStageLd]
+  float* sPart = reinterpret_cast<float*>(sStage + D * C::kStageLd);  // [8 warps][2][D]
   float* sKbar = sPart + 8 * 2 * D;
   float* sS0 = sKbar + D;
 
@@ -117,68 +120,73 @@ stats_kernel(const bf16* __restrict__ K, const bf16* __restrict__ V, int N, int 
   __syncthreads();
 
   // ---- S1 = K^T V - kbar S0^T : M = D (key dim a), N = D (value dim c), K = BLK tokens ----
-  constexpr int TM = D / 4, TN = D / 2;      // warp tile (8 warps as 4 x 2)
+  // Two passes over halves of the value dimension keep 32 accumulators per
+  // thread (4 CTAs per SM); fragments go straight to global memory.
+  constexpr int TM = D / 4, TN = D / 4;      // warp tile per pass (8 warps as 4 x 2)
   constexpr int MT = TM / 16, NT = TN / 8;
   const int a_base = (warp >> 1) * TM;
-  const int c_base = (warp & 1) * TN;
-  float acc[MT][NT][4];
-#pragma unroll
-  for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
-
   const uint32_t sK_u = smem_u32(sK), sV_u = smem_u32(sV);
+  bf16* gS1 = S1 + (bh * size_t(nB) + j) * D * D;
+  const int g = lane >> 2, t4 = lane & 3;
+#pragma unroll 1
+  for (int pass = 0; pass < 2; ++pass) {
+    const int c_base = pass * (D / 2) + (warp & 1) * TN;
+    float acc[MT][NT][4];
 #pragma unroll
-  for (int kt = 0; kt < BLK / 16; ++kt) {
-    uint32_t af[MT][4];
+    for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-      // A[a][n] = K[n][a]: transposed 8x8 loads from rows n, columns a
-      const int row = kt * 16 + (lane & 7) + ((lane >> 4) << 3);
-      const int col = a_base + mt * 16 + (((lane >> 3) & 1) << 3);
-      ldsm_x4_trans(sK_u + (row * C::kLd + col) * 2, af[mt][0], af[mt][1], af[mt][2], af[mt][3]);
-    }
+      for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-    for (int np = 0; np < NT / 2; ++np) {
-      // B[n][c] = V[n][c]: two n8 tiles per x4 load
-      const int row = kt * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
-      const int col = c_base + np * 16 + ((lane >> 4) << 3);
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4_trans(sV_u + (row * C::kLd + col) * 2, b0, b1, b2, b3);
+        for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
+#pragma unroll
+    for (int kt = 0; kt < BLK / 16; ++kt) {
+      uint32_t af[MT][4];
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
-        mma_bf16_16816(acc[mt][2 * np], af[mt], b0, b1);
-        mma_bf16_16816(acc[mt][2 * np + 1], af[mt], b2, b3);
+        // A[a][n] = K[n][a]: transposed 8x8 loads from rows n, columns a
+        const int row = kt * 16 + (lane & 7) + ((lane >> 4) << 3);
+        const int col = a_base + mt * 16 + (((lane >> 3) & 1) << 3);
+        ldsm_x4_trans(sK_u + (row * C::kLd + col) * 2, af[mt][0], af[mt][1], af[mt][2], af[mt][3]);
+      }
+#pragma unroll
+      for (int np = 0; np < NT / 2; ++np) {
+        // B[n][c] = V[n][c]: two n8 tiles per x4 load
+        const int row = kt * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+        const int col = c_base + np * 16 + ((lane >> 4) << 3);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_trans(sV_u + (row * C::kLd + col) * 2, b0, b1, b2, b3);
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          mma_bf16_16816(acc[mt][2 * np], af[mt], b0, b1);
+          mma_bf16_16816(acc[mt][2 * np + 1], af[mt], b2, b3);
+        }
       }
     }
-  }
-  __syncthreads();  // all warps are done reading sK / sV: reuse them as the S1 staging tile
-
-  bf16* sOut = sK;  // [D][kLd]
-  const int g = lane >> 2, t4 = lane & 3;
+    if (pass) __syncthreads();  // the previous half has been copied out of the staging tile
 #pragma unroll
-  for (int mt = 0; mt < MT; ++mt) {
+    for (int mt = 0; mt < MT; ++mt) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int a = a_base + mt * 16 + g;
-      const int c = c_base + nt * 8 + 2 * t4;
-      const float k0 = sKbar[a], k1 = sKbar[a + 8];
-      const float s0 = sS0[c], s1 = sS0[c + 1];
-      *reinterpret_cast<uint32_t*>(sOut + a * C::kLd + c) =
-          pack_bf16x2(acc[mt][nt][0] - k0 * s0, acc[mt][nt][1] - k0 * s1);
-      *reinterpret_cast<uint32_t*>(sOut + (a + 8) * C::kLd + c) =
-          pack_bf16x2(acc[mt][nt][2] - k1 * s0, acc[mt][nt][3] - k1 * s1);
+      for (int nt = 0; nt < NT; ++nt) {
+        const int a = a_base + mt * 16 + g;
+        const int c = c_base + nt * 8 + 2 * t4;  // global value column
+        const int cl = c - pass * (D / 2);       // column inside the staged half
+        const float k0 = sKbar[a], k1 = sKbar[a + 8];
+        const float s0 = sS0[c], s1 = sS0[c + 1];
+        *reinterpret_cast<uint32_t*>(sStage + a * C::kStageLd + cl) =
+            pack_bf16x2(acc[mt][nt][0] - k0 * s0, acc[mt][nt][1] - k0 * s1);
+        *reinterpret_cast<uint32_t*>(sStage + (a + 8) * C::kStageLd + cl) =
+            pack_bf16x2(acc[mt][nt][2] - k1 * s0, acc[mt][nt][3] - k1 * s1);
+      }
     }
-  }
-  __syncthreads();
-  bf16* gS1 = S1 + (bh * size_t(nB) + j) * D * D;
+    __syncthreads();
+    // coalesced 16-byte stores of this half: D rows x (D/2) columns
+    constexpr int HC = D / 16;  // 16-byte chunks per half row
 #pragma unroll 4
-  for (int q = tid; q < D * C::kChunks; q += C::kThreads) {
-    const int a = q / C::kChunks, c8 = q % C::kChunks;
-    *reinterpret_cast<uint4*>(gS1 + size_t(a) * D + c8 * 8) =
-        *reinterpret_cast<const uint4*>(sOut + a * C::kLd + c8 * 8);
+    for (int q = tid; q < D * HC; q += C::kThreads) {
+      const int a = q / HC, c8 = q % HC;
+      *reinterpret_cast<uint4*>(gS1 + size_t(a) * D + pass * (D / 2) + c8 * 8) =
+          *reinterpret_cast<const uint4*>(sStage + a * C::kStageLd + c8 * 8);
+    }
   }
 }
 
