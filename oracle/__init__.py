@@ -28,4 +28,9 @@ from .pisa import (  # noqa: F401
     select,
     attention,
     dense_attention,
+    global_first_order,
+    ORDER_DROP,
+    ORDER_ZERO,
+    ORDER_FIRST,
+    ORDER_HYBRID,
 )

@@ -120,6 +120,16 @@ def _query_blocks(nB, query_blocks):
     return range(nB) if query_blocks is None else query_blocks
 
 
+ORDER_DROP, ORDER_ZERO, ORDER_FIRST, ORDER_HYBRID = -1, 0, 1, 2
+
+
+def global_first_order(S1):
+    """Hbar [B,H,d,d]: the mean of the per-block first-order matrices over all
+    blocks of a head (section 2, "Core algorithm", global first-order correction;
+    "Hardware implementation", precompute step)."""
+    return np.asarray(S1, dtype=np.float64).mean(axis=2)
+
+
 def attention(Q, K, V, kbar, S0, S1, idx, block: int, order: int, scale: float,
               query_blocks=None, heads=None):
     """PISA output rows (float64 [B,H,N,d]; rows of skipped query blocks are NaN).
@@ -127,6 +137,15 @@ def attention(Q, K, V, kbar, S0, S1, idx, block: int, order: int, scale: float,
     ``idx`` [B,H,nB,k] lists the critical blocks of each query block (any
     order; ``k`` may be 0). ``query_blocks`` / ``heads`` restrict the work to a
     sample; ``heads`` is a list of (b, h) pairs.
+
+    ``order`` selects the treatment of the non-critical blocks:
+      -1  drop them (keep-or-drop block-sparse attention, the baseline class the
+          explainer contrasts with, section 1);
+       0  zeroth-order Taylor term only;
+       1  zeroth- plus per-block first-order term (``S1`` = per-block matrices);
+       2  zeroth-order term plus the global first-order correction
+          ``(x_t Hbar) sum_{j in U_i} alpha_{t,j}`` of section 2 ("Core
+          algorithm": hybrid order), with ``S1`` = Hbar [B,H,d,d].
     """
     Q = np.asarray(Q, dtype=np.float64)
     K = np.asarray(K, dtype=np.float64)
@@ -149,6 +168,9 @@ def attention(Q, K, V, kbar, S0, S1, idx, block: int, order: int, scale: float,
             z_ex = X @ K[b, h, keys].T                        # [n_i, |keys|]
             # zeroth-order exponents over the non-critical blocks
             z_ap = X @ kbar[b, h, rest].T                     # [n_i, |U|]
+            if order == ORDER_DROP:
+                z_ap = z_ap[:, :0]
+                rest = []
             m = np.full(e_i - s_i, -np.inf)
             if z_ex.size:
                 m = np.maximum(m, z_ex.max(axis=1))
@@ -158,10 +180,13 @@ def attention(Q, K, V, kbar, S0, S1, idx, block: int, order: int, scale: float,
             alpha = np.exp(z_ap - m[:, None])
             num = w @ V[b, h, keys] + alpha @ S0[b, h, rest]
             den = w.sum(axis=1) + alpha @ counts[rest]
-            if order >= 1 and rest:
+            if order == ORDER_FIRST and rest:
                 # S1_j^T x_t for every (j, t): first[j, t, c] = sum_a x[t, a] S1_j[a, c]
                 first = np.matmul(X[None], S1[b, h, rest])
                 num = num + np.einsum("tj,jtc->tc", alpha, first)
+            elif order == ORDER_HYBRID and rest:
+                # (x_t Hbar) scaled by the row's total non-critical weight
+                num = num + (X @ S1[b, h]) * alpha.sum(axis=1)[:, None]
             O[b, h, s_i:e_i] = num / den[:, None]
     return O
 

@@ -323,3 +323,102 @@ def pin_worked_example(orc, case):
                     den += a * len(toks)
             err = max(err, abs(out[0, 0, t, 0] - num / den))
     return err
+
+
+# ----------------------------------------------------------------------------
+# keep-or-drop and hybrid order
+# ----------------------------------------------------------------------------
+def pin_drop_is_masked_softmax(orc, seed=14):
+    """Keep-or-drop: textbook softmax over the critical blocks' keys only (the
+    other logits masked to -inf), ragged last block included."""
+    r = _rng(seed)
+    B, H, N, d, b = 1, 2, 37, 5, 8
+    Q, K, V = (r.standard_normal((B, H, N, d)) for _ in range(3))
+    kbar, S0, S1 = orc.block_stats(K, V, b)
+    nB = -(-N // b)
+    idx = np.stack([np.sort(r.choice(nB, 2, replace=False)) for _ in range(B * H * nB)])
+    idx = idx.reshape(B, H, nB, 2).astype(np.int32)
+    out = orc.attention(Q, K, V, kbar, S0, S1, idx, b, -1, 0.7)
+    err = 0.0
+    for h in range(H):
+        z = 0.7 * Q[0, h] @ K[0, h].T
+        for t in range(N):
+            keep = np.zeros(N, dtype=bool)
+            for j in idx[0, h, t // b]:
+                keep[j * b:min(j * b + b, N)] = True
+            zt = np.where(keep, z[t], -np.inf)
+            err = max(err, np.abs(softmax(zt) @ V[0, h] - out[0, h, t]).max())
+    return err
+
+
+def pin_hybrid_bruteforce(orc, seed=15):
+    """Hybrid order written out with scalar loops: Hbar = mean over all blocks of
+    sum_n (k_n - kbar_j) v_n^T, then N_t = exact + sum_U alpha (sum v) +
+    (x Hbar) sum_U alpha, D_t = exact + sum_U n_j alpha (ragged last block)."""
+    r = _rng(seed)
+    B, H, N, d, b = 1, 1, 27, 3, 6
+    Q, K, V = (r.standard_normal((B, H, N, d)) for _ in range(3))
+    kbar, S0, S1 = orc.block_stats(K, V, b)
+    Hbar = orc.global_first_order(S1)
+    nB = -(-N // b)
+    blocks = [list(range(j * b, min(j * b + b, N))) for j in range(nB)]
+    cen = [[sum(K[0, 0, n, a] for n in bl) / len(bl) for a in range(d)] for bl in blocks]
+    ref_H = [[sum(sum((K[0, 0, n, a] - cen[j][a]) * V[0, 0, n, c] for n in bl)
+                  for j, bl in enumerate(blocks)) / nB for c in range(d)] for a in range(d)]
+    err = float(np.abs(Hbar[0, 0] - np.array(ref_H)).max())
+    crit = [[i, (i + 2) % nB] for i in range(nB)]
+    idx = np.sort(np.array(crit, dtype=np.int32), axis=1)[None, None]
+    scale = 0.8
+    out = orc.attention(Q, K, V, kbar, S0, Hbar, idx, b, 2, scale)
+    for t in range(N):
+        x = [scale * Q[0, 0, t, a] for a in range(d)]
+        num = [0.0] * d
+        den = 0.0
+        asum = 0.0
+        for j, bl in enumerate(blocks):
+            if j in crit[t // b]:
+                for n in bl:
+                    w = math.exp(sum(x[a] * K[0, 0, n, a] for a in range(d)))
+                    den += w
+                    for c in range(d):
+                        num[c] += w * V[0, 0, n, c]
+            else:
+                al = math.exp(sum(x[a] * cen[j][a] for a in range(d)))
+                asum += al
+                den += len(bl) * al
+                for c in range(d):
+                    num[c] += al * sum(V[0, 0, n, c] for n in bl)
+        for c in range(d):
+            num[c] += asum * sum(x[a] * ref_H[a][c] for a in range(d))
+            err = max(err, abs(out[0, 0, t, c] - num[c] / den))
+    return err
+
+
+def pin_hybrid_shared_first_order(orc, seed=16):
+    """Blocks that are translated copies of one pattern (k = c_j + z_n, v = u_n)
+    share a single first-order matrix, so Hbar = S1_j and the hybrid order equals
+    the per-block first-order output."""
+    r = _rng(seed)
+    B, H, b, nB, d = 1, 1, 8, 6, 5
+    N = b * nB
+    c = r.standard_normal((nB, d)) * 2
+    z = r.standard_normal((b, d)) * 0.3
+    u = r.standard_normal((b, d))
+    K = (np.repeat(c, b, axis=0) + np.tile(z, (nB, 1)))[None, None]
+    V = np.tile(u, (nB, 1))[None, None]
+    Q = r.standard_normal((B, H, N, d))
+    kbar, S0, S1 = orc.block_stats(K, V, b)
+    idx = np.array([[[[i] for i in range(nB)]]], dtype=np.int32)
+    first = orc.attention(Q, K, V, kbar, S0, S1, idx, b, 1, 0.6)
+    hybrid = orc.attention(Q, K, V, kbar, S0, orc.global_first_order(S1), idx, b, 2, 0.6)
+    return float(np.abs(first - hybrid).max())
+
+
+def pin_hybrid_all_selected_is_dense(orc, seed=17):
+    r = _rng(seed)
+    B, H, N, d, b = 1, 1, 30, 4, 8
+    Q, K, V = (r.standard_normal((B, H, N, d)) for _ in range(3))
+    kbar, S0, S1 = orc.block_stats(K, V, b)
+    nB = -(-N // b)
+    out = orc.attention(Q, K, V, kbar, S0, orc.global_first_order(S1), _full_idx(B, H, nB), b, 2, 0.5)
+    return np.abs(out - _textbook(Q, K, V, 0.5)).max()

@@ -38,6 +38,10 @@ def _pins(orc):
         ("permutation_in_block", P.pin_permutation_in_block, lambda e: e < TOL),
         ("order0_convex", P.pin_order0_convex, lambda e: e <= 1e-12),
         ("worked_example", lambda o: P.pin_worked_example(o, EXAMPLE), lambda e: e < TOL),
+        ("drop_is_masked_softmax", P.pin_drop_is_masked_softmax, lambda e: e < TOL),
+        ("hybrid_bruteforce", P.pin_hybrid_bruteforce, lambda e: e < TOL),
+        ("hybrid_shared_first_order", P.pin_hybrid_shared_first_order, lambda e: e < TOL),
+        ("hybrid_all_selected_is_dense", P.pin_hybrid_all_selected_is_dense, lambda e: e < TOL),
     ]:
         try:
             v = fn(orc)
@@ -60,7 +64,8 @@ def real_pins():
     "select_ties", "all_selected_is_dense", "block_one_is_exact", "identical_keys_exact",
     "order0_pseudo_tokens", "first_order_key_form", "linear_in_values",
     "permutation_in_block", "order0_convex", "worked_example",
-    "convergence_order0", "convergence_order1"])
+    "convergence_order0", "convergence_order1", "drop_is_masked_softmax", "hybrid_bruteforce",
+    "hybrid_shared_first_order", "hybrid_all_selected_is_dense"])
 def test_pin(real_pins, name):
     value, ok = real_pins[name]
     assert ok, f"{name}: {value}"
@@ -90,6 +95,12 @@ MUTATIONS = {
     "pooled query over wrong rows": ("Q[:, :, s:e, :].sum(axis=2) / (e - s)",
                                      "Q[:, :, s:s + 1, :].sum(axis=2)"),
     "exact keys from the wrong block": ("for t in range(*bounds[j])]", "for t in range(*bounds[(j + 1) % nB])]"),
+    "drop keeps the zeroth-order terms": ("z_ap = z_ap[:, :0]", "z_ap = z_ap"),
+    "Hbar summed instead of averaged": ("mean(axis=2)", "sum(axis=2)"),
+    "Hbar transposed": ("(X @ S1[b, h])", "(X @ S1[b, h].T)"),
+    "hybrid weight from all blocks": ("* alpha.sum(axis=1)[:, None]",
+                                      "* (alpha.sum(axis=1) + w.sum(axis=1))[:, None]"),
+    "hybrid term dropped": ("num = num + (X @ S1[b, h])", "num = num + 0 * (X @ S1[b, h])"),
 }
 
 
