@@ -139,7 +139,9 @@ def oracle_sample(wl, budget_s: float = 15.0, min_blocks: int = 2):
     q, k, v = W.make_inputs(wl.with_(B=1), heads=[0])
     Qf, Kf, Vf = (W.bf16_bits_to_f32(a).astype(np.float64) for a in (q, k, v))
     t0 = time.perf_counter()
-    kbar, S0, S1 = oracle.block_stats(Kf, Vf, wl.block, wl.order)
+    kbar, S0, S1 = oracle.block_stats(Kf, Vf, wl.block, 1 if wl.order >= 1 else 0)
+    if wl.order == 2:
+        S1 = oracle.global_first_order(S1)
     idx, _, _ = oracle.select(Qf, kbar, wl.block, wl.topk)
     t_pre = time.perf_counter() - t0
     # query blocks spread over the sequence, run until the budget is spent
@@ -266,7 +268,12 @@ def run_ours(args):
     nB = wl.nB
     kbar = torch.empty((wl.B, wl.H, nB, wl.d), device=dev, dtype=torch.float32)
     S0 = torch.empty_like(kbar)
-    S1 = torch.empty((wl.B, wl.H, nB, wl.d, wl.d), device=dev, dtype=torch.bfloat16) if wl.order else None
+    if wl.order == 1:      # per-block first-order matrices
+        S1 = torch.empty((wl.B, wl.H, nB, wl.d, wl.d), device=dev, dtype=torch.bfloat16)
+    elif wl.order == 2:    # the head's global Hbar
+        S1 = torch.empty((wl.B, wl.H, wl.d, wl.d), device=dev, dtype=torch.float32)
+    else:
+        S1 = None
     idx = torch.empty((wl.B, wl.H, nB, wl.topk), device=dev, dtype=torch.int32)
     O = torch.empty_like(Q)
     attn = P.attention if args.kernel == "fused" else P.attention_simt

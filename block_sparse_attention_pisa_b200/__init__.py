@@ -17,8 +17,10 @@ from __future__ import annotations
 import ctypes
 import os
 
+ORDER_DROP, ORDER_ZERO, ORDER_FIRST, ORDER_HYBRID = -1, 0, 1, 2
+
 __all__ = [
-    "PisaError", "Shape", "lib", "block_stats", "select", "attention", "attention_simt",
+    "ORDER_DROP", "ORDER_ZERO", "ORDER_FIRST", "ORDER_HYBRID", "PisaError", "Shape", "lib", "block_stats", "select", "attention", "attention_simt",
     "pisa", "pisa_host", "device_error", "num_blocks", "LIB_PATH", "SYMBOLS",
 ]
 
@@ -104,7 +106,9 @@ def _shape(x, block: int) -> Shape:
 
 
 def block_stats(K, V, block: int, order: int = 1, out=None):
-    """kbar (fp32), S0 (fp32), S1 (bf16, None at order 0) of every key/value block.
+    """kbar (fp32), S0 (fp32) and the first-order statistic of every key/value block:
+    per-block S1 (bf16 [B, H, nB, d, d]) at order 1, the head's Hbar (fp32
+    [B, H, d, d]) at order 2, None at orders 0 and -1.
     ``out`` = (kbar, S0, S1) preallocated outputs (optional)."""
     import torch
     s = _shape(K, block)
@@ -114,8 +118,12 @@ def block_stats(K, V, block: int, order: int = 1, out=None):
     else:
         kbar = torch.empty((s.B, s.H, nB, s.d), device=K.device, dtype=torch.float32)
         S0 = torch.empty_like(kbar)
-        S1 = (torch.empty((s.B, s.H, nB, s.d, s.d), device=K.device, dtype=torch.bfloat16)
-              if order == 1 else None)
+        if order == ORDER_FIRST:
+            S1 = torch.empty((s.B, s.H, nB, s.d, s.d), device=K.device, dtype=torch.bfloat16)
+        elif order == ORDER_HYBRID:
+            S1 = torch.empty((s.B, s.H, s.d, s.d), device=K.device, dtype=torch.float32)
+        else:
+            S1 = None
     _check(lib().pisa_block_stats(_ptr(K), _ptr(V), s, order, _ptr(kbar), _ptr(S0), _ptr(S1),
                                   _stream(K)))
     return kbar, S0, S1
@@ -143,7 +151,8 @@ def _attention(fn, Q, K, V, kbar, S0, S1, idx, block, order, scale, out=None):
 
 
 def attention(Q, K, V, kbar, S0, S1, idx, block: int, order: int, scale: float, out=None):
-    """Fused exact + Taylor attention; bf16 [B, H, N, d]."""
+    """Fused exact + Taylor attention; bf16 [B, H, N, d]. ``order``: -1 keep-or-drop,
+    0 zeroth order, 1 per-block first order (S1 per block), 2 hybrid order (S1 = Hbar)."""
     return _attention(lib().pisa_attention, Q, K, V, kbar, S0, S1, idx, block, order, scale, out)
 
 

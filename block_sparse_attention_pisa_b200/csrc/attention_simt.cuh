@@ -3,7 +3,9 @@
 // Same definition as the fused tensor-core kernel (PISA explainer, technical
 // summary section 2, "Core algorithm": exact sparse term over the critical
 // blocks, zeroth-order term alpha_{t,j} S0_j with alpha = exp(x.kbar_j), and
-// the first-order term alpha_{t,j} S1_j^T x_t; one online-softmax accumulator).
+// the first-order term alpha_{t,j} S1_j^T x_t; one online-softmax accumulator),
+// with the same order codes: -1 keep-or-drop, 0, 1 per-block first order,
+// 2 hybrid order with the global correction (x_t Hbar) sum_U alpha_{t,j}.
 // One CTA per (query block, head), one thread per query row; blocks are visited
 // in ascending order and the accumulator is rescaled whenever the running row
 // maximum grows. Used to cross-check the fused kernel on sizes where the CPU
@@ -32,7 +34,7 @@ __global__ void __launch_bounds__(128)
 attention_simt_kernel(const bf16* __restrict__ Q, const bf16* __restrict__ K,
                       const bf16* __restrict__ V, const float* __restrict__ kbar,
                       const float* __restrict__ S0, const bf16* __restrict__ S1,
-                      const int32_t* __restrict__ idx, int N, int nB, int block, int topk,
+                      const float* __restrict__ hbar, const int32_t* __restrict__ idx, int N, int nB, int block, int topk,
                       int order, float scale, bf16* __restrict__ O) {
   using C = SimtCfg<D>;
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -66,7 +68,7 @@ attention_simt_kernel(const bf16* __restrict__ Q, const bf16* __restrict__ K,
   float acc[D];
 #pragma unroll
   for (int c = 0; c < D; ++c) acc[c] = 0.f;
-  float m = -INFINITY, l = 0.f;
+  float m = -INFINITY, l = 0.f, s_alpha = 0.f;
 
   for (int j = 0; j < nB; ++j) {
     const int s = j * block;
@@ -88,6 +90,7 @@ attention_simt_kernel(const bf16* __restrict__ Q, const bf16* __restrict__ K,
         if (z > m) {
           const float corr = __expf(m - z);
           l *= corr;
+          s_alpha *= corr;
 #pragma unroll
           for (int c = 0; c < D; ++c) acc[c] *= corr;
           m = z;
@@ -97,14 +100,14 @@ attention_simt_kernel(const bf16* __restrict__ Q, const bf16* __restrict__ K,
 #pragma unroll
         for (int c = 0; c < D; ++c) acc[c] = fmaf(p, __bfloat162float(sV[r * D + c]), acc[c]);
       }
-    } else {
+    } else if (order >= 0) {
       const float* gkb = kbar + (bh * size_t(nB) + j) * D;
       const float* gs0 = S0 + (bh * size_t(nB) + j) * D;
       for (int e = t; e < D; e += nthr) {
         sKb[e] = gkb[e];
         sS0[e] = gs0[e];
       }
-      if (order >= 1) {
+      if (order == 1) {
         const bf16* g1 = S1 + (bh * size_t(nB) + j) * size_t(D) * D;
         for (int e = t; e < D * D / 8; e += nthr)
           reinterpret_cast<uint4*>(sS1)[e] = reinterpret_cast<const uint4*>(g1)[e];
@@ -116,21 +119,31 @@ attention_simt_kernel(const bf16* __restrict__ Q, const bf16* __restrict__ K,
       if (z > m) {
         const float corr = __expf(m - z);
         l *= corr;
+        s_alpha *= corr;
 #pragma unroll
         for (int c = 0; c < D; ++c) acc[c] *= corr;
         m = z;
       }
       const float w = __expf(z - m);
       l += float(n) * w;
+      s_alpha += w;
 #pragma unroll
       for (int c = 0; c < D; ++c) acc[c] = fmaf(w, sS0[c], acc[c]);
-      if (order >= 1) {
+      if (order == 1) {
         for (int a = 0; a < D; ++a) {
           const float wx = w * xT[a * C::kMaxRows + t];
 #pragma unroll
           for (int c = 0; c < D; ++c) acc[c] = fmaf(wx, __bfloat162float(sS1[a * D + c]), acc[c]);
         }
       }
+    }
+  }
+  if (order == 2) {
+    const float* gh = hbar + bh * size_t(D) * D;
+    for (int a = 0; a < D; ++a) {
+      const float sx = s_alpha * xT[a * C::kMaxRows + t];
+#pragma unroll
+      for (int c = 0; c < D; ++c) acc[c] = fmaf(sx, __ldg(gh + a * D + c), acc[c]);
     }
   }
   if (valid) {

@@ -8,6 +8,11 @@
 // online softmax with an exact stage over the selected blocks and an
 // approximate stage over the pooled block statistics). The first-order term is
 // the per-block Taylor term alpha_{t,j} S1_j^T x_t with S1_j = sum (k - kbar_j) v^T.
+// Two further treatments of the non-critical blocks share the kernel: the hybrid
+// order of the same section (zeroth order per block plus one global correction
+// (x_t Hbar) sum_{j in U} alpha_{t,j}, Hbar the mean first-order matrix of the
+// head), and keep-or-drop (non-critical blocks contribute nothing; the
+// block-sparse baseline the explainer contrasts PISA with, section 1).
 //
 // One CTA computes a tile of 128 query rows of one head (two query blocks at
 // b = 64, one at b = 128). Warp roles:
@@ -16,8 +21,11 @@
 //   warp 1      MMA issuer (one thread): every tcgen05.mma of the tile;
 //   warps 2-3   build the block lists, then convert fp32 kbar / S0 chunks of 32
 //               blocks into bf16 swizzled shared-memory operands;
-//   warps 4-7   one thread per query row (= TMEM lane): online softmax, the
-//               Taylor weights and the tensor-memory operands.
+//   warps 4-11  two threads per query row (= TMEM lane): warps w and w + 4 share a
+//               lane quarter and each takes half of the row's score columns and
+//               half of O's columns (online softmax, the Taylor weights and the
+//               tensor-memory operands). A pair agrees on its running maximum
+//               through shared memory at one named barrier per block.
 // Tensor memory (512 columns): O accumulator (D), the tile's queries Q (D/2; the A
 // operand of Q K^T and Q Kbar^T), then either a ring of exact score buffers S
 // (P overwrites its own S) or, in the approximate stage, two pooled-score buffers
@@ -27,11 +35,18 @@
 // Exact stage, per block j in the union of the tile's selections:
 //   S = Q K_j^T (TS-MMA), P = exp(x.k - m) (zero for rows whose query block
 //   did not select j and for keys past N), O += P V_j (TS-MMA, V MN-major).
+//   Each half of a row packs P for its own keys into the first half of its own
+//   score columns, so the two halves never touch each other's columns.
 // Approximate stage, per chunk of 32 key blocks that some row approximates:
 //   Sbar = Q Kbar_c^T, alpha = exp(x.kbar - m) (zero for blocks a row's own
 //   query block selected), O += alpha S0_c (zeroth order), and, two blocks per
 //   hand-off, O += A_j S1_j (TS-MMA, S1 MN-major): the first-order term as one
 //   long-K GEMM.
+// Hybrid order: the approximate stage runs at order 0 while each row also sums its
+//   alpha weights (s_t); at the end the converter warps write Hbar as a bf16
+//   operand into the (then idle) first ring stage, the row threads write
+//   A_H = bf16(s_t x_t), and one M128 x D x D MMA adds A_H Hbar to O.
+// Keep-or-drop: no approximate stage at all.
 // Denominator: sum of P plus sum n_j alpha_j, kept in fp32 registers. One running
 // row maximum covers both stages; the accumulator is rescaled only when the
 // maximum grows by more than 2^8 (exact by construction, rare).
@@ -55,6 +70,7 @@ struct TcParams {
   const float* kbar;
   const float* S0;
   const int32_t* idx;
+  const float* hbar;  // hybrid order: fp32 [B*H][D][D]
   bf16* O;
   int N;
   int nB;
@@ -65,10 +81,14 @@ struct TcParams {
 
 template <int D, int BLK>
 struct TcCfg {
-  static constexpr int kThreads = 256;
+  static constexpr int kThreads = 384;
   static constexpr int NS = (D == 128) ? 5 : 10;            // TMA stages
   static constexpr int STAGE = (D == 128) ? 32768 : 16384;  // bytes per stage
   static constexpr int NTF = NS;                            // landed-copy barriers (one per load unit)
+  // K_j and V_j of an exact block share one stage when both fit (b = 64 at d = 128 and
+  // d = 64): twice the blocks in flight for the same shared memory
+  static constexpr bool KV_PACKED = 2 * BLK * D * 2 <= STAGE;
+  static constexpr int TPB = KV_PACKED ? 1 : 2;             // ring stages per exact block
   static constexpr int CHUNK = 32;                          // key blocks per approximate chunk
   static constexpr int CV_HALF = CHUNK * D * 2;             // bf16 kbar (or S0) chunk
   static constexpr int CV_STAGE = 2 * CV_HALF;
@@ -90,20 +110,23 @@ struct TcCfg {
   // barriers
   static constexpr int B_SE = 0;                  // [NS]  stage consumed (MMA commit)
   static constexpr int B_TF = B_SE + NS;          // [NTF] copies of a load unit landed
-  static constexpr int B_Q = B_TF + NTF;          //       queries in TMEM (128 rows)
+  static constexpr int B_Q = B_TF + NTF;          //       queries in TMEM (256 row threads)
   static constexpr int B_SF = B_Q + 1;            // [NSB] S ready (commit)
-  static constexpr int B_PF = B_SF + NSB;         // [NSB] P written (128 rows)
+  static constexpr int B_PF = B_SF + NSB;         // [NSB] P written (256 row threads)
   static constexpr int B_PV = B_PF + NSB;         // [NSB] P V done (commit)
   static constexpr int B_CVF = B_PV + NSB;        // [2]   kbar / S0 chunk converted (64)
   static constexpr int B_CVE = B_CVF + 2;         // [2]   chunk operands consumed (commit)
   static constexpr int B_SBF = B_CVE + 2;         // [2]   Sbar ready (commit)
-  static constexpr int B_A0F = B_SBF + 2;         // [2]   alpha operand written (128)
+  static constexpr int B_A0F = B_SBF + 2;         // [2]   alpha operand written (256)
   static constexpr int B_SBE = B_A0F + 2;         // [2]   alpha MMA done (commit)
-  static constexpr int B_GA = B_SBE + 2;          // [2]   a pair of A_j written (128)
+  static constexpr int B_GA = B_SBE + 2;          // [2]   a pair of A_j written (256)
   static constexpr int B_AE = B_GA + 2;           // [2]   a pair of A_j consumed (commit)
   static constexpr int B_OSYNC = B_AE + 2;        //       end of the exact stage / of a chunk (commit)
   static constexpr int B_ODONE = B_OSYNC + 1;     //       all MMAs done (commit)
-  static constexpr int NBARS = B_ODONE + 1;
+  static constexpr int B_XD = B_ODONE + 1;        //       exact stage done, ring idle (commit; hybrid)
+  static constexpr int B_HF = B_XD + 1;           //       Hbar operand converted (64; hybrid)
+  static constexpr int B_AH = B_HF + 1;           //       A_H = s x written (256; hybrid)
+  static constexpr int NBARS = B_AH + 1;
   // shared memory (offsets from a 1024-byte aligned base)
   static constexpr int OFF_RING = 0;
   static constexpr int OFF_CV = OFF_RING + NS * STAGE;
@@ -112,7 +135,10 @@ struct TcCfg {
   static constexpr int OFF_ACTIVE = OFF_APPROX + 2 * MAXB;  // int16[MAXC]
   static constexpr int OFF_CHUNK = OFF_ACTIVE + 2 * MAXC;   // int32[MAXC + 1]
   static constexpr int OFF_MASK = OFF_CHUNK + 4 * (MAXC + 4);
-  static constexpr int OFF_BAR = OFF_MASK + 2 * (MAXB / 32) * 4;
+  static constexpr int OFF_XCH = OFF_MASK + 2 * (MAXB / 32) * 4;  // float [2 parity][2 half][128] row maxima
+  static constexpr int OFF_XS = OFF_XCH + 2 * 2 * 128 * 4;          // float [2 half][128] alpha sums
+  static constexpr int OFF_XL = OFF_XS + 2 * 128 * 4;               // float [2 half][128] denominators
+  static constexpr int OFF_BAR = OFF_XL + 2 * 128 * 4;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
   static constexpr int SMEM = OFF_MISC + 64 + 1024;  // + alignment slack
   static_assert(OFF_BAR % 8 == 0, "barrier alignment");
@@ -152,11 +178,26 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
   }
 }
 
-// scale one TMEM row of D fp32 columns by f (warp-collective)
-template <int D>
+// named barrier of the two warps of one TMEM lane quarter (64 threads); returns the
+// AND of `ok` over them, so that both warps of a pair take the same exits
+__device__ __forceinline__ bool pair_sync_and(int id, bool ok) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, 64, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(out)
+      : "r"(ok ? 1u : 0u), "r"(id)
+      : "memory");
+  return out != 0;
+}
+
+// scale COLS fp32 TMEM columns of one row by f (warp-collective)
+template <int COLS>
 __device__ __forceinline__ void rescale_row(uint32_t taddr, float f) {
 #pragma unroll
-  for (int ch = 0; ch < D / 16; ++ch) {
+  for (int ch = 0; ch < COLS / 16; ++ch) {
     uint32_t o[16];
     tmem_ld16(taddr + ch * 16, o);
     tmem_wait_ld(o);
@@ -170,7 +211,7 @@ __device__ __forceinline__ void rescale_row(uint32_t taddr, float f) {
 }  // namespace tc
 
 template <int D, int BLK>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
 attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ CUtensorMap tmS1, const TcParams p) {
   using C = TcCfg<D, BLK>;
@@ -204,21 +245,24 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     for (int s = 0; s < C::NTF; ++s) mbar_init(BAR(C::B_TF + s), 1);
     for (int s = 0; s < C::NSB; ++s) {
       mbar_init(BAR(C::B_SF + s), 1);
-      mbar_init(BAR(C::B_PF + s), 128);
+      mbar_init(BAR(C::B_PF + s), 256);
       mbar_init(BAR(C::B_PV + s), 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(BAR(C::B_CVF + s), 64);
       mbar_init(BAR(C::B_CVE + s), 1);
       mbar_init(BAR(C::B_SBF + s), 1);
-      mbar_init(BAR(C::B_A0F + s), 128);
+      mbar_init(BAR(C::B_A0F + s), 256);
       mbar_init(BAR(C::B_SBE + s), 1);
-      mbar_init(BAR(C::B_GA + s), 128);
+      mbar_init(BAR(C::B_GA + s), 256);
       mbar_init(BAR(C::B_AE + s), 1);
     }
-    mbar_init(BAR(C::B_Q), 128);
+    mbar_init(BAR(C::B_Q), 256);
     mbar_init(BAR(C::B_OSYNC), 1);
     mbar_init(BAR(C::B_ODONE), 1);
+    mbar_init(BAR(C::B_XD), 1);
+    mbar_init(BAR(C::B_HF), 64);
+    mbar_init(BAR(C::B_AH), 256);
     misc[1] = 0;
     mbar_init_fence();
   }
@@ -293,7 +337,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       chunk_off[nW] = na;
       misc[2] = ne;
       misc[3] = na;
-      misc[4] = nac;
+      misc[4] = p.order < 0 ? 0 : nac;  // keep-or-drop: no approximate stage
     }
   }
   __syncthreads();
@@ -301,6 +345,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   const uint32_t tmem = uint32_t(misc[0]);
   const int n_exact = misc[2];
   const int n_active = misc[4];
+  const bool hybrid = p.order == 2 && n_active > 0;
 
   if (warp == 0) {
     // ----------------------------------------------------------- TMA producer
@@ -309,17 +354,19 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       bool ok = true;
       for (int e = 0; e < n_exact && ok; ++e, ++u) {
         const int j = exact_list[e];
-        for (int q = 0; q < 2 && ok; ++q)
+        for (int q = 0; q < C::TPB && ok; ++q)
           ok = wait_bounded(BAR(C::B_SE + (t + q) % C::NS), (((t + q) / C::NS) & 1) ^ 1, abort_flag);
         if (!ok) break;
         const uint32_t tf = BAR(C::B_TF + u % C::NTF);
         mbar_arrive_expect_tx(tf, 2 * BLK * D * 2);
-        for (int kv = 0; kv < 2; ++kv, ++t) {
-          const uint32_t dst = base_u + C::OFF_RING + (t % C::NS) * C::STAGE;
+        for (int kv = 0; kv < 2; ++kv) {
+          const uint32_t dst = base_u + C::OFF_RING + ((t + (C::KV_PACKED ? 0 : kv)) % C::NS) * C::STAGE +
+                               (C::KV_PACKED ? kv * BLK * D * 2 : 0);
 #pragma unroll
           for (int pn = 0; pn < D / 64; ++pn)
             tma_load_3d(dst + pn * BLK * 128, kv ? &tmV : &tmK, tf, pn * 64, j * BLK, bh);
         }
+        t += C::TPB;
       }
       if (p.order == 1) {
         for (int ac = 0; ac < n_active && ok; ++ac) {
@@ -359,12 +406,14 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         const int sb = e % C::NSB;
         if (!wait_poll(BAR(C::B_PF + sb), (e / C::NSB) & 1, abort_flag)) return false;
         tc_fence_after();
-        const int sv = (2 * e + 1) % C::NS;
-        const uint32_t vb = base_u + C::OFF_RING + sv * C::STAGE;
+        const int sv = (C::TPB * e + C::TPB - 1) % C::NS;
+        const uint32_t vb = base_u + C::OFF_RING + sv * C::STAGE + (C::KV_PACKED ? BLK * D * 2 : 0);
+        // P of keys [16k, 16k + 16): half (k / (BLK/32)) of the row packed it at the
+        // start of its own score columns
 #pragma unroll
         for (int k = 0; k < BLK / 16; ++k)
-          umma_ts(tmem + C::O_COL, tmem + C::R_COL + sb * BLK + k * 8, sdesc_sw128(vb + k * 2048, BLK * 128, 1024),
-                  idO, (o_acc | uint32_t(k)) ? 1u : 0u);
+          umma_ts(tmem + C::O_COL, tmem + C::R_COL + sb * BLK + (k / (BLK / 32)) * (BLK / 2) + (k % (BLK / 32)) * 8,
+                  sdesc_sw128(vb + k * 2048, BLK * 128, 1024), idO, (o_acc | uint32_t(k)) ? 1u : 0u);
         o_acc = 1;
         umma_commit(BAR(C::B_SE + sv));
         umma_commit(BAR(C::B_PV + sb));
@@ -376,13 +425,13 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         if (e >= C::NSB && !wait_poll(BAR(C::B_PV + sb), ((e - C::NSB) / C::NSB) & 1, abort_flag)) return false;
         if (!wait_poll(BAR(C::B_TF + e % C::NTF), (e / C::NTF) & 1, abort_flag)) return false;
         tc_fence_after();
-        const int sk = (2 * e) % C::NS;
+        const int sk = (C::TPB * e) % C::NS;
         const uint32_t kb = base_u + C::OFF_RING + sk * C::STAGE;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
           umma_ts(tmem + C::R_COL + sb * BLK, tmem + C::Q_COL + k * 8,
                   sdesc_sw128(kb + (k >> 2) * (BLK * 128) + (k & 3) * 32, 16, 1024), idS, k ? 1u : 0u);
-        umma_commit(BAR(C::B_SE + sk));
+        if (!C::KV_PACKED) umma_commit(BAR(C::B_SE + sk));  // a packed stage is released after P V
         umma_commit(BAR(C::B_SF + sb));
         return true;
       };
@@ -394,6 +443,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         if (ok && e + kLook < n_exact) ok = qk(e + kLook);
       }
       umma_commit(BAR(C::B_OSYNC));  // completion 0: end of the exact stage
+      if (hybrid) umma_commit(BAR(C::B_XD));
 
       if (ok && n_active > 0) {
         // the pooled-score and operand columns reuse the exact score buffers
@@ -413,7 +463,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         };
         if (ok) ok = sbar(0);
         int g = 0;               // pair (hand-off) counter
-        int t = 2 * n_exact;     // tile counter
+        int t = C::TPB * n_exact;  // stage-use counter
         int u = n_exact;         // load-unit counter
         for (int ac = 0; ac < n_active && ok; ++ac) {
           const int c = active[ac];
@@ -421,9 +471,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           if (!(ok = wait_poll(BAR(C::B_A0F + b), (ac >> 1) & 1, abort_flag))) break;
           tc_fence_after();
           const uint32_t sb = base_u + C::OFF_CV + b * C::CV_STAGE + C::CV_HALF;
+          // alpha of blocks [16k, 16k + 16): packed by half k of the row at the start of
+          // its own pooled-score columns
 #pragma unroll
           for (int k = 0; k < C::CHUNK / 16; ++k)
-            umma_ts(tmem + C::O_COL, tmem + C::R_COL + b * C::CHUNK + k * 8,
+            umma_ts(tmem + C::O_COL, tmem + C::R_COL + b * C::CHUNK + k * 16,
                     sdesc_sw128(sb + k * 2048, C::CHUNK * 128, 1024), idO, (o_acc | uint32_t(k)) ? 1u : 0u);
           o_acc = 1;
           umma_commit(BAR(C::B_SBE + b));
@@ -452,6 +504,18 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           }
           umma_commit(BAR(C::B_OSYNC));  // completion ac + 1: end of active chunk ac
         }
+        if (ok && hybrid) {
+          // O += A_H Hbar: A_H in the first operand slot, Hbar (MN-major) in ring stage 0
+          ok = wait_poll(BAR(C::B_HF), 0, abort_flag) && wait_poll(BAR(C::B_AH), 0, abort_flag);
+          if (ok) {
+            tc_fence_after();
+            const uint32_t hb = base_u + C::OFF_RING;
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k)
+              umma_ts(tmem + C::O_COL, tmem + C::A_COL0 + k * 8, sdesc_sw128(hb + k * 2048, D * 128, 1024), idO,
+                      1u);
+          }
+        }
       }
       umma_commit(BAR(C::B_ODONE));
       wait_drain(BAR(C::B_ODONE), 0);  // nothing of ours may run on after the CTA frees TMEM
@@ -470,40 +534,90 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       // [CHUNK blocks][D] row-major, 128-byte rows per 64-column panel, 16-byte
       // chunks swizzled by (row % 8): the K-major (kbar) and MN-major (S0) UMMA
       // operand layouts coincide for this row = block, column = d storage
-      for (int q = ct; q < C::CHUNK * (D / 8); q += 64) {
-        const int r = q / (D / 8), c16 = q % (D / 8);
-        uint4 kv = make_uint4(0, 0, 0, 0), sv = make_uint4(0, 0, 0, 0);
-        if (c * C::CHUNK + r < nB) {
-          const float4 k0 = __ldg(reinterpret_cast<const float4*>(gk + r * D + c16 * 8));
-          const float4 k1 = __ldg(reinterpret_cast<const float4*>(gk + r * D + c16 * 8 + 4));
-          const float4 s0 = __ldg(reinterpret_cast<const float4*>(gs + r * D + c16 * 8));
-          const float4 s1 = __ldg(reinterpret_cast<const float4*>(gs + r * D + c16 * 8 + 4));
-          kv = make_uint4(pack_bf16x2(k0.x, k0.y), pack_bf16x2(k0.z, k0.w), pack_bf16x2(k1.x, k1.y),
-                          pack_bf16x2(k1.z, k1.w));
-          sv = make_uint4(pack_bf16x2(s0.x, s0.y), pack_bf16x2(s0.z, s0.w), pack_bf16x2(s1.x, s1.y),
-                          pack_bf16x2(s1.z, s1.w));
+      // all loads of a batch are issued before the first conversion (one L2 round
+      // trip per batch, not per item)
+      constexpr int ITEMS = C::CHUNK * (D / 8) / 64, BATCH = 4;
+      static_assert(ITEMS % BATCH == 0, "converter batches");
+#pragma unroll 1
+      for (int b0 = 0; b0 < ITEMS; b0 += BATCH) {
+        float4 kf[BATCH][2], sf[BATCH][2];
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) {
+          const int q = ct + (b0 + i) * 64;
+          const int r = q / (D / 8), c16 = q % (D / 8);
+          if (c * C::CHUNK + r < nB) {
+            kf[i][0] = __ldg(reinterpret_cast<const float4*>(gk + r * D + c16 * 8));
+            kf[i][1] = __ldg(reinterpret_cast<const float4*>(gk + r * D + c16 * 8 + 4));
+            sf[i][0] = __ldg(reinterpret_cast<const float4*>(gs + r * D + c16 * 8));
+            sf[i][1] = __ldg(reinterpret_cast<const float4*>(gs + r * D + c16 * 8 + 4));
+          } else {
+            kf[i][0] = kf[i][1] = sf[i][0] = sf[i][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
         }
-        const int off = (c16 >> 3) * (C::CHUNK * 128) + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
-        *reinterpret_cast<uint4*>(dk + off) = kv;
-        *reinterpret_cast<uint4*>(ds + off) = sv;
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) {
+          const int q = ct + (b0 + i) * 64;
+          const int r = q / (D / 8), c16 = q % (D / 8);
+          const uint4 kv = make_uint4(pack_bf16x2(kf[i][0].x, kf[i][0].y), pack_bf16x2(kf[i][0].z, kf[i][0].w),
+                                      pack_bf16x2(kf[i][1].x, kf[i][1].y), pack_bf16x2(kf[i][1].z, kf[i][1].w));
+          const uint4 sv = make_uint4(pack_bf16x2(sf[i][0].x, sf[i][0].y), pack_bf16x2(sf[i][0].z, sf[i][0].w),
+                                      pack_bf16x2(sf[i][1].x, sf[i][1].y), pack_bf16x2(sf[i][1].z, sf[i][1].w));
+          const int off = (c16 >> 3) * (C::CHUNK * 128) + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
+          *reinterpret_cast<uint4*>(dk + off) = kv;
+          *reinterpret_cast<uint4*>(ds + off) = sv;
+        }
       }
       fence_proxy_async_smem();
       mbar_arrive(BAR(C::B_CVF + s));
     }
+    if (hybrid && wait_bounded(BAR(C::B_XD), 0, abort_flag)) {
+      // Hbar fp32 [D][D] (row a = key dim, column c = value dim) -> bf16 MN-major
+      // operand in ring stage 0, laid out as a TMA 128-byte-swizzled load of 64-column
+      // panels would place it
+      const float* gh = p.hbar + size_t(bh) * D * D;
+      uint8_t* dh = base + C::OFF_RING;
+      for (int q = ct; q < D * (D / 8); q += 64) {
+        const int r = q / (D / 8), c16 = q % (D / 8);
+        const float4 h0 = __ldg(reinterpret_cast<const float4*>(gh + r * D + c16 * 8));
+        const float4 h1 = __ldg(reinterpret_cast<const float4*>(gh + r * D + c16 * 8 + 4));
+        const uint4 hv = make_uint4(pack_bf16x2(h0.x, h0.y), pack_bf16x2(h0.z, h0.w), pack_bf16x2(h1.x, h1.y),
+                                    pack_bf16x2(h1.z, h1.w));
+        *reinterpret_cast<uint4*>(dh + (c16 >> 3) * (D * 128) + r * 128 + (((c16 & 7) ^ (r & 7)) << 4)) = hv;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(BAR(C::B_HF));
+    }
   } else {
     // ----------------------------------------------------------- row threads
-    const int r = threadIdx.x - 128;                         // row in tile = TMEM lane
-    const uint32_t lrow = uint32_t((warp & 3) * 32) << 16;   // this warp's TMEM lane quarter
+    // Two threads per query row: half 0 (warps 4-7) and half 1 (warps 8-11) of a lane
+    // quarter. Half hf owns score columns [hf * BLK/2, (hf + 1) * BLK/2) of each exact
+    // block, blocks [hf * 16, hf * 16 + 16) of each approximate chunk, and O / Q / A
+    // columns of dimensions [hf * D/2, (hf + 1) * D/2). Both halves hold the same
+    // running maximum m; l and the alpha sum are per-half partial sums.
+    const int rt = threadIdx.x - 128;
+    const int hf = rt >> 7;                                  // column half
+    const int r = rt & 127;                                  // row in tile = TMEM lane
+    const int quarter = warp & 3;
+    const uint32_t lrow = uint32_t(quarter * 32) << 16;      // this warp's TMEM lane quarter
+    const int pair_id = 1 + quarter;                         // named barrier of the pair
     const int grow = tile * 128 + r;
     const bool valid = grow < N;
     const uint32_t* mymask = (kTwo && r >= 64) ? mask + C::MAXB / 32 : mask;
+    float* xmax = reinterpret_cast<float*>(base + C::OFF_XCH);
+    float* xs = reinterpret_cast<float*>(base + C::OFF_XS);
+    float* xl = reinterpret_cast<float*>(base + C::OFF_XL);
+    constexpr int HK = BLK / 2;     // exact keys per half
+    constexpr int HD = D / 2;       // O / value dimensions per half
+    constexpr int HA = D / 4;       // packed bf16 Q / A columns per half
+    constexpr int HC = C::CHUNK / 2;
     bool ok = true;
 
-    // queries -> TMEM (the A operand of Q K^T and Q Kbar^T)
+    // queries -> TMEM (the A operand of Q K^T and Q Kbar^T): this half's dimensions
     {
-      const uint4* src = reinterpret_cast<const uint4*>(p.Q + (size_t(bh) * N + (valid ? grow : 0)) * D);
+      const uint4* src =
+          reinterpret_cast<const uint4*>(p.Q + (size_t(bh) * N + (valid ? grow : 0)) * D + hf * HD);
 #pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) {
+      for (int ch = 0; ch < HA / 16; ++ch) {
         uint32_t t[16];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -513,7 +627,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           t[4 * i + 2] = v.z;
           t[4 * i + 3] = v.w;
         }
-        tmem_st16(tmem + lrow + C::Q_COL + ch * 16, t);
+        tmem_st16(tmem + lrow + C::Q_COL + hf * HA + ch * 16, t);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -522,184 +636,247 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
 
     const float sl2 = p.scale * 1.4426950408889634f;  // exponents in base 2
     float m = -INFINITY, l = 0.f;
+    float s_alpha = 0.f;  // hybrid order: this half's sum of alpha weights (same frame as l)
 
     // ------------------------------------------------ exact stage
     for (int e = 0; e < n_exact; ++e) {
       const int j = exact_list[e], sb = e % C::NSB;
       const bool sel = (mymask[j >> 5] >> (j & 31)) & 1u;  // uniform per warp
-      const int nj = min(BLK, N - j * BLK);
-      ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SF + sb), (e / C::NSB) & 1, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t sa = tmem + lrow + C::R_COL + sb * BLK;
-      uint32_t s[BLK];
+      const int nmine = min(HK, N - j * BLK - hf * HK);     // this half's real keys (may be <= 0)
+      if (ok) ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SF + sb), (e / C::NSB) & 1, abort_flag));
+      uint32_t s[HK];
+      const uint32_t sa = tmem + lrow + C::R_COL + sb * BLK + hf * HK;
+      float pm = -INFINITY;
+      if (ok) {
+        tc_fence_after();
 #pragma unroll
-      for (int ch = 0; ch < BLK / 16; ++ch) tmem_ld16(sa + ch * 16, *reinterpret_cast<uint32_t(*)[16]>(&s[ch * 16]));
+        for (int ch = 0; ch < HK / 16; ++ch) tmem_ld16(sa + ch * 16, *reinterpret_cast<uint32_t(*)[16]>(&s[ch * 16]));
 #pragma unroll
-      for (int ch = 0; ch < BLK / 16; ++ch) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&s[ch * 16]));
-      // (independent partial maxima: one warp per SMSP cannot hide a serial chain)
-      float mxp[8];
+        for (int ch = 0; ch < HK / 16; ++ch) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&s[ch * 16]));
+        if (nmine < HK) {  // ragged last block: keys past N take no weight
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mxp[i] = -INFINITY;
+          for (int k = 0; k < HK; ++k)
+            if (k >= nmine) s[k] = __float_as_uint(-INFINITY);
+        }
+        if (sel) {
+          // raw-score maximum (the positive scale commutes with it); independent partial
+          // maxima, because one warp per scheduler cannot hide a serial chain
+          float mxp[8];
 #pragma unroll
-      for (int k = 0; k < BLK; ++k) {
-        const float v = (sel && k < nj) ? __uint_as_float(s[k]) * sl2 : -INFINITY;
-        s[k] = __float_as_uint(v);
-        mxp[k & 7] = fmaxf(mxp[k & 7], v);
+          for (int i = 0; i < 8; ++i) mxp[i] = -INFINITY;
+#pragma unroll
+          for (int k = 0; k < HK; ++k) mxp[k & 7] = fmaxf(mxp[k & 7], __uint_as_float(s[k]));
+          pm = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                     fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+        }
       }
-      const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
-                             fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+      xmax[((e & 1) * 2 + hf) * 128 + r] = pm;
+      ok = pair_sync_and(pair_id, ok);
+      if (!ok) break;
+      const float mx = fmaxf(pm, xmax[((e & 1) * 2 + (hf ^ 1)) * 128 + r]) * sl2;
       const bool grow_max = mx > m + 8.f;          // false for rows that did not select j
       const bool need_o = grow_max && m != -INFINITY;
       if (__any_sync(0xffffffffu, need_o)) {
-        if (e >= 1) {
+        if (e >= 1)
           ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_PV + (e - 1) % C::NSB), ((e - 1) / C::NSB) & 1,
                                                     abort_flag));
-          if (!ok) break;
+        if (ok) {
+          tc_fence_after();
+          const float f = need_o ? ex2(m - mx) : 1.f;
+          rescale_row<HD>(tmem + lrow + C::O_COL + hf * HD, f);
+          l *= f;
         }
-        tc_fence_after();
-        const float f = need_o ? ex2(m - mx) : 1.f;
-        rescale_row<D>(tmem + lrow + C::O_COL, f);
-        l *= f;
       }
       if (grow_max) m = mx;
       float rsp[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[HK / 2];
+      if (sel) {
+        const float negm = -m;
 #pragma unroll
-      for (int ch = 0; ch < BLK / 32; ++ch) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          // rows whose query block did not select j take no exact weight (m may
-          // still be -inf for them, so no exponential is evaluated)
-          const float p0 = sel ? ex2(__uint_as_float(s[ch * 32 + 2 * i]) - m) : 0.f;
-          const float p1 = sel ? ex2(__uint_as_float(s[ch * 32 + 2 * i + 1]) - m) : 0.f;
+        for (int i = 0; i < HK / 2; ++i) {
+          const float p0 = ex2(fmaf(__uint_as_float(s[2 * i]), sl2, negm));
+          const float p1 = ex2(fmaf(__uint_as_float(s[2 * i + 1]), sl2, negm));
           rsp[i & 3] += p0 + p1;
           pk[i] = pack_bf16x2_int(p0, p1);
         }
-        tmem_st16(sa + ch * 16, pk);
+      } else {
+        // rows whose query block did not select j take no exact weight (m may still be
+        // -inf for them, so no exponential is evaluated)
+#pragma unroll
+        for (int i = 0; i < HK / 2; ++i) pk[i] = 0u;
       }
+#pragma unroll
+      for (int ch = 0; ch < HK / 32; ++ch) tmem_st16(sa + ch * 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[ch * 16]));
       l += (rsp[0] + rsp[1]) + (rsp[2] + rsp[3]);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(BAR(C::B_PF + sb));
     }
+    ok = pair_sync_and(pair_id, ok);
 
     // ------------------------------------------------ approximate stage
     if (ok && n_active > 0) {
       // every exact-stage MMA is done: the operand slots may reuse their columns
       ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_OSYNC), 0, abort_flag));
-      uint32_t q[D / 2];
+      uint32_t q[HA];  // this half's packed query dimensions
       if (ok) {
         tc_fence_after();
 #pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch)
-          tmem_ld16(tmem + lrow + C::Q_COL + ch * 16, *reinterpret_cast<uint32_t(*)[16]>(&q[ch * 16]));
+        for (int ch = 0; ch < HA / 16; ++ch)
+          tmem_ld16(tmem + lrow + C::Q_COL + hf * HA + ch * 16, *reinterpret_cast<uint32_t(*)[16]>(&q[ch * 16]));
 #pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&q[ch * 16]));
+        for (int ch = 0; ch < HA / 16; ++ch) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&q[ch * 16]));
       }
       const int nlast = N - (nB - 1) * BLK;
+      const bool first = p.order == 1;
       int g = 0;
-      for (int ac = 0; ac < n_active && ok; ++ac) {
+      for (int ac = 0; ac < n_active; ++ac) {
         const int c = active[ac];
         const int b = ac & 1;
-        ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SBF + b), (ac >> 1) & 1, abort_flag));
+        if (ok) ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SBF + b), (ac >> 1) & 1, abort_flag));
+        const uint32_t sa = tmem + lrow + C::R_COL + b * C::CHUNK;
+        uint32_t sv[C::CHUNK];   // both halves read all pooled scores of the chunk
+        float mx = -INFINITY;
+        if (ok) {
+          tc_fence_after();
+          tmem_ld16(sa, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
+          tmem_ld16(sa + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
+          tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
+          tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
+          const uint32_t myw = mymask[c];
+          const int kmax = nB - c * C::CHUNK;  // blocks of this chunk that exist
+          float mxp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int k = 0; k < C::CHUNK; ++k) {
+            const bool mine = k < kmax && !((myw >> k) & 1u);
+            const float v = mine ? __uint_as_float(sv[k]) * sl2 : -INFINITY;
+            sv[k] = __float_as_uint(v);
+            mxp[k & 3] = fmaxf(mxp[k & 3], v);
+          }
+          mx = fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3]));
+          tc_fence_before();
+        }
+        // both halves have read the chunk's pooled scores before either overwrites them
+        ok = pair_sync_and(pair_id, ok);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t sa = tmem + lrow + C::R_COL + b * C::CHUNK;
-        uint32_t sv[C::CHUNK];
-        tmem_ld16(sa, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
-        tmem_ld16(sa + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
-        tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
-        tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
-        const uint32_t myw = mymask[c];
-        const int kmax = nB - c * C::CHUNK;  // blocks of this chunk that exist
-        float mxp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int k = 0; k < C::CHUNK; ++k) {
-          const bool mine = k < kmax && !((myw >> k) & 1u);
-          const float v = mine ? __uint_as_float(sv[k]) * sl2 : -INFINITY;
-          sv[k] = __float_as_uint(v);
-          mxp[k & 3] = fmaxf(mxp[k & 3], v);
-        }
-        const float mx = fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3]));
         const bool need_o = mx > m + 8.f;
         if (__any_sync(0xffffffffu, need_o)) {
           ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_OSYNC), ac & 1, abort_flag));
-          if (!ok) break;
-          tc_fence_after();
-          const float f = need_o ? ex2(m - mx) : 1.f;
-          rescale_row<D>(tmem + lrow + C::O_COL, f);
-          l *= f;
+          if (ok) {
+            tc_fence_after();
+            const float f = need_o ? ex2(m - mx) : 1.f;
+            rescale_row<HD>(tmem + lrow + C::O_COL + hf * HD, f);
+            l *= f;
+            s_alpha *= f;
+          }
           if (need_o) m = mx;
         }
+        // alpha of this half's blocks (and, at order 1, of the other half's: the
+        // first-order operands of every approximated block need them)
         float lsp[4] = {0.f, 0.f, 0.f, 0.f};
-        uint32_t a0[C::CHUNK / 2];
+        float ssp[2] = {0.f, 0.f};
+        uint32_t a0[HC / 2], a1[HC / 2];  // packed alpha: own blocks, other half's blocks
 #pragma unroll
-        for (int k = 0; k < C::CHUNK; k += 2) {
-          const float x0 = ex2(__uint_as_float(sv[k]) - m);
-          const float x1 = ex2(__uint_as_float(sv[k + 1]) - m);
-          const float n0 = (c * C::CHUNK + k == nB - 1) ? float(nlast) : float(BLK);
-          const float n1 = (c * C::CHUNK + k + 1 == nB - 1) ? float(nlast) : float(BLK);
+        for (int k = 0; k < HC; k += 2) {
+          const int kk = hf * HC + k;
+          const float x0 = ex2(__uint_as_float(sv[kk]) - m);
+          const float x1 = ex2(__uint_as_float(sv[kk + 1]) - m);
+          const float n0 = (c * C::CHUNK + kk == nB - 1) ? float(nlast) : float(BLK);
+          const float n1 = (c * C::CHUNK + kk + 1 == nB - 1) ? float(nlast) : float(BLK);
           lsp[(k >> 1) & 3] = fmaf(n1, x1, fmaf(n0, x0, lsp[(k >> 1) & 3]));
+          ssp[(k >> 1) & 1] += x0 + x1;
           a0[k >> 1] = pack_bf16x2_int(x0, x1);
         }
         l += (lsp[0] + lsp[1]) + (lsp[2] + lsp[3]);
-        tmem_st16(sa, a0);
-        tmem_wait_st();
-        tc_fence_before();
+        s_alpha += ssp[0] + ssp[1];
+        if (ok) {
+          tmem_st8(sa + hf * HC, a0);
+          tmem_wait_st();
+          tc_fence_before();
+        }
         mbar_arrive(BAR(C::B_A0F + b));
 
-        if (p.order == 1) {
+        if (first && ok) {
+#pragma unroll
+          for (int k = 0; k < HC; k += 2) {
+            const int kk = (hf ^ 1) * HC + k;
+            a1[k >> 1] = pack_bf16x2_int(ex2(__uint_as_float(sv[kk]) - m), ex2(__uint_as_float(sv[kk + 1]) - m));
+          }
           // one runtime iteration per pair of approximated blocks (kept rolled: an
           // unrolled copy evicts the MMA warp's instructions). alpha comes from the
-          // packed bf16 operand a0 (zero where the row's own block is exact).
+          // packed bf16 weights (zero where the row's own block is exact).
           const int a_end = chunk_off[c + 1];
 #pragma unroll 1
           for (int a = chunk_off[c]; a < a_end; a += C::GROUP, ++g) {
             const int n = min(C::GROUP, a_end - a);
             const int gs = g & 1;
-            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_AE + gs), ((g >> 1) & 1) ^ 1, abort_flag));
-            if (!ok) break;
-            tc_fence_after();
+            if (ok) ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_AE + gs), ((g >> 1) & 1) ^ 1, abort_flag));
+            if (ok) {
+              tc_fence_after();
 #pragma unroll 1
-            for (int qq = 0; qq < n; ++qq) {
-              const int k = approx_list[a + qq] - c * C::CHUNK;
-              const uint32_t w = a0[k >> 1];
-              const float coef = ((k & 1) ? bf16_hi(w) : bf16_lo(w)) * p.scale;
-              const __nv_bfloat162 c2 = __floats2bfloat162_rn(coef, coef);
-              const uint32_t cw = *reinterpret_cast<const uint32_t*>(&c2);
-              const uint32_t aa = tmem + lrow + C::A_COL0 + (gs * C::GROUP + qq) * C::A_COLS;
+              for (int qq = 0; qq < n; ++qq) {
+                const int k = approx_list[a + qq] - c * C::CHUNK;
+                const bool own = (k >> 4) == hf;
+                const int kl = k & (HC - 1);
+                const uint32_t w = own ? a0[kl >> 1] : a1[kl >> 1];
+                const float coef = ((kl & 1) ? bf16_hi(w) : bf16_lo(w)) * p.scale;
+                const __nv_bfloat162 c2 = __floats2bfloat162_rn(coef, coef);
+                const uint32_t cw = *reinterpret_cast<const uint32_t*>(&c2);
+                const uint32_t aa = tmem + lrow + C::A_COL0 + (gs * C::GROUP + qq) * C::A_COLS + hf * HA;
 #pragma unroll
-              for (int ch = 0; ch < D / 32; ++ch) {
-                uint32_t t[16];
+                for (int ch = 0; ch < HA / 16; ++ch) {
+                  uint32_t t[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) t[i] = hmul2_bf16(q[ch * 16 + i], cw);
-                tmem_st16(aa + ch * 16, t);
+                  for (int i = 0; i < 16; ++i) t[i] = hmul2_bf16(q[ch * 16 + i], cw);
+                  tmem_st16(aa + ch * 16, t);
+                }
               }
+              tmem_wait_st();
+              tc_fence_before();
+              // the pair's S1 tiles (load unit n_exact + g) must have landed as well
+              const int u = n_exact + g;
+              ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_TF + u % C::NTF), (u / C::NTF) & 1, abort_flag));
             }
-            tmem_wait_st();
-            tc_fence_before();
-            // the pair's S1 tiles (load unit n_exact + g) must have landed as well
-            const int u = n_exact + g;
-            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_TF + u % C::NTF), (u / C::NTF) & 1, abort_flag));
-            if (!ok) break;
             mbar_arrive(BAR(C::B_GA + gs));
           }
+        }
+      }
+      if (hybrid) {
+        // A_H = bf16(s_t * scale * q_t), one rounding from fp32 (operand slot 0); s_t is
+        // the sum of both halves' alpha weights
+        xs[hf * 128 + r] = s_alpha;
+        ok = pair_sync_and(pair_id, ok);
+        if (ok) {
+          const float coef = (s_alpha + xs[(hf ^ 1) * 128 + r]) * p.scale;
+#pragma unroll
+          for (int ch = 0; ch < HA / 16; ++ch) {
+            uint32_t t[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              t[i] = pack_bf16x2(bf16_lo(q[ch * 16 + i]) * coef, bf16_hi(q[ch * 16 + i]) * coef);
+            tmem_st16(tmem + lrow + C::A_COL0 + hf * HA + ch * 16, t);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(BAR(C::B_AH));
         }
       }
     }
 
     // ------------------------------------------------ epilogue
+    xl[hf * 128 + r] = l;
+    ok = pair_sync_and(pair_id, ok);
     if (ok) {
       ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_ODONE), 0, abort_flag));
       if (ok) {
         tc_fence_after();
-        const float inv = 1.f / l;
-        bf16* dst = p.O + (size_t(bh) * N + (valid ? grow : 0)) * D;
+        const float inv = 1.f / (l + xl[(hf ^ 1) * 128 + r]);
+        bf16* dst = p.O + (size_t(bh) * N + (valid ? grow : 0)) * D + hf * HD;
 #pragma unroll
-        for (int ch = 0; ch < D / 16; ++ch) {
+        for (int ch = 0; ch < HD / 16; ++ch) {
           uint32_t o[16];
-          tmem_ld16(tmem + lrow + C::O_COL + ch * 16, o);
+          tmem_ld16(tmem + lrow + C::O_COL + hf * HD + ch * 16, o);
           tmem_wait_ld(o);
           uint4 w0, w1;
           w0.x = pack_bf16x2(__uint_as_float(o[0]) * inv, __uint_as_float(o[1]) * inv);

@@ -74,7 +74,8 @@ pisa_status_t check_ptr(const void* p, const char* name) {
 }
 
 pisa_status_t check_order(int32_t order) {
-  if (order != 0 && order != 1) return fail(PISA_ERR_INVALID_ARG, "order=%d (must be 0 or 1)", order);
+  if (order < PISA_ORDER_DROP || order > PISA_ORDER_HYBRID)
+    return fail(PISA_ERR_INVALID_ARG, "order=%d (must be -1, 0, 1 or 2)", order);
   return ok();
 }
 
@@ -128,13 +129,25 @@ pisa_status_t set_smem(Kernel k, size_t bytes) {
 
 template <int D, int BLK>
 pisa_status_t launch_stats(const pisa_shape_t& s, const bf16* K, const bf16* V, int order, float* kbar,
-                           float* S0, bf16* S1, cudaStream_t st) {
+                           float* S0, void* S1, cudaStream_t st) {
   using C = pisa::StatsCfg<D, BLK>;
+  const int nB = int(num_blocks(s));
+  if (order == PISA_ORDER_HYBRID) {
+    // Hbar is accumulated with atomics: zero it first, on the same stream
+    const size_t bytes = size_t(s.B) * s.H * D * D * sizeof(float);
+    cudaError_t e = cudaMemsetAsync(S1, 0, bytes, st);
+    if (e != cudaSuccess) return fail(PISA_ERR_CUDA, "cudaMemsetAsync(Hbar): %s", cudaGetErrorString(e));
+    auto k = pisa::stats_hbar_kernel<D, BLK>;
+    using H = pisa::HbarCfg<D, BLK>;
+    PISA_TRY(set_smem(k, H::kSmem));
+    dim3 grid((nB + pisa::kHbarBlocks - 1) / pisa::kHbarBlocks, s.B * s.H);
+    k<<<grid, C::kThreads, H::kSmem, st>>>(K, V, s.N, nB, kbar, S0, static_cast<float*>(S1));
+    return check_launch("stats_hbar_kernel");
+  }
   auto k = pisa::stats_kernel<D, BLK>;
   PISA_TRY(set_smem(k, C::kSmem));
-  const int nB = int(num_blocks(s));
   dim3 grid(nB, s.B * s.H);
-  k<<<grid, C::kThreads, C::kSmem, st>>>(K, V, s.N, nB, order, kbar, S0, S1);
+  k<<<grid, C::kThreads, C::kSmem, st>>>(K, V, s.N, nB, order, kbar, S0, static_cast<bf16*>(S1));
   return check_launch("stats_kernel");
 }
 
@@ -152,14 +165,16 @@ pisa_status_t launch_select(const pisa_shape_t& s, const bf16* Q, const float* k
 
 template <int D>
 pisa_status_t launch_attention_simt(const pisa_shape_t& s, const bf16* Q, const bf16* K, const bf16* V,
-                                    const float* kbar, const float* S0, const bf16* S1, const int32_t* idx,
+                                    const float* kbar, const float* S0, const void* S1, const int32_t* idx,
                                     int topk, int order, float scale, bf16* O, cudaStream_t st) {
   auto k = pisa::attention_simt_kernel<D>;
   const size_t smem = pisa::SimtCfg<D>::smem_bytes();
   PISA_TRY(set_smem(k, smem));
   const int nB = int(num_blocks(s));
   dim3 grid(nB, s.B * s.H);
-  k<<<grid, s.block, smem, st>>>(Q, K, V, kbar, S0, S1, idx, s.N, nB, s.block, topk, order, scale, O);
+  const bf16* s1 = order == PISA_ORDER_FIRST ? static_cast<const bf16*>(S1) : nullptr;
+  const float* hbar = order == PISA_ORDER_HYBRID ? static_cast<const float*>(S1) : nullptr;
+  k<<<grid, s.block, smem, st>>>(Q, K, V, kbar, S0, s1, hbar, idx, s.N, nB, s.block, topk, order, scale, O);
   return check_launch("attention_simt_kernel");
 }
 
@@ -195,7 +210,7 @@ pisa_status_t make_map(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1
 
 template <int D, int BLK>
 pisa_status_t launch_attention_tc(const pisa_shape_t& s, const bf16* Q, const bf16* K, const bf16* V,
-                                  const float* kbar, const float* S0, const bf16* S1, const int32_t* idx, int topk,
+                                  const float* kbar, const float* S0, const void* S1, const int32_t* idx, int topk,
                                   int order, float scale, bf16* O, cudaStream_t st) {
   using C = pisa::TcCfg<D, BLK>;
   const int nB = int(num_blocks(s));
@@ -203,11 +218,12 @@ pisa_status_t launch_attention_tc(const pisa_shape_t& s, const bf16* Q, const bf
   CUtensorMap mK, mV, mS1;
   PISA_TRY(make_map(&mK, K, D, uint64_t(s.N), BH, BLK));
   PISA_TRY(make_map(&mV, V, D, uint64_t(s.N), BH, BLK));
-  if (order == 1) PISA_TRY(make_map(&mS1, S1, D, D, BH * nB, D));
-  else mS1 = mK;  // never read at order 0
+  if (order == PISA_ORDER_FIRST) PISA_TRY(make_map(&mS1, S1, D, D, BH * nB, D));
+  else mS1 = mK;  // never read at the other orders
   auto k = pisa::attention_tc_kernel<D, BLK>;
   PISA_TRY(set_smem(k, C::SMEM));
-  pisa::TcParams p{Q, kbar, S0, idx, O, s.N, nB, topk, order, scale};
+  const float* hbar = order == PISA_ORDER_HYBRID ? static_cast<const float*>(S1) : nullptr;
+  pisa::TcParams p{Q, kbar, S0, idx, hbar, O, s.N, nB, topk, order, scale};
   dim3 grid((s.N + 127) / 128, unsigned(BH));
   k<<<grid, C::kThreads, C::SMEM, st>>>(mK, mV, mS1, p);
   return check_launch("attention_tc_kernel");
@@ -233,12 +249,15 @@ pisa_status_t validate_attention(const pisa_shape_t& shape, const AttnArgs& a, b
   PISA_TRY(check_ptr(a.Q, "Q"));
   PISA_TRY(check_ptr(a.K, "K"));
   PISA_TRY(check_ptr(a.V, "V"));
-  PISA_TRY(check_ptr(a.kbar, "kbar"));
-  PISA_TRY(check_ptr(a.S0, "S0"));
   PISA_TRY(check_ptr(a.idx, "idx"));
   PISA_TRY(check_ptr(a.O, "O"));
   PISA_TRY(check_order(a.order));
-  if (a.order == 1) PISA_TRY(check_ptr(a.S1, "S1"));
+  if (a.order != PISA_ORDER_DROP) {
+    PISA_TRY(check_ptr(a.kbar, "kbar"));
+    PISA_TRY(check_ptr(a.S0, "S0"));
+  }
+  if (a.order == PISA_ORDER_FIRST) PISA_TRY(check_ptr(a.S1, "S1"));
+  if (a.order == PISA_ORDER_HYBRID) PISA_TRY(check_ptr(a.S1, "Hbar (S1)"));
   PISA_TRY(check_topk(shape, a.topk));
   if (!std::isfinite(a.scale) || !(a.scale > 0.f))
     return fail(PISA_ERR_INVALID_ARG, "scale=%g (must be finite and > 0)", double(a.scale));
@@ -259,18 +278,18 @@ pisa_status_t pisa_block_stats(const void* K, const void* V, pisa_shape_t shape,
   PISA_TRY(check_ptr(kbar, "kbar"));
   PISA_TRY(check_ptr(S0, "S0"));
   PISA_TRY(check_order(order));
-  if (order == 1) PISA_TRY(check_ptr(S1, "S1"));
+  if (order == PISA_ORDER_FIRST) PISA_TRY(check_ptr(S1, "S1"));
+  if (order == PISA_ORDER_HYBRID) PISA_TRY(check_ptr(S1, "Hbar (S1)"));
   PISA_TRY(check_support(shape));
   int sms = 0;
   PISA_TRY(check_device(&sms));
   auto st = static_cast<cudaStream_t>(stream);
   auto k = static_cast<const bf16*>(K);
   auto v = static_cast<const bf16*>(V);
-  auto s1 = static_cast<bf16*>(S1);
-  if (shape.d == 128 && shape.block == 64) return launch_stats<128, 64>(shape, k, v, order, kbar, S0, s1, st);
-  if (shape.d == 128 && shape.block == 128) return launch_stats<128, 128>(shape, k, v, order, kbar, S0, s1, st);
-  if (shape.d == 64 && shape.block == 64) return launch_stats<64, 64>(shape, k, v, order, kbar, S0, s1, st);
-  return launch_stats<64, 128>(shape, k, v, order, kbar, S0, s1, st);
+  if (shape.d == 128 && shape.block == 64) return launch_stats<128, 64>(shape, k, v, order, kbar, S0, S1, st);
+  if (shape.d == 128 && shape.block == 128) return launch_stats<128, 128>(shape, k, v, order, kbar, S0, S1, st);
+  if (shape.d == 64 && shape.block == 64) return launch_stats<64, 64>(shape, k, v, order, kbar, S0, S1, st);
+  return launch_stats<64, 128>(shape, k, v, order, kbar, S0, S1, st);
 }
 
 pisa_status_t pisa_select(const void* Q, const float* kbar, pisa_shape_t shape, int32_t topk, int32_t* idx,
@@ -304,7 +323,7 @@ pisa_status_t pisa_attention(const void* Q, const void* K, const void* V, const 
   auto q = static_cast<const bf16*>(Q);
   auto k = static_cast<const bf16*>(K);
   auto v = static_cast<const bf16*>(V);
-  auto s1 = static_cast<const bf16*>(S1);
+  const void* s1 = S1;
   auto o = static_cast<bf16*>(O);
   if (shape.d == 128 && shape.block == 64)
     return launch_attention_tc<128, 64>(shape, q, k, v, kbar, S0, s1, idx, topk, order, scale, o, st);
@@ -328,7 +347,7 @@ pisa_status_t pisa_attention_simt(const void* Q, const void* K, const void* V, c
   auto q = static_cast<const bf16*>(Q);
   auto k = static_cast<const bf16*>(K);
   auto v = static_cast<const bf16*>(V);
-  auto s1 = static_cast<const bf16*>(S1);
+  const void* s1 = S1;
   auto o = static_cast<bf16*>(O);
   if (shape.d == 128) return launch_attention_simt<128>(shape, q, k, v, kbar, S0, s1, idx, topk, order, scale, o, st);
   return launch_attention_simt<64>(shape, q, k, v, kbar, S0, s1, idx, topk, order, scale, o, st);

@@ -17,6 +17,15 @@
 // The kernel is HBM-bound (K, V in; S1 out). The d x b x d contraction is ~32
 // flop/byte, below the tensor ridge, so the warp-level mma.sync path keeps it
 // under the memory time.
+//
+// Hybrid order (section 2, "Core algorithm": one global first-order statistic
+// Hbar, the mean of the per-block first-order matrices over all blocks of a head;
+// "Hardware implementation": formed in the precompute step). stats_hbar_kernel
+// gives each CTA kHbarBlocks consecutive blocks of one head, keeps the sum of
+// their S1_j (formed exactly as above, in fp32) in registers and adds it, scaled
+// by 1/nB, into the fp32 Hbar of the head with vector atomics. Per-block S1 is
+// never written, so the kernel moves K and V in and little else out. The fp32
+// atomic sum makes Hbar reproducible to fp32 rounding, not bit for bit.
 #pragma once
 
 #include "common.cuh"
@@ -37,31 +46,18 @@ struct StatsCfg {
                                   + size_t(2) * D * sizeof(float);       // kbar, S0
 };
 
+// Streams block j (n real rows; rows >= n are zero-filled) into sK / sV, and
+// writes its centroid and value sum to sKbar / sS0 and to global memory. Ends
+// with the block's shared-memory tiles and sums visible to the whole CTA.
 template <int D, int BLK>
-__global__ void __launch_bounds__(256, 3)
-stats_kernel(const bf16* __restrict__ K, const bf16* __restrict__ V, int N, int nB, int order,
-             float* __restrict__ kbar, float* __restrict__ S0, bf16* __restrict__ S1) {
+__device__ __forceinline__ void load_block_and_sums(const bf16* __restrict__ gK, const bf16* __restrict__ gV,
+                                                    int n, bf16* sK, bf16* sV, float* sPart, float* sKbar,
+                                                    float* sS0, float* __restrict__ kbar_out,
+                                                    float* __restrict__ S0_out) {
   using C = StatsCfg<D, BLK>;
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  bf16* sK = reinterpret_cast<bf16*>(smem_raw);
-  bf16* sV = sK + C::kTileElems;
-  bf16* sStage = sV + C::kTileElems;                            // [D][kStageLd]
-  float* sPart = reinterpret_cast<float*>(sStage + D * C::kStageLd);  // [8 warps][2][D]
-  float* sKbar = sPart + 8 * 2 * D;
-  float* sS0 = sKbar + D;
-
-  const int j = blockIdx.x;
-  const size_t bh = blockIdx.y;
-  const int start = j * BLK;
-  const int n = min(BLK, N - start);
-  const bf16* gK = K + (bh * size_t(N) + start) * D;
-  const bf16* gV = V + (bh * size_t(N) + start) * D;
-
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int ch = tid % C::kChunks;
   const int r0 = tid / C::kChunks;
-
-  // ---- stream K_j, V_j once (rows >= n are zero-filled) and sum columns ----
   float ks[8], vs[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) ks[e] = vs[e] = 0.f;
@@ -103,25 +99,86 @@ stats_kernel(const bf16* __restrict__ K, const bf16* __restrict__ V, int N, int 
   __syncthreads();
   if (tid < 2 * D) {
     const int which = tid / D, col = tid % D;
-    float s = 0.f;
+    float sum = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) s += sPart[(w * 2 + which) * D + col];
-    const size_t o = (bh * size_t(nB) + j) * D + col;
+    for (int w = 0; w < 8; ++w) sum += sPart[(w * 2 + which) * D + col];
     if (which == 0) {
-      const float kb = s / float(n);
+      const float kb = sum / float(n);
       sKbar[col] = kb;
-      kbar[o] = kb;
+      kbar_out[col] = kb;
     } else {
-      sS0[col] = s;
-      S0[o] = s;
+      sS0[col] = sum;
+      S0_out[col] = sum;
     }
   }
-  if (order == 0) return;
   __syncthreads();
+}
+
+// One pass of K_j^T V_j over half of the value dimension on the tensor cores:
+// acc (warp tile D/4 x D/4 of the key x value-half plane, 8 warps as 4 x 2) +=
+// the block's products. Operands from the padded shared-memory tiles.
+template <int D, int BLK>
+__device__ __forceinline__ void s1_half_mma(uint32_t sK_u, uint32_t sV_u, int pass,
+                                            float (&acc)[D / 64][D / 32][4]) {
+  using C = StatsCfg<D, BLK>;
+  constexpr int TM = D / 4, TN = D / 4;
+  constexpr int MT = TM / 16, NT = TN / 8;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int a_base = (warp >> 1) * TM;
+  const int c_base = pass * (D / 2) + (warp & 1) * TN;
+#pragma unroll
+  for (int kt = 0; kt < BLK / 16; ++kt) {
+    uint32_t af[MT][4];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      // A[a][n] = K[n][a]: transposed 8x8 loads from rows n, columns a
+      const int row = kt * 16 + (lane & 7) + ((lane >> 4) << 3);
+      const int col = a_base + mt * 16 + (((lane >> 3) & 1) << 3);
+      ldsm_x4_trans(sK_u + (row * C::kLd + col) * 2, af[mt][0], af[mt][1], af[mt][2], af[mt][3]);
+    }
+#pragma unroll
+    for (int np = 0; np < NT / 2; ++np) {
+      // B[n][c] = V[n][c]: two n8 tiles per x4 load
+      const int row = kt * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+      const int col = c_base + np * 16 + ((lane >> 4) << 3);
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_trans(sV_u + (row * C::kLd + col) * 2, b0, b1, b2, b3);
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        mma_bf16_16816(acc[mt][2 * np], af[mt], b0, b1);
+        mma_bf16_16816(acc[mt][2 * np + 1], af[mt], b2, b3);
+      }
+    }
+  }
+}
+
+template <int D, int BLK>
+__global__ void __launch_bounds__(256, 3)
+stats_kernel(const bf16* __restrict__ K, const bf16* __restrict__ V, int N, int nB, int order,
+             float* __restrict__ kbar, float* __restrict__ S0, bf16* __restrict__ S1) {
+  using C = StatsCfg<D, BLK>;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  bf16* sK = reinterpret_cast<bf16*>(smem_raw);
+  bf16* sV = sK + C::kTileElems;
+  bf16* sStage = sV + C::kTileElems;                            // [D][kStageLd]
+  float* sPart = reinterpret_cast<float*>(sStage + D * C::kStageLd);  // [8 warps][2][D]
+  float* sKbar = sPart + 8 * 2 * D;
+  float* sS0 = sKbar + D;
+
+  const int j = blockIdx.x;
+  const size_t bh = blockIdx.y;
+  const int start = j * BLK;
+  const int n = min(BLK, N - start);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const size_t so = (bh * size_t(nB) + j) * D;
+  load_block_and_sums<D, BLK>(K + (bh * size_t(N) + start) * D, V + (bh * size_t(N) + start) * D, n, sK, sV,
+                              sPart, sKbar, sS0, kbar + so, S0 + so);
+  if (order != 1) return;
 
   // ---- S1 = K^T V - kbar S0^T : M = D (key dim a), N = D (value dim c), K = BLK tokens ----
   // Two passes over halves of the value dimension keep 32 accumulators per
-  // thread (4 CTAs per SM); fragments go straight to global memory.
+  // thread (3 CTAs per SM); each half is staged in shared memory and written
+  // with coalesced 16-byte stores.
   constexpr int TM = D / 4, TN = D / 4;      // warp tile per pass (8 warps as 4 x 2)
   constexpr int MT = TM / 16, NT = TN / 8;
   const int a_base = (warp >> 1) * TM;
@@ -138,30 +195,7 @@ stats_kernel(const bf16* __restrict__ K, const bf16* __restrict__ V, int N, int 
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
-#pragma unroll
-    for (int kt = 0; kt < BLK / 16; ++kt) {
-      uint32_t af[MT][4];
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        // A[a][n] = K[n][a]: transposed 8x8 loads from rows n, columns a
-        const int row = kt * 16 + (lane & 7) + ((lane >> 4) << 3);
-        const int col = a_base + mt * 16 + (((lane >> 3) & 1) << 3);
-        ldsm_x4_trans(sK_u + (row * C::kLd + col) * 2, af[mt][0], af[mt][1], af[mt][2], af[mt][3]);
-      }
-#pragma unroll
-      for (int np = 0; np < NT / 2; ++np) {
-        // B[n][c] = V[n][c]: two n8 tiles per x4 load
-        const int row = kt * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
-        const int col = c_base + np * 16 + ((lane >> 4) << 3);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_trans(sV_u + (row * C::kLd + col) * 2, b0, b1, b2, b3);
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          mma_bf16_16816(acc[mt][2 * np], af[mt], b0, b1);
-          mma_bf16_16816(acc[mt][2 * np + 1], af[mt], b2, b3);
-        }
-      }
-    }
+    s1_half_mma<D, BLK>(sK_u, sV_u, pass, acc);
     if (pass) __syncthreads();  // the previous half has been copied out of the staging tile
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
@@ -188,6 +222,94 @@ stats_kernel(const bf16* __restrict__ K, const bf16* __restrict__ V, int N, int 
           *reinterpret_cast<const uint4*>(sStage + a * C::kStageLd + c8 * 8);
     }
   }
+}
+
+constexpr int kHbarBlocks = 8;  // key blocks per CTA of the hybrid-order statistics
+
+template <int D, int BLK>
+struct HbarCfg {
+  static constexpr size_t kSmem = size_t(2) * StatsCfg<D, BLK>::kTileElems * sizeof(bf16)  // sK, sV
+                                  + size_t(8) * 2 * D * sizeof(float)                      // partial sums
+                                  + size_t(2) * D * sizeof(float);                         // kbar, S0
+};
+
+// kbar, S0 of every block, and Hbar += (1/nB) sum_j S1_j over this CTA's blocks
+// (Hbar zeroed by the caller before the launch).
+template <int D, int BLK>
+__global__ void __launch_bounds__(256, 2)
+stats_hbar_kernel(const bf16* __restrict__ K, const bf16* __restrict__ V, int N, int nB,
+                  float* __restrict__ kbar, float* __restrict__ S0, float* __restrict__ Hbar) {
+  using C = StatsCfg<D, BLK>;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  bf16* sK = reinterpret_cast<bf16*>(smem_raw);
+  bf16* sV = sK + C::kTileElems;
+  float* sPart = reinterpret_cast<float*>(sV + C::kTileElems);  // [8 warps][2][D]
+  float* sKbar = sPart + 8 * 2 * D;
+  float* sS0 = sKbar + D;
+
+  constexpr int TM = D / 4, TN = D / 4;
+  constexpr int MT = TM / 16, NT = TN / 8;
+  const size_t bh = blockIdx.y;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int a_base = (warp >> 1) * TM;
+  const int g = lane >> 2, t4 = lane & 3;
+  const uint32_t sK_u = smem_u32(sK), sV_u = smem_u32(sV);
+
+  float acc[2][MT][NT][4];
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[h][mt][nt][e] = 0.f;
+
+  const int j0 = blockIdx.x * kHbarBlocks;
+  const int j1 = min(nB, j0 + kHbarBlocks);
+#pragma unroll 1
+  for (int j = j0; j < j1; ++j) {
+    const int start = j * BLK;
+    const int n = min(BLK, N - start);
+    const size_t so = (bh * size_t(nB) + j) * D;
+    if (j > j0) __syncthreads();  // the previous block's tiles and sums are no longer read
+    load_block_and_sums<D, BLK>(K + (bh * size_t(N) + start) * D, V + (bh * size_t(N) + start) * D, n, sK, sV,
+                                sPart, sKbar, sS0, kbar + so, S0 + so);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      s1_half_mma<D, BLK>(sK_u, sV_u, h, acc[h]);
+      const int c_base = h * (D / 2) + (warp & 1) * TN;
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        const int a = a_base + mt * 16 + g;
+        const float k0 = sKbar[a], k1 = sKbar[a + 8];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const int c = c_base + nt * 8 + 2 * t4;
+          const float s0 = sS0[c], s1 = sS0[c + 1];
+          acc[h][mt][nt][0] -= k0 * s0;
+          acc[h][mt][nt][1] -= k0 * s1;
+          acc[h][mt][nt][2] -= k1 * s0;
+          acc[h][mt][nt][3] -= k1 * s1;
+        }
+      }
+    }
+  }
+  const float inv = 1.f / float(nB);
+  float* gH = Hbar + bh * size_t(D) * D;
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int a = a_base + mt * 16 + g;
+        const int c = h * (D / 2) + (warp & 1) * TN + nt * 8 + 2 * t4;
+        atomicAdd(reinterpret_cast<float2*>(gH + size_t(a) * D + c),
+                  make_float2(acc[h][mt][nt][0] * inv, acc[h][mt][nt][1] * inv));
+        atomicAdd(reinterpret_cast<float2*>(gH + size_t(a + 8) * D + c),
+                  make_float2(acc[h][mt][nt][2] * inv, acc[h][mt][nt][3] * inv));
+      }
 }
 
 }  // namespace pisa

@@ -3,12 +3,14 @@
 Per-unit figures:
 
 * attention: 4*b*d flops per (query, critical block) -- QK^T and PV --
-  plus 4*d per (query, non-critical block) -- x.kbar and alpha*S0 -- plus,
-  at order 1, 2*d*d per (query, non-critical block) -- S1^T x. Ragged blocks
-  count at their mean size N / nB.
+  plus 4*d per (query, non-critical block) -- x.kbar and alpha*S0 (orders 0,
+  1, 2) -- plus, at order 1, 2*d*d per (query, non-critical block) -- S1^T x --
+  or, at order 2 (hybrid), 2*d*d once per query -- x Hbar. Keep-or-drop
+  (order -1) has the exact term only. Ragged blocks count at their mean size
+  N / nB.
 * stats: bytes = K and V read (2*N*d*2 per head) + kbar and S0 written
-  (2*nB*d*4) + S1 written (nB*d*d*2 at order 1); flops = 2*n*d*d per block
-  for K^T V.
+  (2*nB*d*4) + S1 written (nB*d*d*2 at order 1) or Hbar written (d*d*4 at
+  order 2); flops = 2*n*d*d per block for K^T V (orders 1 and 2).
 * select: bytes = Q read (N*d*2) + kbar read (nB*d*4) + idx written
   (nB*k*4); flops = 2*d per (query block, key block) pooled score.
 * dense-equivalent attention flops: 4*N*N*d per head.
@@ -24,15 +26,25 @@ def attention_flops(B, H, N, d, block, topk, order) -> float:
     nB = num_blocks(N, block)
     mean_n = N / nB
     rest = nB - topk
-    per_q = 4.0 * mean_n * d * topk + 4.0 * d * rest + (2.0 * d * d * rest if order >= 1 else 0.0)
+    per_q = 4.0 * mean_n * d * topk
+    if order >= 0:
+        per_q += 4.0 * d * rest
+    if order == 1:
+        per_q += 2.0 * d * d * rest
+    elif order == 2 and rest > 0:
+        per_q += 2.0 * d * d
     return float(B * H * N * per_q)
+
+
+def _first_order_bytes(nB, d, order) -> int:
+    return nB * d * d * 2 if order == 1 else (d * d * 4 if order == 2 else 0)
 
 
 def attention_bytes(B, H, N, d, block, topk, order) -> float:
     """Compulsory HBM traffic of one attention call (each operand once)."""
     nB = num_blocks(N, block)
     qkvo = 4 * N * d * 2
-    stats = 2 * nB * d * 4 + (nB * d * d * 2 if order >= 1 else 0)
+    stats = (2 * nB * d * 4 if order >= 0 else 0) + _first_order_bytes(nB, d, order)
     return float(B * H * (qkvo + stats + nB * topk * 4))
 
 
@@ -42,7 +54,7 @@ def dense_flops(B, H, N, d) -> float:
 
 def stats_bytes(B, H, N, d, block, order) -> float:
     nB = num_blocks(N, block)
-    return float(B * H * (2 * N * d * 2 + 2 * nB * d * 4 + (nB * d * d * 2 if order >= 1 else 0)))
+    return float(B * H * (2 * N * d * 2 + 2 * nB * d * 4 + _first_order_bytes(nB, d, order)))
 
 
 def stats_flops(B, H, N, d, block, order) -> float:

@@ -19,8 +19,8 @@
  *    exponent, including the Taylor term).
  *  - All pointers are DEVICE pointers owned by the caller, 16-byte aligned, on the
  *    current CUDA device. The library allocates no device memory and never frees or
- *    retains caller memory after the call returns (it does cache TMA descriptors that
- *    hold the pointer values, keyed by pointer and shape).
+ *    retains caller memory after the call returns (TMA descriptors are encoded on the
+ *    host for each call and passed by value to the kernel).
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream). Every call only
  *    enqueues work on it and returns; results are ready when the stream has reached them.
  *  - Supported: d in {64, 128}; block in {64, 128}; nB <= PISA_MAX_BLOCKS; compute
@@ -33,6 +33,18 @@
  *    that pisa_device_error() reports as PISA_ERR_TIMEOUT / PISA_ERR_INVALID_ARG.
  *  - The calls are thread-safe with respect to one another; pisa_last_error() is per
  *    host thread.
+ *
+ * Orders (how the non-critical blocks U_i of a query block enter the softmax)
+ * -------------------------------------------------------------------------
+ *  PISA_ORDER_DROP   (-1) keep-or-drop: they are left out (block-sparse attention,
+ *                         the baseline class of the explainer's section 1).
+ *  PISA_ORDER_ZERO    (0) zeroth-order Taylor term alpha_{t,j} S0_j.
+ *  PISA_ORDER_FIRST   (1) zeroth order plus the per-block first-order term
+ *                         alpha_{t,j} S1_j^T x_t.
+ *  PISA_ORDER_HYBRID  (2) section 2, "Core algorithm": zeroth order per block plus ONE
+ *                         global first-order correction (x_t Hbar) sum_{j in U_i}
+ *                         alpha_{t,j}, Hbar the mean over all blocks of the head of
+ *                         the per-block first-order matrices.
  */
 #ifndef PISA_H_
 #define PISA_H_
@@ -44,6 +56,11 @@ extern "C" {
 #endif
 
 #define PISA_MAX_BLOCKS 2048
+
+#define PISA_ORDER_DROP (-1)
+#define PISA_ORDER_ZERO 0
+#define PISA_ORDER_FIRST 1
+#define PISA_ORDER_HYBRID 2
 
 typedef enum {
   PISA_OK = 0,
@@ -71,8 +88,13 @@ typedef struct {
  *   S1_j   = sum_{n in j} (k_n - kbar_j) v_n^T        bf16  [B, H, nB, d, d]
  *            (row a = key dimension, column c = value dimension; fp32 accumulation,
  *             rounded once to bf16)
- * K, V: bf16 [B, H, N, d]. order: 0 or 1; S1 is written only when order == 1 and may
- * be NULL when order == 0.
+ *   Hbar   = (1/nB) sum_j S1_j                        fp32  [B, H, d, d]
+ * K, V: bf16 [B, H, N, d]. order (-1, 0, 1 or 2) selects what the S1 argument receives:
+ *   order 1: S1 = the per-block matrices, bf16 [B, H, nB, d, d];
+ *   order 2: S1 = Hbar, fp32 [B, H, d, d]. The call zeroes it on `stream`, then
+ *            accumulates it with fp32 atomics (reproducible to fp32 rounding, not bit
+ *            for bit); per-block S1 is not written;
+ *   order 0, -1: S1 is not touched and may be NULL.
  */
 pisa_status_t pisa_block_stats(const void* K, const void* V, pisa_shape_t shape, int32_t order,
                                float* kbar, float* S0, void* S1, void* stream);
@@ -102,12 +124,16 @@ pisa_status_t pisa_select(const void* Q, const float* kbar, pisa_shape_t shape, 
  * approximate stage). For query row t of block i with critical set S_i = idx[b,h,i,:]:
  *   N_t = sum_{j in S_i} sum_n e^{x_t.k_n} v_n
  *       + sum_{j not in S_i} e^{x_t.kbar_j} (S0_j + [order == 1] S1_j^T x_t)
+ *       + [order == 2] (x_t Hbar) sum_{j not in S_i} e^{x_t.kbar_j}
  *   D_t = sum_{j in S_i} sum_n e^{x_t.k_n} + sum_{j not in S_i} n_j e^{x_t.kbar_j}
  *   O_t = N_t / D_t                                  bf16 [B, H, N, d]
+ * (at order -1 both sums over j not in S_i are absent).
  * All exponents are taken relative to one running row maximum (a single online-softmax
  * accumulator). idx rows must hold topk distinct blocks in [0, nB) (the order inside a
  * row does not matter); out-of-range entries are ignored and flagged in the device
- * error word. S1 may be NULL when order == 0. scale must be finite and > 0.
+ * error word. S1 is the per-block bf16 S1 at order 1 and the fp32 Hbar at order 2 (both
+ * from pisa_block_stats at the same order); it may be NULL at orders 0 and -1, and kbar
+ * and S0 may be NULL at order -1. scale must be finite and > 0.
  */
 pisa_status_t pisa_attention(const void* Q, const void* K, const void* V, const float* kbar,
                              const float* S0, const void* S1, const int32_t* idx,

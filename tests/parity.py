@@ -44,9 +44,30 @@ def compare_idx(gpu_idx: np.ndarray, ref_idx: np.ndarray, near: np.ndarray):
     return int(bad.sum()), int((bad & near).sum()), bad
 
 
+def oracle_stats(Kf, Vf, wl: W.Workload):
+    """kbar, S0 and the order's first-order statistic (per-block S1 at order 1, the
+    head's Hbar at order 2, None otherwise)."""
+    kbar, S0, S1 = oracle.block_stats(Kf, Vf, wl.block, 1 if wl.order >= 1 else 0)
+    if wl.order == oracle.ORDER_HYBRID:
+        S1 = oracle.global_first_order(S1)
+    return kbar, S0, S1
+
+
+def check_first_order_stat(gpu_S1, ref_S1, order: int):
+    """Per-block S1 (bf16, one rounding) or Hbar (fp32 sum of fp32 terms)."""
+    if order == 1:
+        g1 = bf16_to_f64(gpu_S1)
+        assert np.all(np.abs(g1 - ref_S1) <= 2.0 ** -8 * np.abs(ref_S1) + 1e-3)
+    elif order == 2:
+        g = gpu_S1.double().cpu().numpy()
+        scale = np.abs(ref_S1).max()
+        # fp32 terms of magnitude ~|S1_j| summed over the blocks: allow 1e-4 of the largest entry
+        assert np.abs(g - ref_S1).max() <= 1e-4 * scale + 1e-5, np.abs(g - ref_S1).max() / scale
+
+
 def oracle_pipeline(Qf, Kf, Vf, wl: W.Workload, query_blocks=None):
     """Oracle stats -> select -> attention on fp64 copies of the inputs."""
-    kbar, S0, S1 = oracle.block_stats(Kf, Vf, wl.block, wl.order)
+    kbar, S0, S1 = oracle_stats(Kf, Vf, wl)
     idx, near, _ = oracle.select(Qf, kbar, wl.block, wl.topk)
     O = oracle.attention(Qf, Kf, Vf, kbar, S0, S1, idx, wl.block, wl.order, wl.scale,
                          query_blocks=query_blocks)

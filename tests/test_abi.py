@@ -82,11 +82,13 @@ def test_null_and_misaligned_pointers(L):
 
 
 def test_bad_scalars(L):
-    assert stats(L, order=2) == INVALID
+    assert stats(L, order=3) == INVALID
+    assert stats(L, order=-2) == INVALID
     assert sel(L, topk=0) == INVALID
     assert sel(L, topk=5) == INVALID            # nB = 4
     assert attn(L, topk=0) == INVALID
-    assert attn(L, order=-1) == INVALID
+    assert attn(L, order=3) == INVALID
+    assert attn(L, order=-2) == INVALID
     for sc in (0.0, -1.0, float("nan"), float("inf")):
         assert attn(L, scale=sc) == INVALID, sc
     assert attn(L, s=shape(N=-1)) == INVALID
@@ -100,12 +102,41 @@ def test_unsupported_shapes(L):
     assert attn(L, s=shape(B=300, H=300)) == UNSUPPORTED
 
 
+def _no_device():
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("fake pointers must never reach a real device")
+
+
+def _passes_validation(st, L):
+    # validation passed: only the device check (no GPU here) remains
+    assert st == CUDA_ERR, L.pisa_last_error()
+    assert b"cuda" in L.pisa_last_error().lower()
+
+
 def test_order0_needs_no_S1(L):
-    # with S1 = NULL at order 0 validation passes and only the device check remains
-    st = stats(L, order=0, S1=0)
-    assert st in (OK, CUDA_ERR, UNSUPPORTED)
-    if st != OK:
-        assert b"cuda" in L.pisa_last_error().lower() or b"sm_" in L.pisa_last_error()
+    _no_device()
+    _passes_validation(stats(L, order=0, S1=0), L)
+    _passes_validation(attn(L, order=0, S1=0), L)
+
+
+def test_hybrid_order_needs_hbar(L):
+    assert stats(L, order=2, S1=0) == INVALID
+    assert b"Hbar" in L.pisa_last_error()
+    assert attn(L, order=2, S1=0) == INVALID
+    assert attn(L, order=2, S1=MISALIGNED) == INVALID
+    _no_device()
+    _passes_validation(stats(L, order=2), L)
+    _passes_validation(attn(L, order=2), L)
+
+
+def test_drop_needs_no_statistics(L):
+    # keep-or-drop reads no kbar, S0 or S1 in the attention call
+    assert attn(L, order=-1, idx=0) == INVALID
+    _no_device()
+    _passes_validation(attn(L, order=-1, kbar=0, S0=0, S1=0), L)
+    _passes_validation(attn(L, order=-1, kbar=0, S0=0, S1=0, fn="pisa_attention_simt"), L)
+    _passes_validation(stats(L, order=-1, S1=0), L)
 
 
 def test_empty_problem_touches_nothing(L):

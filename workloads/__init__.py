@@ -86,6 +86,10 @@ WORKLOADS = {
     "long": Workload("long", 1, 40, 75600, 128, 128, _ceil_keep(0.10, 591), 1,
                      1.0 / math.sqrt(128), "video", (21, 60, 60), 1005),
 }
+# the video workloads under the hybrid order (global Hbar) and keep-or-drop
+WORKLOADS["video_hybrid"] = WORKLOADS["video"].with_(name="video_hybrid", order=2)
+WORKLOADS["video_drop"] = WORKLOADS["video"].with_(name="video_drop", order=-1)
+WORKLOADS["long_hybrid"] = WORKLOADS["long"].with_(name="long_hybrid", order=2)
 
 
 def get(name: str) -> Workload:
