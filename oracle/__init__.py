@@ -29,6 +29,8 @@ from .pisa import (  # noqa: F401
     attention,
     dense_attention,
     global_first_order,
+    routing_norms,
+    round_to_bf16,
     ORDER_DROP,
     ORDER_ZERO,
     ORDER_FIRST,

@@ -81,14 +81,19 @@ def pooled_queries(Q, block: int):
     return qbar
 
 
-def select(Q, kbar, block: int, topk: int):
+def select(Q, kbar, block: int, topk: int, route=None, lam: float = 0.0):
     """Top-k critical blocks of every query block.
 
-    The page states only that the critical blocks are the ones with the highest
-    attention relevance (section 2, "Covariance-aware routing", first sentence
-    without the covariance term). Relevance here is the pooled score
-    ``qbar_i . kbar_j`` with ``qbar_i`` the mean query of block i. A positive
-    softmax scale cannot change the order, so the scores are unscaled.
+    The page states that the critical blocks are the ones with the highest
+    attention relevance (section 2, "Covariance-aware routing", first sentence).
+    Relevance here is the pooled score ``qbar_i . kbar_j`` with ``qbar_i`` the
+    mean query of block i. A positive softmax scale cannot change the order, so
+    the scores are unscaled.
+
+    Covariance-aware routing (same paragraph): with ``route`` = M [B,H,nB] (see
+    ``routing_norms``) and a weight ``lam`` >= 0, the score of key block j is
+    ``qbar_i . kbar_j + lam * M_j``, so that blocks whose first-order matrix
+    departs most from the head's mean are favoured for exact treatment.
 
     Returns ``idx`` int32 [B,H,nB,topk] (each row ascending; ties between equal
     scores go to the lower block index), ``near_tie`` bool [B,H,nB] (the k-th
@@ -100,6 +105,8 @@ def select(Q, kbar, block: int, topk: int):
     if not (0 <= topk <= nB):
         raise ValueError("topk out of range")
     scores = np.matmul(qbar, np.swapaxes(kbar, -1, -2))
+    if route is not None:
+        scores = scores + lam * np.asarray(route, dtype=np.float64)[:, :, None, :]
     idx = np.empty((B, H, nB, topk), dtype=np.int32)
     near = np.zeros((B, H, nB), dtype=bool)
     cols = np.arange(nB)
@@ -114,6 +121,33 @@ def select(Q, kbar, block: int, topk: int):
                     a, c = row[order[topk - 1]], row[order[topk]]
                     near[b, h, i] = abs(a - c) <= NEAR_TIE_REL * max(abs(a), abs(c))
     return idx, near, scores
+
+
+def round_to_bf16(x):
+    """Round to the nearest bf16 value (ties to even) through fp32, as a value
+    computed in fp32 and stored as bf16 is rounded."""
+    f = np.ascontiguousarray(np.asarray(x, dtype=np.float64).astype(np.float32))
+    u = f.view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def routing_norms(S1, stored_bf16: bool = True):
+    """M_j = || H_j - Hbar ||_F for every block (section 2, "Covariance-aware
+    routing": the norm of the block's deviation from the global first-order
+    statistic; H_j is the block's first-order matrix S1_j and Hbar their mean
+    over the head's blocks). The page writes a 2-norm without naming it; the
+    Frobenius norm (the 2-norm of the matrix as a vector) is taken here.
+
+    The norm feeds a top-k decision, so it is formed from S1 as it is stored
+    for the kernels (fp32 values rounded to bf16) when ``stored_bf16``.
+    Returns float64 [B,H,nB]."""
+    S1 = np.asarray(S1, dtype=np.float64)
+    if stored_bf16:
+        S1 = round_to_bf16(S1)
+    Hbar = S1.mean(axis=2)
+    dev = S1 - Hbar[:, :, None]
+    return np.sqrt((dev * dev).sum(axis=(-2, -1)))
 
 
 def _query_blocks(nB, query_blocks):

@@ -422,3 +422,78 @@ def pin_hybrid_all_selected_is_dense(orc, seed=17):
     nB = -(-N // b)
     out = orc.attention(Q, K, V, kbar, S0, orc.global_first_order(S1), _full_idx(B, H, nB), b, 2, 0.5)
     return np.abs(out - _textbook(Q, K, V, 0.5)).max()
+
+
+# ----------------------------------------------------------------------------
+# covariance-aware routing
+# ----------------------------------------------------------------------------
+def pin_round_to_bf16(orc, seed=18):
+    """Nearest bf16 by enumeration of the neighbouring bf16 values (ties to the
+    even mantissa), on random fp32 values and on planted halfway cases."""
+    r = _rng(seed)
+    x = (r.standard_normal(400) * np.exp(r.uniform(-20, 20, 400))).astype(np.float32)
+    half = np.array([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -2.0 - 2.0 ** -7, 3.0 + 2.0 ** -7], dtype=np.float32)
+    x = np.concatenate([x, half])
+    got = orc.round_to_bf16(x.astype(np.float64))
+    bad = 0
+    for v, g in zip(x.tolist(), got.tolist()):
+        bits = int(np.array(v, dtype=np.float32).view(np.uint32))
+        lo = bits & 0xFFFF0000                     # truncation toward zero (same sign)
+        hi = lo + 0x10000                          # next bf16 away from zero
+        cand = [float(np.array(c, dtype=np.uint32).view(np.float32)) for c in (lo, hi)]
+        dl, dh = abs(v - cand[0]), abs(v - cand[1])
+        if dl < dh or (dl == dh and ((lo >> 16) & 1) == 0):
+            ref = cand[0]
+        else:
+            ref = cand[1]
+        bad += g != ref
+    return bad
+
+
+def pin_routing_norms_bruteforce(orc, seed=19):
+    """M_j = sqrt(sum_{a,c} (S1_j[a,c] - Hbar[a,c])^2) by scalar loops; the inputs are
+    bf16 values already, so the stored-precision rounding is the identity."""
+    r = _rng(seed)
+    nB, d = 5, 3
+    S1 = orc.round_to_bf16(r.standard_normal((1, 2, nB, d, d)) * 3)
+    M = orc.routing_norms(S1)
+    err = 0.0
+    for h in range(2):
+        mean = [[sum(S1[0, h, k, a, c] for k in range(nB)) / nB for c in range(d)] for a in range(d)]
+        for j in range(nB):
+            ref = math.sqrt(sum((S1[0, h, j, a, c] - mean[a][c]) ** 2 for a in range(d) for c in range(d)))
+            err = max(err, abs(M[0, h, j] - ref))
+    return err
+
+
+def pin_routed_select_bruteforce(orc, seed=20, trials=30):
+    """Exhaustive subset search over the scores qbar . kbar_j + lam * M_j (ragged N,
+    planted ties). Returns #mismatches."""
+    r = _rng(seed)
+    bad = 0
+    for t in range(trials):
+        b = int(r.integers(1, 5))
+        nB = int(r.integers(4, 9))
+        N = b * nB - int(r.integers(0, b))
+        nB = -(-N // b)
+        d = int(r.integers(1, 4))
+        k = int(r.integers(1, nB + 1))
+        lam = float(r.uniform(0.1, 3.0))
+        Q = r.standard_normal((1, 1, N, d))
+        kbar = r.standard_normal((1, 1, nB, d))
+        M = np.abs(r.standard_normal((1, 1, nB)))
+        if t % 3 == 0:            # ties: two blocks with equal centroid and equal norm
+            kbar[0, 0, nB - 1] = kbar[0, 0, 0]
+            M[0, 0, nB - 1] = M[0, 0, 0]
+        idx, _, _ = orc.select(Q, kbar, b, k, route=M, lam=lam)
+        for i in range(nB):
+            rows = list(range(i * b, min(i * b + b, N)))
+            qbar = [sum(Q[0, 0, s, a] for s in rows) / len(rows) for a in range(d)]
+            sc = [sum(qbar[a] * kbar[0, 0, j, a] for a in range(d)) + lam * M[0, 0, j] for j in range(nB)]
+            best, best_set = -math.inf, None
+            for sub in itertools.combinations(range(nB), k):
+                tot = sum(sc[j] for j in sub)
+                if tot > best + 1e-12:
+                    best, best_set = tot, sub
+            bad += list(idx[0, 0, i]) != list(best_set)
+    return bad

@@ -42,6 +42,9 @@ def _pins(orc):
         ("hybrid_bruteforce", P.pin_hybrid_bruteforce, lambda e: e < TOL),
         ("hybrid_shared_first_order", P.pin_hybrid_shared_first_order, lambda e: e < TOL),
         ("hybrid_all_selected_is_dense", P.pin_hybrid_all_selected_is_dense, lambda e: e < TOL),
+        ("round_to_bf16", P.pin_round_to_bf16, lambda e: e == 0),
+        ("routing_norms_bruteforce", P.pin_routing_norms_bruteforce, lambda e: e < TOL),
+        ("routed_select_bruteforce", P.pin_routed_select_bruteforce, lambda e: e == 0),
     ]:
         try:
             v = fn(orc)
@@ -65,7 +68,8 @@ def real_pins():
     "order0_pseudo_tokens", "first_order_key_form", "linear_in_values",
     "permutation_in_block", "order0_convex", "worked_example",
     "convergence_order0", "convergence_order1", "drop_is_masked_softmax", "hybrid_bruteforce",
-    "hybrid_shared_first_order", "hybrid_all_selected_is_dense"])
+    "hybrid_shared_first_order", "hybrid_all_selected_is_dense", "round_to_bf16",
+    "routing_norms_bruteforce", "routed_select_bruteforce"])
 def test_pin(real_pins, name):
     value, ok = real_pins[name]
     assert ok, f"{name}: {value}"
@@ -101,6 +105,12 @@ MUTATIONS = {
     "hybrid weight from all blocks": ("* alpha.sum(axis=1)[:, None]",
                                       "* (alpha.sum(axis=1) + w.sum(axis=1))[:, None]"),
     "hybrid term dropped": ("num = num + (X @ S1[b, h])", "num = num + 0 * (X @ S1[b, h])"),
+    "routing norm not centred": ("dev = S1 - Hbar[:, :, None]", "dev = S1"),
+    "routing weight sign flipped": ("scores + lam * np.asarray(route", "scores - lam * np.asarray(route"),
+    "routing bias on the query axis": ("dtype=np.float64)[:, :, None, :]", "dtype=np.float64)[:, :, :, None]"),
+    "bf16 rounding truncates": ("r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16", "r = (u >> 16) << 16"),
+    "bf16 ties away from even": ("r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16",
+                                 "r = ((u + 0x8000) >> 16) << 16"),
 }
 
 
