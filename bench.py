@@ -139,10 +139,16 @@ def oracle_sample(wl, budget_s: float = 15.0, min_blocks: int = 2):
     q, k, v = W.make_inputs(wl.with_(B=1), heads=[0])
     Qf, Kf, Vf = (W.bf16_bits_to_f32(a).astype(np.float64) for a in (q, k, v))
     t0 = time.perf_counter()
-    kbar, S0, S1 = oracle.block_stats(Kf, Vf, wl.block, 1 if wl.order >= 1 else 0)
-    if wl.order == 2:
+    routed = wl.route_lambda > 0
+    kbar, S0, S1 = oracle.block_stats(Kf, Vf, wl.block, 1 if (wl.order >= 1 or routed) else 0)
+    route = None
+    if routed:
+        route = oracle.routing_norms(S1)
+        if wl.order == 2:
+            S1 = oracle.round_to_bf16(S1).mean(axis=2)
+    elif wl.order == 2:
         S1 = oracle.global_first_order(S1)
-    idx, _, _ = oracle.select(Qf, kbar, wl.block, wl.topk)
+    idx, _, _ = oracle.select(Qf, kbar, wl.block, wl.topk, route=route, lam=wl.route_lambda)
     t_pre = time.perf_counter() - t0
     # query blocks spread over the sequence, run until the budget is spent
     order = np.random.default_rng(0).permutation(wl.nB)
@@ -154,7 +160,7 @@ def oracle_sample(wl, budget_s: float = 15.0, min_blocks: int = 2):
     t_attn = time.perf_counter() - t1
     frac_q = done / wl.nB
     flops = (R.attention_flops(1, 1, wl.N, wl.d, wl.block, wl.topk, wl.order) * frac_q
-             + R.stats_flops(1, 1, wl.N, wl.d, wl.block, wl.order)
+             + R.stats_flops(1, 1, wl.N, wl.d, wl.block, 1 if routed else wl.order)
              + R.select_flops(1, 1, wl.N, wl.d, wl.block))
     secs = t_pre + t_attn
     threads = _blas_threads()
@@ -187,7 +193,7 @@ def run_reference(args):
         if i >= args.warmup:
             per_step.append((tf, secs))
     tf = statistics.mean(t for t, _ in per_step)
-    full_ms = R.step_flops(wl.B, wl.H, wl.N, wl.d, wl.block, wl.topk, wl.order) / (tf * 1e12) * 1e3
+    full_ms = _step_flops(wl) / (tf * 1e12) * 1e3
     line = {
         "impl": "reference", "metric": METRIC, "value": tf, "unit": UNIT, "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": full_ms,
@@ -232,6 +238,14 @@ def _captured_traffic(wl):
     return d["dram_bytes_per_full_launch"] if h == d["sources_sha256"] else None
 
 
+def _step_flops(wl):
+    flops = R.step_flops(wl.B, wl.H, wl.N, wl.d, wl.block, wl.topk, wl.order)
+    if wl.route_lambda > 0 and wl.order != 1:   # per-block S1 is formed for the routing norms
+        flops += R.stats_flops(wl.B, wl.H, wl.N, wl.d, wl.block, 1) - R.stats_flops(
+            wl.B, wl.H, wl.N, wl.d, wl.block, wl.order)
+    return flops
+
+
 def _workload(args):
     wl = W.get(args.workload)
     return wl.with_(H=args.heads) if args.heads else wl
@@ -240,7 +254,7 @@ def _workload(args):
 def _config(wl, ws):
     return {"workload": _workload_desc(wl), "global_batch": wl.B * ws, "seq_len": wl.N,
             "heads": wl.H, "head_dim": wl.d, "block": wl.block, "topk": wl.topk,
-            "keep": wl.topk / wl.nB, "order": wl.order,
+            "keep": wl.topk / wl.nB, "order": wl.order, "route_lambda": wl.route_lambda,
             "l2": "inputs larger than L2 (Q+K+V %.0f MB per GPU), no flush" % (3 * wl.B * wl.H * wl.N * wl.d * 2 / 1e6),
             "parallelism": f"dp{ws} (independent batches per GPU, no collective)"}
 
@@ -268,12 +282,17 @@ def run_ours(args):
     nB = wl.nB
     kbar = torch.empty((wl.B, wl.H, nB, wl.d), device=dev, dtype=torch.float32)
     S0 = torch.empty_like(kbar)
-    if wl.order == 1:      # per-block first-order matrices
+    routed = wl.route_lambda > 0
+    stats_order = 1 if routed else wl.order
+    if stats_order == 1:   # per-block first-order matrices
         S1 = torch.empty((wl.B, wl.H, nB, wl.d, wl.d), device=dev, dtype=torch.bfloat16)
     elif wl.order == 2:    # the head's global Hbar
         S1 = torch.empty((wl.B, wl.H, wl.d, wl.d), device=dev, dtype=torch.float32)
     else:
         S1 = None
+    Hbar = torch.empty((wl.B, wl.H, wl.d, wl.d), device=dev, dtype=torch.float32) if routed else None
+    M = torch.empty((wl.B, wl.H, nB), device=dev, dtype=torch.float32) if routed else None
+    first = (Hbar if wl.order == 2 else (S1 if wl.order == 1 else None)) if routed else S1
     idx = torch.empty((wl.B, wl.H, nB, wl.topk), device=dev, dtype=torch.int32)
     O = torch.empty_like(Q)
     attn = P.attention if args.kernel == "fused" else P.attention_simt
@@ -282,21 +301,25 @@ def run_ours(args):
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        P.block_stats(K, V, wl.block, wl.order, out=(kbar, S0, S1))
+        P.block_stats(K, V, wl.block, stats_order, out=(kbar, S0, S1))
         if ev is not None:
             ev[1].record(stream)
-        P.select(Q, kbar, wl.block, wl.topk, out=idx)
+        if routed:
+            P.routing_norms(S1, wl.block, wl.N, out=(Hbar, M))
         if ev is not None:
             ev[2].record(stream)
-        attn(Q, K, V, kbar, S0, S1, idx, wl.block, wl.order, wl.scale, out=O)
+        P.select(Q, kbar, wl.block, wl.topk, out=idx, route=M, lam=wl.route_lambda)
         if ev is not None:
             ev[3].record(stream)
+        attn(Q, K, V, kbar, S0, first, idx, wl.block, wl.order, wl.scale, out=O)
+        if ev is not None:
+            ev[4].record(stream)
 
     for _ in range(args.warmup):
         step()
     P.device_error()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     sampler = ClockSampler(_physical_gpu(local)).start() if rank == 0 else None
     time.sleep(0.3 if sampler else 0)
     if pg:
@@ -315,14 +338,16 @@ def run_ours(args):
     ms_total = max_over_ranks(start.elapsed_time(end), pg, dev)
     ms_step = ms_total / args.steps
     k_ms = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
-            for i, n in enumerate(("stats", "select", "attention"))}
+            for i, n in enumerate(("stats", "routing", "select", "attention"))}
+    if not routed:
+        del k_ms["routing"]
 
-    flops_step = R.step_flops(wl.B, wl.H, wl.N, wl.d, wl.block, wl.topk, wl.order)
+    flops_step = _step_flops(wl)
     value = job_throughput(flops_step, ws, ms_step)
     att_flops = R.attention_flops(wl.B, wl.H, wl.N, wl.d, wl.block, wl.topk, wl.order)
     att_tf = att_flops / (k_ms["attention"] * 1e-3) / 1e12
     dense_tf = R.dense_flops(wl.B, wl.H, wl.N, wl.d) / (k_ms["attention"] * 1e-3) / 1e12
-    st_gbs = R.stats_bytes(wl.B, wl.H, wl.N, wl.d, wl.block, wl.order) / (k_ms["stats"] * 1e-3) / 1e9
+    st_gbs = R.stats_bytes(wl.B, wl.H, wl.N, wl.d, wl.block, stats_order) / (k_ms["stats"] * 1e-3) / 1e9
     se_gbs = R.select_bytes(wl.B, wl.H, wl.N, wl.d, wl.block, wl.topk) / (k_ms["select"] * 1e-3) / 1e9
     pk = _peaks()
     peak = pk["bf16_sus"]
@@ -332,7 +357,8 @@ def run_ours(args):
     if not args.no_e2e:
         hq, hk, hv = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in (q, k, v))
         for _ in range(2):
-            P.pisa_host(hq, hk, hv, wl.block, wl.topk, wl.order, wl.scale, device=dev)
+            P.pisa_host(hq, hk, hv, wl.block, wl.topk, wl.order, wl.scale, device=dev,
+                        route_lambda=wl.route_lambda)
         n_e2e = max(2, min(args.steps, 5))
         if pg:
             pg.barrier()
@@ -342,7 +368,8 @@ def run_ours(args):
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(n_e2e):
-            P.pisa_host(hq, hk, hv, wl.block, wl.topk, wl.order, wl.scale, device=dev)
+            P.pisa_host(hq, hk, hv, wl.block, wl.topk, wl.order, wl.scale, device=dev,
+                        route_lambda=wl.route_lambda)
         e1.record(stream)
         torch.cuda.synchronize()
         wall = (time.perf_counter() - t0) * 1e3 / n_e2e
@@ -377,7 +404,9 @@ def run_ours(args):
         "attention_dense_equivalent_tflops": dense_tf,
         "stats_gbs": st_gbs, "stats_hbm_frac": st_gbs / pk["hbm"],
         "select_gbs": se_gbs, "select_hbm_frac": se_gbs / pk["hbm"],
-        "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": 3 * args.steps, "clocks": clocks,
+        **({"routing_gbs": R.routing_bytes(wl.B, wl.H, wl.N, wl.d, wl.block) / (k_ms["routing"] * 1e-3) / 1e9}
+           if routed else {}),
+        "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": (6 if routed else 3) * args.steps, "clocks": clocks,
         "attention_kernel": args.kernel,
     }
     print(json.dumps(line), flush=True)

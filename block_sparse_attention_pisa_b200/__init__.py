@@ -21,14 +21,14 @@ ORDER_DROP, ORDER_ZERO, ORDER_FIRST, ORDER_HYBRID = -1, 0, 1, 2
 
 __all__ = [
     "ORDER_DROP", "ORDER_ZERO", "ORDER_FIRST", "ORDER_HYBRID", "PisaError", "Shape", "lib", "block_stats", "select", "attention", "attention_simt",
-    "pisa", "pisa_host", "device_error", "num_blocks", "LIB_PATH", "SYMBOLS",
+    "pisa", "pisa_host", "device_error", "num_blocks", "LIB_PATH", "SYMBOLS", "routing_norms",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpisa.so")
 
 # entry points declared in include/pisa.h
 SYMBOLS = (
-    "pisa_block_stats", "pisa_select", "pisa_attention", "pisa_attention_simt",
+    "pisa_block_stats", "pisa_select", "pisa_routing_norms", "pisa_attention", "pisa_attention_simt",
     "pisa_device_error", "pisa_status_string", "pisa_last_error", "pisa_version",
 )
 
@@ -61,7 +61,8 @@ def lib():
     L = ctypes.CDLL(LIB_PATH)
     vp, i32, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
     L.pisa_block_stats.argtypes = [vp, vp, Shape, i32, vp, vp, vp, vp]
-    L.pisa_select.argtypes = [vp, vp, Shape, i32, vp, vp]
+    L.pisa_select.argtypes = [vp, vp, vp, f32, Shape, i32, vp, vp]
+    L.pisa_routing_norms.argtypes = [vp, Shape, vp, vp, vp]
     attn = [vp, vp, vp, vp, vp, vp, vp, Shape, i32, i32, f32, vp, vp]
     L.pisa_attention.argtypes = attn
     L.pisa_attention_simt.argtypes = attn
@@ -71,7 +72,7 @@ def lib():
     L.pisa_last_error.argtypes = []
     L.pisa_last_error.restype = ctypes.c_char_p
     L.pisa_version.argtypes = []
-    for name in ("pisa_block_stats", "pisa_select", "pisa_attention", "pisa_attention_simt",
+    for name in ("pisa_block_stats", "pisa_select", "pisa_routing_norms", "pisa_attention", "pisa_attention_simt",
                  "pisa_device_error", "pisa_version"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
@@ -129,15 +130,37 @@ def block_stats(K, V, block: int, order: int = 1, out=None):
     return kbar, S0, S1
 
 
-def select(Q, kbar, block: int, topk: int, out=None):
-    """int32 [B, H, nB, topk]: critical blocks of every query block (ascending)."""
+def select(Q, kbar, block: int, topk: int, out=None, route=None, lam: float = 0.0):
+    """int32 [B, H, nB, topk]: critical blocks of every query block (ascending).
+    ``route`` (fp32 [B, H, nB], from ``routing_norms``) and ``lam`` add the
+    covariance term lam * M_j to every score."""
     import torch
     s = _shape(Q, block)
     nB = num_blocks(s.N, block)
     idx = (torch.empty((s.B, s.H, nB, topk), device=Q.device, dtype=torch.int32)
            if out is None else out)
-    _check(lib().pisa_select(_ptr(Q), _ptr(kbar), s, topk, _ptr(idx), _stream(Q)))
+    _check(lib().pisa_select(_ptr(Q), _ptr(kbar), _ptr(route), float(lam), s, topk, _ptr(idx),
+                             _stream(Q)))
     return idx
+
+
+def routing_norms(S1, block: int, N: int, out=None):
+    """(Hbar fp32 [B, H, d, d], M fp32 [B, H, nB]) from per-block bf16 S1 [B, H, nB, d, d]:
+    the mean first-order matrix and each block's Frobenius deviation from it."""
+    import torch
+    B, H, nB, d, _ = S1.shape
+    if not S1.is_contiguous():
+        raise ValueError("S1 must be contiguous")
+    if nB != num_blocks(N, block):
+        raise ValueError("S1 block count does not match N and block")
+    s = Shape(B, H, N, d, block)
+    if out is not None:
+        Hbar, M = out
+    else:
+        Hbar = torch.empty((B, H, d, d), device=S1.device, dtype=torch.float32)
+        M = torch.empty((B, H, nB), device=S1.device, dtype=torch.float32)
+    _check(lib().pisa_routing_norms(_ptr(S1), s, _ptr(Hbar), _ptr(M), _stream(S1)))
+    return Hbar, M
 
 
 def _attention(fn, Q, K, V, kbar, S0, S1, idx, block, order, scale, out=None):
@@ -161,24 +184,34 @@ def attention_simt(Q, K, V, kbar, S0, S1, idx, block: int, order: int, scale: fl
     return _attention(lib().pisa_attention_simt, Q, K, V, kbar, S0, S1, idx, block, order, scale, out)
 
 
-def pisa(Q, K, V, block: int, topk: int, order: int = 1, scale: float | None = None):
-    """The whole path on device tensors: stats -> select -> attention. Returns (O, idx)."""
+def pisa(Q, K, V, block: int, topk: int, order: int = 1, scale: float | None = None,
+         route_lambda: float = 0.0):
+    """The whole path on device tensors: stats -> select -> attention. Returns (O, idx).
+    With ``route_lambda`` > 0 the selection is covariance-aware: stats at order 1 ->
+    routing norms -> routed select -> attention (at order 2 with the routing call's
+    Hbar)."""
     if scale is None:
         scale = Q.shape[-1] ** -0.5
+    if route_lambda > 0.0:
+        kbar, S0, S1 = block_stats(K, V, block, ORDER_FIRST)
+        Hbar, M = routing_norms(S1, block, Q.shape[2])
+        idx = select(Q, kbar, block, topk, route=M, lam=route_lambda)
+        first = Hbar if order == ORDER_HYBRID else (S1 if order == ORDER_FIRST else None)
+        return attention(Q, K, V, kbar, S0, first, idx, block, order, scale), idx
     kbar, S0, S1 = block_stats(K, V, block, order)
     idx = select(Q, kbar, block, topk)
     return attention(Q, K, V, kbar, S0, S1, idx, block, order, scale), idx
 
 
 def pisa_host(Q, K, V, block: int, topk: int, order: int = 1, scale: float | None = None,
-              device="cuda"):
+              device="cuda", route_lambda: float = 0.0):
     """The whole path on HOST tensors: copies Q, K, V to the device, runs it, and copies
     the output back (pinned host memory gives asynchronous copies). Returns O on the host."""
     import torch
     dq = Q.to(device, non_blocking=True)
     dk = K.to(device, non_blocking=True)
     dv = V.to(device, non_blocking=True)
-    O, _ = pisa(dq, dk, dv, block, topk, order, scale)
+    O, _ = pisa(dq, dk, dv, block, topk, order, scale, route_lambda)
     out = torch.empty(O.shape, dtype=O.dtype, pin_memory=Q.is_pinned())
     out.copy_(O, non_blocking=True)
     torch.cuda.current_stream(O.device).synchronize()

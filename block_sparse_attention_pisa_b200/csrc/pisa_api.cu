@@ -12,6 +12,7 @@
 #include "common.cuh"
 #include "stats.cuh"
 #include "select.cuh"
+#include "routing.cuh"
 #include "attention_simt.cuh"
 #include "attention_tc.cuh"
 
@@ -152,15 +153,33 @@ pisa_status_t launch_stats(const pisa_shape_t& s, const bf16* K, const bf16* V, 
 }
 
 template <int D>
-pisa_status_t launch_select(const pisa_shape_t& s, const bf16* Q, const float* kbar, int topk, int32_t* idx,
-                            cudaStream_t st) {
+pisa_status_t launch_select(const pisa_shape_t& s, const bf16* Q, const float* kbar, const float* route,
+                            float lambda, int topk, int32_t* idx, cudaStream_t st) {
   auto k = pisa::select_kernel<D>;
   const int nB = int(num_blocks(s));
   const size_t smem = pisa::select_smem_bytes(D, nB);
   PISA_TRY(set_smem(k, smem));
   dim3 grid((nB + pisa::kSelectQB - 1) / pisa::kSelectQB, s.B * s.H);
-  k<<<grid, pisa::kSelectThreads, smem, st>>>(Q, kbar, s.N, nB, s.block, topk, idx);
+  k<<<grid, pisa::kSelectThreads, smem, st>>>(Q, kbar, route, lambda, s.N, nB, s.block, topk, idx);
   return check_launch("select_kernel");
+}
+
+pisa_status_t launch_routing(const pisa_shape_t& s, const bf16* S1, float* Hbar, float* M, cudaStream_t st) {
+  const int nB = int(num_blocks(s));
+  const int dd = s.d * s.d;
+  const size_t BH = size_t(s.B) * s.H;
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(Hbar, 0, BH * dd * sizeof(float), st)) != cudaSuccess ||
+      (e = cudaMemsetAsync(M, 0, BH * nB * sizeof(float), st)) != cudaSuccess)
+    return fail(PISA_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+  dim3 grid(dd / pisa::kRouteSlice, (nB + pisa::kRouteChunk - 1) / pisa::kRouteChunk, unsigned(BH));
+  pisa::routing_hbar_kernel<<<grid, pisa::kRouteThreads, 0, st>>>(S1, nB, dd, Hbar);
+  PISA_TRY(check_launch("routing_hbar_kernel"));
+  pisa::routing_norm_kernel<<<grid, pisa::kRouteThreads, 0, st>>>(S1, Hbar, nB, dd, M);
+  PISA_TRY(check_launch("routing_norm_kernel"));
+  const size_t n = BH * nB;
+  pisa::routing_sqrt_kernel<<<unsigned((n + 255) / 256), 256, 0, st>>>(M, n);
+  return check_launch("routing_sqrt_kernel");
 }
 
 template <int D>
@@ -292,22 +311,40 @@ pisa_status_t pisa_block_stats(const void* K, const void* V, pisa_shape_t shape,
   return launch_stats<64, 128>(shape, k, v, order, kbar, S0, S1, st);
 }
 
-pisa_status_t pisa_select(const void* Q, const float* kbar, pisa_shape_t shape, int32_t topk, int32_t* idx,
-                          void* stream) {
+pisa_status_t pisa_select(const void* Q, const float* kbar, const float* route, float lambda, pisa_shape_t shape,
+                          int32_t topk, int32_t* idx, void* stream) {
   bool empty = false;
   PISA_TRY(check_shape(shape, &empty));
   if (empty) return ok();
   PISA_TRY(check_ptr(Q, "Q"));
   PISA_TRY(check_ptr(kbar, "kbar"));
   PISA_TRY(check_ptr(idx, "idx"));
+  if (route != nullptr) {
+    PISA_TRY(check_ptr(route, "route"));
+    if (!std::isfinite(lambda) || lambda < 0.f)
+      return fail(PISA_ERR_INVALID_ARG, "lambda=%g (must be finite and >= 0)", double(lambda));
+  }
   PISA_TRY(check_topk(shape, topk));
   PISA_TRY(check_support(shape));
   int sms = 0;
   PISA_TRY(check_device(&sms));
   auto st = static_cast<cudaStream_t>(stream);
   auto q = static_cast<const bf16*>(Q);
-  if (shape.d == 128) return launch_select<128>(shape, q, kbar, topk, idx, st);
-  return launch_select<64>(shape, q, kbar, topk, idx, st);
+  if (shape.d == 128) return launch_select<128>(shape, q, kbar, route, lambda, topk, idx, st);
+  return launch_select<64>(shape, q, kbar, route, lambda, topk, idx, st);
+}
+
+pisa_status_t pisa_routing_norms(const void* S1, pisa_shape_t shape, float* Hbar, float* M, void* stream) {
+  bool empty = false;
+  PISA_TRY(check_shape(shape, &empty));
+  if (empty) return ok();
+  PISA_TRY(check_ptr(S1, "S1"));
+  PISA_TRY(check_ptr(Hbar, "Hbar"));
+  PISA_TRY(check_ptr(M, "M"));
+  PISA_TRY(check_support(shape));
+  int sms = 0;
+  PISA_TRY(check_device(&sms));
+  return launch_routing(shape, static_cast<const bf16*>(S1), Hbar, M, static_cast<cudaStream_t>(stream));
 }
 
 pisa_status_t pisa_attention(const void* Q, const void* K, const void* V, const float* kbar, const float* S0,

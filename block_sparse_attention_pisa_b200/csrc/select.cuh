@@ -5,7 +5,8 @@
 // relevance of key block j to query block i is the pooled score
 // qbar_i . kbar_j, with qbar_i the mean of the query block's real rows (fp32
 // throughout, so that the ranking matches an exact evaluation except at
-// near-ties).
+// near-ties). With covariance-aware routing (same paragraph) each key block's
+// score also carries lambda * M_j, M_j = || S1_j - Hbar ||_F (routing.cuh).
 //
 // One CTA handles kSelectQB consecutive query blocks of one head:
 //   1. pool: stream the query blocks once (16-byte coalesced loads, two row
@@ -32,8 +33,8 @@ __host__ __device__ constexpr int select_score_ld(int nB) { return ((nB + 31) / 
 
 template <int D>
 __global__ void __launch_bounds__(kSelectThreads)
-select_kernel(const bf16* __restrict__ Q, const float* __restrict__ kbar, int N, int nB,
-              int block, int topk, int32_t* __restrict__ idx) {
+select_kernel(const bf16* __restrict__ Q, const float* __restrict__ kbar, const float* __restrict__ route,
+              float lambda, int N, int nB, int block, int topk, int32_t* __restrict__ idx) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   float* sQbar = reinterpret_cast<float*>(smem_raw);                    // [QB][D]
   float* sHalf = sQbar + kSelectQB * D;                                 // [QB][D] second-half row sums
@@ -106,6 +107,15 @@ select_kernel(const bf16* __restrict__ Q, const float* __restrict__ kbar, int N,
         a1[q] = fmaf(x.y, k1.y, a1[q]);
         a1[q] = fmaf(x.z, k1.z, a1[q]);
         a1[q] = fmaf(x.w, k1.w, a1[q]);
+      }
+    }
+    if (route != nullptr) {
+      const float b0 = lambda * route[bh * size_t(nB) + j0];
+      const float b1 = has1 ? lambda * route[bh * size_t(nB) + j1] : 0.f;
+#pragma unroll
+      for (int q = 0; q < kSelectQB; ++q) {
+        a0[q] += b0;
+        a1[q] += b1;
       }
     }
 #pragma unroll

@@ -13,6 +13,9 @@ Per-unit figures:
   order 2); flops = 2*n*d*d per block for K^T V (orders 1 and 2).
 * select: bytes = Q read (N*d*2) + kbar read (nB*d*4) + idx written
   (nB*k*4); flops = 2*d per (query block, key block) pooled score.
+* routing (covariance-aware): bytes = per-block S1 read twice (2*nB*d*d*2:
+  once for Hbar, once for the deviations) + Hbar written and read (2*d*d*4)
+  + M written (nB*4).
 * dense-equivalent attention flops: 4*N*N*d per head.
 """
 from __future__ import annotations
@@ -64,6 +67,11 @@ def stats_flops(B, H, N, d, block, order) -> float:
 def select_bytes(B, H, N, d, block, topk) -> float:
     nB = num_blocks(N, block)
     return float(B * H * (N * d * 2 + nB * d * 4 + nB * topk * 4))
+
+
+def routing_bytes(B, H, N, d, block) -> float:
+    nB = num_blocks(N, block)
+    return float(B * H * (2 * nB * d * d * 2 + 2 * d * d * 4 + nB * 4))
 
 
 def select_flops(B, H, N, d, block) -> float:

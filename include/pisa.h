@@ -102,17 +102,34 @@ pisa_status_t pisa_block_stats(const void* K, const void* V, pisa_shape_t shape,
 /*
  * pisa_select -- top-k critical key blocks of every query block.
  *
- * Section 2, "Covariance-aware routing" (selection by attention relevance; the
- * covariance term is not part of this call): the relevance of key block j to query
- * block i is the pooled score qbar_i . kbar_j, with qbar_i the mean of query block
- * i's real rows, computed in fp32. idx[b,h,i,:] receives the topk blocks with the
- * largest scores, equal scores resolved toward the lower block index, written in
+ * Section 2, "Covariance-aware routing": the relevance of key block j to query block
+ * i is the pooled score qbar_i . kbar_j, with qbar_i the mean of query block i's real
+ * rows, plus, when `route` is given, the covariance term lambda * M_j (M from
+ * pisa_routing_norms); computed in fp32. idx[b,h,i,:] receives the topk blocks with
+ * the largest scores, equal scores resolved toward the lower block index, written in
  * ascending block order.
  * Q: bf16 [B, H, N, d]; kbar: fp32 [B, H, nB, d] (from pisa_block_stats);
- * idx: int32 [B, H, nB, topk]; 1 <= topk <= nB.
+ * route: fp32 [B, H, nB] or NULL (plain relevance); lambda: finite, >= 0 (ignored
+ * when route is NULL); idx: int32 [B, H, nB, topk]; 1 <= topk <= nB.
  */
-pisa_status_t pisa_select(const void* Q, const float* kbar, pisa_shape_t shape, int32_t topk,
-                          int32_t* idx, void* stream);
+pisa_status_t pisa_select(const void* Q, const float* kbar, const float* route, float lambda,
+                          pisa_shape_t shape, int32_t topk, int32_t* idx, void* stream);
+
+/*
+ * pisa_routing_norms -- the covariance-aware routing statistic.
+ *
+ * Section 2, "Covariance-aware routing": the selection score of a block carries the
+ * norm of its first-order matrix's deviation from the global statistic,
+ *   Hbar = (1/nB) sum_j S1_j                          fp32  [B, H, d, d]
+ *   M_j  = || S1_j - Hbar ||_F                         fp32  [B, H, nB]
+ * (the pages write a 2-norm without naming it; this is the Frobenius norm). S1 is the
+ * per-block bf16 output of pisa_block_stats at order 1, read as stored, so this Hbar
+ * is the mean of the stored bf16 matrices; it serves as the Hbar argument of
+ * pisa_attention at order 2 as well. Hbar and M are overwritten (zeroed on `stream`,
+ * then accumulated with fp32 atomics: reproducible to fp32 rounding).
+ */
+pisa_status_t pisa_routing_norms(const void* S1, pisa_shape_t shape, float* Hbar, float* M,
+                                 void* stream);
 
 /*
  * pisa_attention -- fused exact + Taylor attention.

@@ -56,8 +56,8 @@ def stats(L, s=None, K=FAKE, V=FAKE, order=1, kbar=FAKE, S0=FAKE, S1=FAKE):
     return L.pisa_block_stats(vp(K), vp(V), s or shape(), order, vp(kbar), vp(S0), vp(S1), None)
 
 
-def sel(L, s=None, Q=FAKE, kbar=FAKE, topk=2, idx=FAKE):
-    return L.pisa_select(vp(Q), vp(kbar), s or shape(), topk, vp(idx), None)
+def sel(L, s=None, Q=FAKE, kbar=FAKE, topk=2, idx=FAKE, route=0, lam=0.0):
+    return L.pisa_select(vp(Q), vp(kbar), vp(route), lam, s or shape(), topk, vp(idx), None)
 
 
 def attn(L, s=None, topk=2, order=1, scale=0.125, fn="pisa_attention", **ptrs):
@@ -128,6 +128,25 @@ def test_hybrid_order_needs_hbar(L):
     _no_device()
     _passes_validation(stats(L, order=2), L)
     _passes_validation(attn(L, order=2), L)
+
+
+def routing(L, s=None, S1=FAKE, Hbar=FAKE, M=FAKE):
+    return L.pisa_routing_norms(vp(S1), s or shape(), vp(Hbar), vp(M), None)
+
+
+def test_routing_arguments(L):
+    for name in ("S1", "Hbar", "M"):
+        assert routing(L, **{name: 0}) == INVALID, name
+        assert routing(L, **{name: MISALIGNED}) == INVALID, name
+    assert routing(L, s=shape(d=96)) == UNSUPPORTED
+    assert routing(L, s=shape(N=0), S1=0, Hbar=0, M=0) == OK
+    assert sel(L, route=MISALIGNED, lam=1.0) == INVALID
+    for lam in (-1.0, float("nan"), float("inf")):
+        assert sel(L, route=FAKE, lam=lam) == INVALID, lam
+    _no_device()
+    _passes_validation(routing(L), L)
+    _passes_validation(sel(L, route=FAKE, lam=0.5), L)
+    _passes_validation(sel(L, lam=-1.0), L)      # lambda is ignored without a route
 
 
 def test_drop_needs_no_statistics(L):

@@ -59,6 +59,7 @@ class Workload:
     kind: str            # "normal" | "image" | "video"
     grid: tuple = ()     # token grid for the smooth generators
     seed: int = 0
+    route_lambda: float = 0.0   # covariance-aware routing weight (0: plain relevance)
 
     @property
     def nB(self) -> int:
@@ -90,6 +91,9 @@ WORKLOADS = {
 WORKLOADS["video_hybrid"] = WORKLOADS["video"].with_(name="video_hybrid", order=2)
 WORKLOADS["video_drop"] = WORKLOADS["video"].with_(name="video_drop", order=-1)
 WORKLOADS["long_hybrid"] = WORKLOADS["long"].with_(name="long_hybrid", order=2)
+# the hybrid order with covariance-aware routing; the weight puts lambda * std(M_j)
+# at about half the spread between a row's best and k-th pooled score
+WORKLOADS["video_routed"] = WORKLOADS["video"].with_(name="video_routed", order=2, route_lambda=0.015)
 
 
 def get(name: str) -> Workload:
