@@ -110,22 +110,22 @@ struct TcCfg {
   // barriers
   static constexpr int B_SE = 0;                  // [NS]  stage consumed (MMA commit)
   static constexpr int B_TF = B_SE + NS;          // [NTF] copies of a load unit landed
-  static constexpr int B_Q = B_TF + NTF;          //       queries in TMEM (256 row threads)
+  static constexpr int B_Q = B_TF + NTF;          //       queries in TMEM (8 row warps)
   static constexpr int B_SF = B_Q + 1;            // [NSB] S ready (commit)
-  static constexpr int B_PF = B_SF + NSB;         // [NSB] P written (256 row threads)
+  static constexpr int B_PF = B_SF + NSB;         // [NSB] P written (8 row warps)
   static constexpr int B_PV = B_PF + NSB;         // [NSB] P V done (commit)
-  static constexpr int B_CVF = B_PV + NSB;        // [2]   kbar / S0 chunk converted (64)
+  static constexpr int B_CVF = B_PV + NSB;        // [2]   kbar / S0 chunk converted (2 warps)
   static constexpr int B_CVE = B_CVF + 2;         // [2]   chunk operands consumed (commit)
   static constexpr int B_SBF = B_CVE + 2;         // [2]   Sbar ready (commit)
-  static constexpr int B_A0F = B_SBF + 2;         // [2]   alpha operand written (256)
+  static constexpr int B_A0F = B_SBF + 2;         // [2]   alpha operand written (8 warps)
   static constexpr int B_SBE = B_A0F + 2;         // [2]   alpha MMA done (commit)
-  static constexpr int B_GA = B_SBE + 2;          // [2]   a pair of A_j written (256)
+  static constexpr int B_GA = B_SBE + 2;          // [2]   a pair of A_j written (8 warps)
   static constexpr int B_AE = B_GA + 2;           // [2]   a pair of A_j consumed (commit)
   static constexpr int B_OSYNC = B_AE + 2;        //       end of the exact stage / of a chunk (commit)
   static constexpr int B_ODONE = B_OSYNC + 1;     //       all MMAs done (commit)
   static constexpr int B_XD = B_ODONE + 1;        //       exact stage done, ring idle (commit; hybrid)
-  static constexpr int B_HF = B_XD + 1;           //       Hbar operand converted (64; hybrid)
-  static constexpr int B_AH = B_HF + 1;           //       A_H = s x written (256; hybrid)
+  static constexpr int B_HF = B_XD + 1;           //       Hbar operand converted (2 warps; hybrid)
+  static constexpr int B_AH = B_HF + 1;           //       A_H = s x written (8 warps; hybrid)
   static constexpr int NBARS = B_AH + 1;
   // shared memory (offsets from a 1024-byte aligned base)
   static constexpr int OFF_RING = 0;
@@ -176,6 +176,13 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
       return;
     }
   }
+}
+
+// one arrival per warp: every lane has finished its part (its tensor-memory stores
+// waited for, its shared-memory writes fenced) before lane 0 arrives
+__device__ __forceinline__ void warp_arrive(uint32_t bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
 // named barrier of the two warps of one TMEM lane quarter (64 threads); returns the
@@ -240,29 +247,30 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   static_assert(C::CHUNK == 32, "chunk == mask word");
 
   // ------------------------------------------------------------- prologue
+  constexpr uint32_t kRowWarps = 8;  // hand-off barriers count one arrival per row warp
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NS; ++s) mbar_init(BAR(C::B_SE + s), 1);
     for (int s = 0; s < C::NTF; ++s) mbar_init(BAR(C::B_TF + s), 1);
     for (int s = 0; s < C::NSB; ++s) {
       mbar_init(BAR(C::B_SF + s), 1);
-      mbar_init(BAR(C::B_PF + s), 256);
+      mbar_init(BAR(C::B_PF + s), kRowWarps);
       mbar_init(BAR(C::B_PV + s), 1);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(BAR(C::B_CVF + s), 64);
+      mbar_init(BAR(C::B_CVF + s), 2);
       mbar_init(BAR(C::B_CVE + s), 1);
       mbar_init(BAR(C::B_SBF + s), 1);
-      mbar_init(BAR(C::B_A0F + s), 256);
+      mbar_init(BAR(C::B_A0F + s), kRowWarps);
       mbar_init(BAR(C::B_SBE + s), 1);
-      mbar_init(BAR(C::B_GA + s), 256);
+      mbar_init(BAR(C::B_GA + s), kRowWarps);
       mbar_init(BAR(C::B_AE + s), 1);
     }
-    mbar_init(BAR(C::B_Q), 256);
+    mbar_init(BAR(C::B_Q), kRowWarps);
     mbar_init(BAR(C::B_OSYNC), 1);
     mbar_init(BAR(C::B_ODONE), 1);
     mbar_init(BAR(C::B_XD), 1);
-    mbar_init(BAR(C::B_HF), 64);
-    mbar_init(BAR(C::B_AH), 256);
+    mbar_init(BAR(C::B_HF), 2);
+    mbar_init(BAR(C::B_AH), kRowWarps);
     misc[1] = 0;
     mbar_init_fence();
   }
@@ -526,7 +534,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     for (int ac = 0; ac < n_active; ++ac) {
       const int c = active[ac];
       const int s = ac & 1;
-      if (!wait_bounded(BAR(C::B_CVE + s), ((ac >> 1) & 1) ^ 1, abort_flag)) break;
+      if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_CVE + s), ((ac >> 1) & 1) ^ 1, abort_flag))) break;
       uint8_t* dk = base + C::OFF_CV + s * C::CV_STAGE;
       uint8_t* ds = dk + C::CV_HALF;
       const float* gk = p.kbar + (size_t(bh) * nB + size_t(c) * C::CHUNK) * D;
@@ -568,9 +576,9 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         }
       }
       fence_proxy_async_smem();
-      mbar_arrive(BAR(C::B_CVF + s));
+      warp_arrive(BAR(C::B_CVF + s));
     }
-    if (hybrid && wait_bounded(BAR(C::B_XD), 0, abort_flag)) {
+    if (hybrid && __all_sync(0xffffffffu, wait_bounded(BAR(C::B_XD), 0, abort_flag))) {
       // Hbar fp32 [D][D] (row a = key dim, column c = value dim) -> bf16 MN-major
       // operand in ring stage 0, laid out as a TMA 128-byte-swizzled load of 64-column
       // panels would place it
@@ -585,7 +593,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         *reinterpret_cast<uint4*>(dh + (c16 >> 3) * (D * 128) + r * 128 + (((c16 & 7) ^ (r & 7)) << 4)) = hv;
       }
       fence_proxy_async_smem();
-      mbar_arrive(BAR(C::B_HF));
+      warp_arrive(BAR(C::B_HF));
     }
   } else {
     // ----------------------------------------------------------- row threads
@@ -631,7 +639,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(BAR(C::B_Q));
+      warp_arrive(BAR(C::B_Q));
     }
 
     const float sl2 = p.scale * 1.4426950408889634f;  // exponents in base 2
@@ -710,7 +718,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       l += (rsp[0] + rsp[1]) + (rsp[2] + rsp[3]);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(BAR(C::B_PF + sb));
+      warp_arrive(BAR(C::B_PF + sb));
     }
     ok = pair_sync_and(pair_id, ok);
 
@@ -795,7 +803,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           tmem_wait_st();
           tc_fence_before();
         }
-        mbar_arrive(BAR(C::B_A0F + b));
+        warp_arrive(BAR(C::B_A0F + b));
 
         if (first && ok) {
 #pragma unroll
@@ -838,7 +846,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
               const int u = n_exact + g;
               ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_TF + u % C::NTF), (u / C::NTF) & 1, abort_flag));
             }
-            mbar_arrive(BAR(C::B_GA + gs));
+            warp_arrive(BAR(C::B_GA + gs));
           }
         }
       }
@@ -859,7 +867,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           }
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(BAR(C::B_AH));
+          warp_arrive(BAR(C::B_AH));
         }
       }
     }
