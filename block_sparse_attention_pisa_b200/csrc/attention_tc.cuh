@@ -248,6 +248,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
 
   // ------------------------------------------------------------- prologue
   constexpr uint32_t kRowWarps = 8;  // hand-off barriers count one arrival per row warp
+  // at order 1 the approximate stage is run by one half of the row threads (4 warps)
+  const uint32_t approx_warps = p.order == 1 ? 4u : kRowWarps;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NS; ++s) mbar_init(BAR(C::B_SE + s), 1);
     for (int s = 0; s < C::NTF; ++s) mbar_init(BAR(C::B_TF + s), 1);
@@ -260,9 +262,9 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       mbar_init(BAR(C::B_CVF + s), 2);
       mbar_init(BAR(C::B_CVE + s), 1);
       mbar_init(BAR(C::B_SBF + s), 1);
-      mbar_init(BAR(C::B_A0F + s), kRowWarps);
+      mbar_init(BAR(C::B_A0F + s), approx_warps);
       mbar_init(BAR(C::B_SBE + s), 1);
-      mbar_init(BAR(C::B_GA + s), kRowWarps);
+      mbar_init(BAR(C::B_GA + s), approx_warps);
       mbar_init(BAR(C::B_AE + s), 1);
     }
     mbar_init(BAR(C::B_Q), kRowWarps);
@@ -722,8 +724,121 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     }
     ok = pair_sync_and(pair_id, ok);
 
-    // ------------------------------------------------ approximate stage
-    if (ok && n_active > 0) {
+    // ------------------------------------------------ approximate stage, order 1
+    // Half 0 of each row runs it alone on full-width operands (O, alpha, A_j): the
+    // per-block operand hand-offs then wait on four warps, not eight. Half 1 hands its
+    // partial denominator over and goes on to the epilogue.
+    if (ok && n_active > 0 && p.order == 1) {
+      xs[hf * 128 + r] = l;
+      ok = pair_sync_and(pair_id, ok);
+      if (hf == 1) {
+        l = 0.f;
+      } else if (ok) {
+        l += xs[128 + r];
+        ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_OSYNC), 0, abort_flag));
+        uint32_t qf[D / 2];  // all packed query dimensions of the row
+        if (ok) {
+          tc_fence_after();
+#pragma unroll
+          for (int ch = 0; ch < D / 32; ++ch)
+            tmem_ld16(tmem + lrow + C::Q_COL + ch * 16, *reinterpret_cast<uint32_t(*)[16]>(&qf[ch * 16]));
+#pragma unroll
+          for (int ch = 0; ch < D / 32; ++ch) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&qf[ch * 16]));
+        }
+        const int nlast = N - (nB - 1) * BLK;
+        int g = 0;
+        for (int ac = 0; ac < n_active && ok; ++ac) {
+          const int c = active[ac];
+          const int b = ac & 1;
+          ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SBF + b), (ac >> 1) & 1, abort_flag));
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t sa = tmem + lrow + C::R_COL + b * C::CHUNK;
+          uint32_t sv[C::CHUNK];
+          tmem_ld16(sa, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
+          tmem_ld16(sa + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
+          tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
+          tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
+          const uint32_t myw = mymask[c];
+          const int kmax = nB - c * C::CHUNK;
+          float mxp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int k = 0; k < C::CHUNK; ++k) {
+            const bool mine = k < kmax && !((myw >> k) & 1u);
+            const float v = mine ? __uint_as_float(sv[k]) * sl2 : -INFINITY;
+            sv[k] = __float_as_uint(v);
+            mxp[k & 3] = fmaxf(mxp[k & 3], v);
+          }
+          const float mx = fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3]));
+          const bool need_o = mx > m + 8.f;
+          if (__any_sync(0xffffffffu, need_o)) {
+            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_OSYNC), ac & 1, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            const float f = need_o ? ex2(m - mx) : 1.f;
+            rescale_row<D>(tmem + lrow + C::O_COL, f);
+            l *= f;
+            if (need_o) m = mx;
+          }
+          float lsp[4] = {0.f, 0.f, 0.f, 0.f};
+          uint32_t a0[C::CHUNK / 2];
+#pragma unroll
+          for (int k = 0; k < C::CHUNK; k += 2) {
+            const float x0 = ex2(__uint_as_float(sv[k]) - m);
+            const float x1 = ex2(__uint_as_float(sv[k + 1]) - m);
+            const float n0 = (c * C::CHUNK + k == nB - 1) ? float(nlast) : float(BLK);
+            const float n1 = (c * C::CHUNK + k + 1 == nB - 1) ? float(nlast) : float(BLK);
+            lsp[(k >> 1) & 3] = fmaf(n1, x1, fmaf(n0, x0, lsp[(k >> 1) & 3]));
+            a0[k >> 1] = pack_bf16x2_int(x0, x1);
+          }
+          l += (lsp[0] + lsp[1]) + (lsp[2] + lsp[3]);
+          // alpha of blocks [16k, 16k + 16) at columns [16k, 16k + 8) (the layout the
+          // zeroth-order MMA reads)
+          tmem_st8(sa, *reinterpret_cast<const uint32_t(*)[8]>(&a0[0]));
+          tmem_st8(sa + 16, *reinterpret_cast<const uint32_t(*)[8]>(&a0[8]));
+          tmem_wait_st();
+          tc_fence_before();
+          warp_arrive(BAR(C::B_A0F + b));
+          // one runtime iteration per pair of approximated blocks (kept rolled: an
+          // unrolled copy evicts the MMA warp's instructions)
+          const int a_end = chunk_off[c + 1];
+#pragma unroll 1
+          for (int a = chunk_off[c]; a < a_end; a += C::GROUP, ++g) {
+            const int n = min(C::GROUP, a_end - a);
+            const int gs = g & 1;
+            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_AE + gs), ((g >> 1) & 1) ^ 1, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int qq = 0; qq < n; ++qq) {
+              const int k = approx_list[a + qq] - c * C::CHUNK;
+              const uint32_t w = a0[k >> 1];
+              const float coef = ((k & 1) ? bf16_hi(w) : bf16_lo(w)) * p.scale;
+              const __nv_bfloat162 c2 = __floats2bfloat162_rn(coef, coef);
+              const uint32_t cw = *reinterpret_cast<const uint32_t*>(&c2);
+              const uint32_t aa = tmem + lrow + C::A_COL0 + (gs * C::GROUP + qq) * C::A_COLS;
+#pragma unroll
+              for (int ch = 0; ch < D / 32; ++ch) {
+                uint32_t t[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) t[i] = hmul2_bf16(qf[ch * 16 + i], cw);
+                tmem_st16(aa + ch * 16, t);
+              }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            // the pair's S1 tiles (load unit n_exact + g) must have landed as well
+            const int u = n_exact + g;
+            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_TF + u % C::NTF), (u / C::NTF) & 1, abort_flag));
+            if (!ok) break;
+            warp_arrive(BAR(C::B_GA + gs));
+          }
+        }
+      }
+    }
+
+    // ------------------------------------------------ approximate stage, orders 0 and 2
+    else if (ok && n_active > 0) {
       // every exact-stage MMA is done: the operand slots may reuse their columns
       ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_OSYNC), 0, abort_flag));
       uint32_t q[HA];  // this half's packed query dimensions
@@ -736,8 +851,6 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         for (int ch = 0; ch < HA / 16; ++ch) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&q[ch * 16]));
       }
       const int nlast = N - (nB - 1) * BLK;
-      const bool first = p.order == 1;
-      int g = 0;
       for (int ac = 0; ac < n_active; ++ac) {
         const int c = active[ac];
         const int b = ac & 1;
@@ -780,11 +893,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           }
           if (need_o) m = mx;
         }
-        // alpha of this half's blocks (and, at order 1, of the other half's: the
-        // first-order operands of every approximated block need them)
+        // alpha of this half's blocks
         float lsp[4] = {0.f, 0.f, 0.f, 0.f};
         float ssp[2] = {0.f, 0.f};
-        uint32_t a0[HC / 2], a1[HC / 2];  // packed alpha: own blocks, other half's blocks
+        uint32_t a0[HC / 2];  // packed alpha of this half's blocks
 #pragma unroll
         for (int k = 0; k < HC; k += 2) {
           const int kk = hf * HC + k;
@@ -804,51 +916,6 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           tc_fence_before();
         }
         warp_arrive(BAR(C::B_A0F + b));
-
-        if (first && ok) {
-#pragma unroll
-          for (int k = 0; k < HC; k += 2) {
-            const int kk = (hf ^ 1) * HC + k;
-            a1[k >> 1] = pack_bf16x2_int(ex2(__uint_as_float(sv[kk]) - m), ex2(__uint_as_float(sv[kk + 1]) - m));
-          }
-          // one runtime iteration per pair of approximated blocks (kept rolled: an
-          // unrolled copy evicts the MMA warp's instructions). alpha comes from the
-          // packed bf16 weights (zero where the row's own block is exact).
-          const int a_end = chunk_off[c + 1];
-#pragma unroll 1
-          for (int a = chunk_off[c]; a < a_end; a += C::GROUP, ++g) {
-            const int n = min(C::GROUP, a_end - a);
-            const int gs = g & 1;
-            if (ok) ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_AE + gs), ((g >> 1) & 1) ^ 1, abort_flag));
-            if (ok) {
-              tc_fence_after();
-#pragma unroll 1
-              for (int qq = 0; qq < n; ++qq) {
-                const int k = approx_list[a + qq] - c * C::CHUNK;
-                const bool own = (k >> 4) == hf;
-                const int kl = k & (HC - 1);
-                const uint32_t w = own ? a0[kl >> 1] : a1[kl >> 1];
-                const float coef = ((kl & 1) ? bf16_hi(w) : bf16_lo(w)) * p.scale;
-                const __nv_bfloat162 c2 = __floats2bfloat162_rn(coef, coef);
-                const uint32_t cw = *reinterpret_cast<const uint32_t*>(&c2);
-                const uint32_t aa = tmem + lrow + C::A_COL0 + (gs * C::GROUP + qq) * C::A_COLS + hf * HA;
-#pragma unroll
-                for (int ch = 0; ch < HA / 16; ++ch) {
-                  uint32_t t[16];
-#pragma unroll
-                  for (int i = 0; i < 16; ++i) t[i] = hmul2_bf16(q[ch * 16 + i], cw);
-                  tmem_st16(aa + ch * 16, t);
-                }
-              }
-              tmem_wait_st();
-              tc_fence_before();
-              // the pair's S1 tiles (load unit n_exact + g) must have landed as well
-              const int u = n_exact + g;
-              ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_TF + u % C::NTF), (u / C::NTF) & 1, abort_flag));
-            }
-            warp_arrive(BAR(C::B_GA + gs));
-          }
-        }
       }
       if (hybrid) {
         // A_H = bf16(s_t * scale * q_t), one rounding from fp32 (operand slot 0); s_t is
