@@ -22,10 +22,11 @@
 //   warps 2-3   build the block lists, then convert fp32 kbar / S0 chunks of 32
 //               blocks into bf16 swizzled shared-memory operands;
 //   warps 4-11  two threads per query row (= TMEM lane): warps w and w + 4 share a
-//               lane quarter and each takes half of the row's score columns and
-//               half of O's columns (online softmax, the Taylor weights and the
-//               tensor-memory operands). A pair agrees on its running maximum
-//               through shared memory at one named barrier per block.
+//               lane quarter. In the exact stage each takes half of the row's score
+//               columns and half of O's columns, and a pair agrees on its running
+//               maximum through shared memory at one named barrier per block. The
+//               approximate stage runs on warps 4-7 alone with full-width operands
+//               (its hand-offs are short; fewer warps to wait for pays more there).
 // Tensor memory (512 columns): O accumulator (D), the tile's queries Q (D/2; the A
 // operand of Q K^T and Q Kbar^T), then either a ring of exact score buffers S
 // (P overwrites its own S) or, in the approximate stage, two pooled-score buffers
@@ -248,8 +249,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
 
   // ------------------------------------------------------------- prologue
   constexpr uint32_t kRowWarps = 8;  // hand-off barriers count one arrival per row warp
-  // at order 1 the approximate stage is run by one half of the row threads (4 warps)
-  const uint32_t approx_warps = p.order == 1 ? 4u : kRowWarps;
+  constexpr uint32_t kApproxWarps = 4;  // the approximate stage runs on one half of the row threads
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NS; ++s) mbar_init(BAR(C::B_SE + s), 1);
     for (int s = 0; s < C::NTF; ++s) mbar_init(BAR(C::B_TF + s), 1);
@@ -262,9 +262,9 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       mbar_init(BAR(C::B_CVF + s), 2);
       mbar_init(BAR(C::B_CVE + s), 1);
       mbar_init(BAR(C::B_SBF + s), 1);
-      mbar_init(BAR(C::B_A0F + s), approx_warps);
+      mbar_init(BAR(C::B_A0F + s), kApproxWarps);
       mbar_init(BAR(C::B_SBE + s), 1);
-      mbar_init(BAR(C::B_GA + s), approx_warps);
+      mbar_init(BAR(C::B_GA + s), kApproxWarps);
       mbar_init(BAR(C::B_AE + s), 1);
     }
     mbar_init(BAR(C::B_Q), kRowWarps);
@@ -272,7 +272,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     mbar_init(BAR(C::B_ODONE), 1);
     mbar_init(BAR(C::B_XD), 1);
     mbar_init(BAR(C::B_HF), 2);
-    mbar_init(BAR(C::B_AH), kRowWarps);
+    mbar_init(BAR(C::B_AH), kApproxWarps);
     misc[1] = 0;
     mbar_init_fence();
   }
@@ -619,7 +619,6 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     constexpr int HK = BLK / 2;     // exact keys per half
     constexpr int HD = D / 2;       // O / value dimensions per half
     constexpr int HA = D / 4;       // packed bf16 Q / A columns per half
-    constexpr int HC = C::CHUNK / 2;
     bool ok = true;
 
     // queries -> TMEM (the A operand of Q K^T and Q Kbar^T): this half's dimensions
@@ -724,11 +723,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     }
     ok = pair_sync_and(pair_id, ok);
 
-    // ------------------------------------------------ approximate stage, order 1
-    // Half 0 of each row runs it alone on full-width operands (O, alpha, A_j): the
-    // per-block operand hand-offs then wait on four warps, not eight. Half 1 hands its
-    // partial denominator over and goes on to the epilogue.
-    if (ok && n_active > 0 && p.order == 1) {
+    // ------------------------------------------------ approximate stage
+    // Half 0 of each row runs it alone on full-width operands (O, alpha, A_j, A_H): the
+    // per-chunk and per-block operand hand-offs then wait on four warps, not eight.
+    // Half 1 hands its partial denominator over and goes on to the epilogue.
+    if (ok && n_active > 0) {
       xs[hf * 128 + r] = l;
       ok = pair_sync_and(pair_id, ok);
       if (hf == 1) {
@@ -778,9 +777,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             const float f = need_o ? ex2(m - mx) : 1.f;
             rescale_row<D>(tmem + lrow + C::O_COL, f);
             l *= f;
+            s_alpha *= f;
             if (need_o) m = mx;
           }
           float lsp[4] = {0.f, 0.f, 0.f, 0.f};
+          float ssp[2] = {0.f, 0.f};
           uint32_t a0[C::CHUNK / 2];
 #pragma unroll
           for (int k = 0; k < C::CHUNK; k += 2) {
@@ -789,9 +790,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             const float n0 = (c * C::CHUNK + k == nB - 1) ? float(nlast) : float(BLK);
             const float n1 = (c * C::CHUNK + k + 1 == nB - 1) ? float(nlast) : float(BLK);
             lsp[(k >> 1) & 3] = fmaf(n1, x1, fmaf(n0, x0, lsp[(k >> 1) & 3]));
+            if (hybrid) ssp[(k >> 1) & 1] += x0 + x1;
             a0[k >> 1] = pack_bf16x2_int(x0, x1);
           }
           l += (lsp[0] + lsp[1]) + (lsp[2] + lsp[3]);
+          s_alpha += ssp[0] + ssp[1];
           // alpha of blocks [16k, 16k + 16) at columns [16k, 16k + 8) (the layout the
           // zeroth-order MMA reads)
           tmem_st8(sa, *reinterpret_cast<const uint32_t(*)[8]>(&a0[0]));
@@ -799,6 +802,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           tmem_wait_st();
           tc_fence_before();
           warp_arrive(BAR(C::B_A0F + b));
+          if (p.order != 1) continue;
           // one runtime iteration per pair of approximated blocks (kept rolled: an
           // unrolled copy evicts the MMA warp's instructions)
           const int a_end = chunk_off[c + 1];
@@ -834,103 +838,16 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             warp_arrive(BAR(C::B_GA + gs));
           }
         }
-      }
-    }
-
-    // ------------------------------------------------ approximate stage, orders 0 and 2
-    else if (ok && n_active > 0) {
-      // every exact-stage MMA is done: the operand slots may reuse their columns
-      ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_OSYNC), 0, abort_flag));
-      uint32_t q[HA];  // this half's packed query dimensions
-      if (ok) {
-        tc_fence_after();
+        if (ok && hybrid) {
+          // A_H = bf16(s_t * scale * q_t), one rounding from fp32 (operand slot 0)
+          const float coef = s_alpha * p.scale;
 #pragma unroll
-        for (int ch = 0; ch < HA / 16; ++ch)
-          tmem_ld16(tmem + lrow + C::Q_COL + hf * HA + ch * 16, *reinterpret_cast<uint32_t(*)[16]>(&q[ch * 16]));
-#pragma unroll
-        for (int ch = 0; ch < HA / 16; ++ch) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&q[ch * 16]));
-      }
-      const int nlast = N - (nB - 1) * BLK;
-      for (int ac = 0; ac < n_active; ++ac) {
-        const int c = active[ac];
-        const int b = ac & 1;
-        if (ok) ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SBF + b), (ac >> 1) & 1, abort_flag));
-        const uint32_t sa = tmem + lrow + C::R_COL + b * C::CHUNK;
-        uint32_t sv[C::CHUNK];   // both halves read all pooled scores of the chunk
-        float mx = -INFINITY;
-        if (ok) {
-          tc_fence_after();
-          tmem_ld16(sa, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
-          tmem_ld16(sa + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
-          tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
-          tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
-          const uint32_t myw = mymask[c];
-          const int kmax = nB - c * C::CHUNK;  // blocks of this chunk that exist
-          float mxp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-          for (int k = 0; k < C::CHUNK; ++k) {
-            const bool mine = k < kmax && !((myw >> k) & 1u);
-            const float v = mine ? __uint_as_float(sv[k]) * sl2 : -INFINITY;
-            sv[k] = __float_as_uint(v);
-            mxp[k & 3] = fmaxf(mxp[k & 3], v);
-          }
-          mx = fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3]));
-          tc_fence_before();
-        }
-        // both halves have read the chunk's pooled scores before either overwrites them
-        ok = pair_sync_and(pair_id, ok);
-        if (!ok) break;
-        tc_fence_after();
-        const bool need_o = mx > m + 8.f;
-        if (__any_sync(0xffffffffu, need_o)) {
-          ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_OSYNC), ac & 1, abort_flag));
-          if (ok) {
-            tc_fence_after();
-            const float f = need_o ? ex2(m - mx) : 1.f;
-            rescale_row<HD>(tmem + lrow + C::O_COL + hf * HD, f);
-            l *= f;
-            s_alpha *= f;
-          }
-          if (need_o) m = mx;
-        }
-        // alpha of this half's blocks
-        float lsp[4] = {0.f, 0.f, 0.f, 0.f};
-        float ssp[2] = {0.f, 0.f};
-        uint32_t a0[HC / 2];  // packed alpha of this half's blocks
-#pragma unroll
-        for (int k = 0; k < HC; k += 2) {
-          const int kk = hf * HC + k;
-          const float x0 = ex2(__uint_as_float(sv[kk]) - m);
-          const float x1 = ex2(__uint_as_float(sv[kk + 1]) - m);
-          const float n0 = (c * C::CHUNK + kk == nB - 1) ? float(nlast) : float(BLK);
-          const float n1 = (c * C::CHUNK + kk + 1 == nB - 1) ? float(nlast) : float(BLK);
-          lsp[(k >> 1) & 3] = fmaf(n1, x1, fmaf(n0, x0, lsp[(k >> 1) & 3]));
-          ssp[(k >> 1) & 1] += x0 + x1;
-          a0[k >> 1] = pack_bf16x2_int(x0, x1);
-        }
-        l += (lsp[0] + lsp[1]) + (lsp[2] + lsp[3]);
-        s_alpha += ssp[0] + ssp[1];
-        if (ok) {
-          tmem_st8(sa + hf * HC, a0);
-          tmem_wait_st();
-          tc_fence_before();
-        }
-        warp_arrive(BAR(C::B_A0F + b));
-      }
-      if (hybrid) {
-        // A_H = bf16(s_t * scale * q_t), one rounding from fp32 (operand slot 0); s_t is
-        // the sum of both halves' alpha weights
-        xs[hf * 128 + r] = s_alpha;
-        ok = pair_sync_and(pair_id, ok);
-        if (ok) {
-          const float coef = (s_alpha + xs[(hf ^ 1) * 128 + r]) * p.scale;
-#pragma unroll
-          for (int ch = 0; ch < HA / 16; ++ch) {
+          for (int ch = 0; ch < D / 32; ++ch) {
             uint32_t t[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-              t[i] = pack_bf16x2(bf16_lo(q[ch * 16 + i]) * coef, bf16_hi(q[ch * 16 + i]) * coef);
-            tmem_st16(tmem + lrow + C::A_COL0 + hf * HA + ch * 16, t);
+              t[i] = pack_bf16x2(bf16_lo(qf[ch * 16 + i]) * coef, bf16_hi(qf[ch * 16 + i]) * coef);
+            tmem_st16(tmem + lrow + C::A_COL0 + ch * 16, t);
           }
           tmem_wait_st();
           tc_fence_before();
