@@ -128,28 +128,32 @@ pisa_status_t set_smem(Kernel k, size_t bytes) {
   return ok();
 }
 
+template <int D, int BLK, int MODE>
+pisa_status_t launch_stats_mode(const pisa_shape_t& s, const bf16* K, const bf16* V, float* kbar, float* S0,
+                                bf16* S1, float* Hbar, cudaStream_t st) {
+  using P = pisa::StatsPipeCfg<D, BLK>;
+  auto k = pisa::stats_pipe_kernel<D, BLK, MODE>;
+  PISA_TRY(set_smem(k, P::kSmem));
+  const int nB = int(num_blocks(s));
+  const int G = P::blocks_per_cta(MODE);
+  dim3 grid((nB + G - 1) / G, s.B * s.H);
+  k<<<grid, pisa::StatsCfg<D, BLK>::kThreads, P::kSmem, st>>>(K, V, s.N, nB, kbar, S0, S1, Hbar);
+  return check_launch("stats_pipe_kernel");
+}
+
 template <int D, int BLK>
 pisa_status_t launch_stats(const pisa_shape_t& s, const bf16* K, const bf16* V, int order, float* kbar,
                            float* S0, void* S1, cudaStream_t st) {
-  using C = pisa::StatsCfg<D, BLK>;
-  const int nB = int(num_blocks(s));
   if (order == PISA_ORDER_HYBRID) {
     // Hbar is accumulated with atomics: zero it first, on the same stream
     const size_t bytes = size_t(s.B) * s.H * D * D * sizeof(float);
     cudaError_t e = cudaMemsetAsync(S1, 0, bytes, st);
     if (e != cudaSuccess) return fail(PISA_ERR_CUDA, "cudaMemsetAsync(Hbar): %s", cudaGetErrorString(e));
-    auto k = pisa::stats_hbar_kernel<D, BLK>;
-    using H = pisa::HbarCfg<D, BLK>;
-    PISA_TRY(set_smem(k, H::kSmem));
-    dim3 grid((nB + pisa::kHbarBlocks - 1) / pisa::kHbarBlocks, s.B * s.H);
-    k<<<grid, C::kThreads, H::kSmem, st>>>(K, V, s.N, nB, kbar, S0, static_cast<float*>(S1));
-    return check_launch("stats_hbar_kernel");
+    return launch_stats_mode<D, BLK, pisa::kStatsHbar>(s, K, V, kbar, S0, nullptr, static_cast<float*>(S1), st);
   }
-  auto k = pisa::stats_kernel<D, BLK>;
-  PISA_TRY(set_smem(k, C::kSmem));
-  dim3 grid(nB, s.B * s.H);
-  k<<<grid, C::kThreads, C::kSmem, st>>>(K, V, s.N, nB, order, kbar, S0, static_cast<bf16*>(S1));
-  return check_launch("stats_kernel");
+  if (order == PISA_ORDER_FIRST)
+    return launch_stats_mode<D, BLK, pisa::kStatsS1>(s, K, V, kbar, S0, static_cast<bf16*>(S1), nullptr, st);
+  return launch_stats_mode<D, BLK, pisa::kStatsSums>(s, K, V, kbar, S0, nullptr, nullptr, st);
 }
 
 template <int D>
