@@ -21,7 +21,7 @@ ORDER_DROP, ORDER_ZERO, ORDER_FIRST, ORDER_HYBRID = -1, 0, 1, 2
 
 __all__ = [
     "ORDER_DROP", "ORDER_ZERO", "ORDER_FIRST", "ORDER_HYBRID", "PisaError", "Shape", "lib", "block_stats", "select", "attention", "attention_simt",
-    "pisa", "pisa_host", "device_error", "num_blocks", "LIB_PATH", "SYMBOLS", "routing_norms",
+    "pisa", "pisa_host", "head_chunks", "device_error", "num_blocks", "LIB_PATH", "SYMBOLS", "routing_norms",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpisa.so")
@@ -185,7 +185,7 @@ def attention_simt(Q, K, V, kbar, S0, S1, idx, block: int, order: int, scale: fl
 
 
 def pisa(Q, K, V, block: int, topk: int, order: int = 1, scale: float | None = None,
-         route_lambda: float = 0.0):
+         route_lambda: float = 0.0, out=None):
     """The whole path on device tensors: stats -> select -> attention. Returns (O, idx).
     With ``route_lambda`` > 0 the selection is covariance-aware: stats at order 1 ->
     routing norms -> routed select -> attention (at order 2 with the routing call's
@@ -197,24 +197,67 @@ def pisa(Q, K, V, block: int, topk: int, order: int = 1, scale: float | None = N
         Hbar, M = routing_norms(S1, block, Q.shape[2])
         idx = select(Q, kbar, block, topk, route=M, lam=route_lambda)
         first = Hbar if order == ORDER_HYBRID else (S1 if order == ORDER_FIRST else None)
-        return attention(Q, K, V, kbar, S0, first, idx, block, order, scale), idx
+        return attention(Q, K, V, kbar, S0, first, idx, block, order, scale, out=out), idx
     kbar, S0, S1 = block_stats(K, V, block, order)
     idx = select(Q, kbar, block, topk)
-    return attention(Q, K, V, kbar, S0, S1, idx, block, order, scale), idx
+    return attention(Q, K, V, kbar, S0, S1, idx, block, order, scale, out=out), idx
+
+
+def head_chunks(BH: int, chunks: int):
+    """Split the flattened (batch, head) axis into `chunks` contiguous ranges of near-equal size."""
+    chunks = max(1, min(chunks, BH))
+    edges = [BH * c // chunks for c in range(chunks + 1)]
+    return [(edges[c], edges[c + 1]) for c in range(chunks) if edges[c + 1] > edges[c]]
 
 
 def pisa_host(Q, K, V, block: int, topk: int, order: int = 1, scale: float | None = None,
-              device="cuda", route_lambda: float = 0.0):
-    """The whole path on HOST tensors: copies Q, K, V to the device, runs it, and copies
-    the output back (pinned host memory gives asynchronous copies). Returns O on the host."""
+              device="cuda", route_lambda: float = 0.0, chunks: int = 8):
+    """The whole path on HOST tensors [B, H, N, d]: copies Q, K, V to the device, runs it,
+    and copies the output back. Returns O on the host.
+
+    (batch, head) pairs are independent in every step, so the call is pipelined over
+    `chunks` ranges of them: the host-to-device copy of range c + 1 and the
+    device-to-host copy of range c - 1 run on their own streams while range c
+    computes. With pinned host tensors the copies are asynchronous and overlap the
+    kernels; the result is identical to running the whole batch at once."""
     import torch
-    dq = Q.to(device, non_blocking=True)
-    dk = K.to(device, non_blocking=True)
-    dv = V.to(device, non_blocking=True)
-    O, _ = pisa(dq, dk, dv, block, topk, order, scale, route_lambda)
-    out = torch.empty(O.shape, dtype=O.dtype, pin_memory=Q.is_pinned())
-    out.copy_(O, non_blocking=True)
-    torch.cuda.current_stream(O.device).synchronize()
+    if Q.dim() != 4 or not (Q.is_contiguous() and K.is_contiguous() and V.is_contiguous()):
+        raise ValueError("expected contiguous [B, H, N, d] host tensors")
+    B, H, N, d = Q.shape
+    BH = B * H
+    dev = torch.device(device)
+    if dev.index is None:
+        dev = torch.device("cuda", torch.cuda.current_device())
+    flat = [t.view(BH, N, d) for t in (Q, K, V)]
+    dbuf = [torch.empty((BH, N, d), device=dev, dtype=t.dtype) for t in (Q, K, V)]
+    dO = torch.empty((BH, N, d), device=dev, dtype=Q.dtype)
+    out = torch.empty(Q.shape, dtype=Q.dtype, pin_memory=Q.is_pinned())
+    out_flat = out.view(BH, N, d)
+    compute = torch.cuda.current_stream(dev)
+    h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ranges = head_chunks(BH, chunks)
+    landed = [torch.cuda.Event() for _ in ranges]
+    done = [torch.cuda.Event() for _ in ranges]
+    h2d.wait_stream(compute)  # the device buffers are fresh allocations of this stream
+    with torch.cuda.stream(h2d):
+        for c, (a, b) in enumerate(ranges):
+            for src, dst in zip(flat, dbuf):
+                dst[a:b].copy_(src[a:b], non_blocking=True)
+            landed[c].record(h2d)
+    for c, (a, b) in enumerate(ranges):
+        compute.wait_event(landed[c])
+        q, k, v = (t[a:b].view(1, b - a, N, d) for t in dbuf)
+        with torch.cuda.stream(compute):
+            pisa(q, k, v, block, topk, order, scale, route_lambda, out=dO[a:b].view(1, b - a, N, d))
+        done[c].record(compute)
+        d2h.wait_event(done[c])
+        with torch.cuda.stream(d2h):
+            out_flat[a:b].copy_(dO[a:b], non_blocking=True)
+    compute.wait_stream(d2h)
+    for t in dbuf + [dO]:
+        t.record_stream(h2d)
+        t.record_stream(d2h)
+    compute.synchronize()
     return out
 
 

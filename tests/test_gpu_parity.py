@@ -200,3 +200,16 @@ def test_host_entry_point_matches_device():
     Oh = P.pisa_host(hq, hk, hv, wl.block, wl.topk, wl.order, wl.scale)
     Od, _ = P.pisa(hq.cuda(), hk.cuda(), hv.cuda(), wl.block, wl.topk, wl.order, wl.scale)
     assert torch.equal(Oh.view(torch.int16), Od.cpu().view(torch.int16))
+
+
+def test_host_entry_point_pipelined_over_heads():
+    """The host entry point splits (batch, head) pairs into ranges that copy and compute
+    on separate streams; every chunking gives the device path's bits."""
+    wl = W.get("image").with_(B=2, H=3)
+    q, k, v = W.make_inputs(wl)
+    hq, hk, hv = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in (q, k, v))
+    Od, _ = P.pisa(hq.cuda(), hk.cuda(), hv.cuda(), wl.block, wl.topk, wl.order, wl.scale)
+    ref = Od.cpu().view(torch.int16)
+    for chunks in (1, 4, 6, 16):
+        Oh = P.pisa_host(hq, hk, hv, wl.block, wl.topk, wl.order, wl.scale, chunks=chunks)
+        assert torch.equal(Oh.view(torch.int16), ref), chunks
