@@ -95,7 +95,10 @@ struct TcCfg {
   static constexpr int CV_STAGE = 2 * CV_HALF;
   static constexpr int GROUP = 2;                           // approximated blocks per hand-off
   static constexpr int NA = 2 * GROUP;                      // A operand slots (two groups)
-  static constexpr int NSB = (BLK == 64) ? 4 : 2;           // exact score buffers
+  // exact score buffers. At d = 128 as many as the columns after Q hold (the approximate
+  // stage's operand slots reuse the same columns later): five at b = 64 measured 1-2%
+  // faster than four. At d = 64 a deeper ring measured slower (b = 128: 3.20 vs 3.14 ms).
+  static constexpr int NSB = (D == 128) ? (512 - (D + D / 2)) / BLK : ((BLK == 64) ? 4 : 2);
   static constexpr int MAXB = 2048;
   static constexpr int MAXC = MAXB / CHUNK;
   // tensor-memory columns
@@ -446,7 +449,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         return true;
       };
       // the scores run kLook blocks ahead of the row threads' softmax
-      constexpr int kLook = C::NSB >= 4 ? C::NSB - 2 : 1;
+      constexpr int kLook = C::NSB >= 3 ? C::NSB - 2 : 1;
       for (int e = 0; e < kLook && e < n_exact && ok; ++e) ok = qk(e);
       for (int e = 0; e < n_exact && ok; ++e) {
         ok = pv(e);
