@@ -16,8 +16,9 @@
 //
 // One CTA computes a tile of 128 query rows of one head (two query blocks at
 // b = 64, one at b = 128). Warp roles:
-//   warp 0      TMA producer: K_j and V_j of the exact blocks, then S1_j of the
-//               approximated blocks, through a ring of shared-memory stages;
+//   warp 0      TMA producer: K_j and V_j of the exact blocks (in one stage when they
+//               fit), then S1_j of the approximated blocks, through a ring of
+//               shared-memory stages;
 //   warp 1      MMA issuer (one thread): every tcgen05.mma of the tile;
 //   warps 2-3   build the block lists, then convert fp32 kbar / S0 chunks of 32
 //               blocks into bf16 swizzled shared-memory operands;
@@ -57,9 +58,11 @@
 // tensor-pipe time: per exact block once for K_j and V_j (one barrier) and once
 // for P; per pair of approximated blocks once (the row threads signal a pair only
 // after writing both A operands and seeing both S1 tiles land). The exact scores
-// run two blocks ahead of the softmax (b = 64). Every wait is bounded by clock64; on timeout a
-// CTA raises the device error word, drains its copies and MMAs, frees TMEM and
-// exits.
+// run NSB - 2 blocks ahead of the softmax (three at d = 128, b = 64). Hand-off
+// barriers count one arrival per warp. Every wait is bounded by clock64; on timeout
+// a CTA raises the device error word, drains its copies and MMAs, frees TMEM and
+// exits. The two warps of a row pair leave together: their named barriers AND-reduce
+// the status.
 #pragma once
 
 #include "tc_ptx.cuh"
