@@ -29,3 +29,21 @@ def test_ragged_counts_real_tokens():
     # long workload: 75600 tokens in 591 blocks of <= 128
     f = R.attention_flops(1, 40, 75600, 128, 128, 60, 1)
     assert f / 1e12 == pytest.approx(65.33, abs=0.05)
+
+
+def test_hybrid_and_drop_flops():
+    # hybrid: exact + order-0 + one d x d product per query; keep-or-drop: exact only
+    exact = 24 * 32768 * 4 * 64 * 128 * 64
+    zero = 24 * 32768 * 4 * 128 * 448
+    hbar = 24 * 32768 * 2 * 128 * 128
+    assert R.attention_flops(1, 24, 32768, 128, 64, 64, 2) == pytest.approx(exact + zero + hbar)
+    assert R.attention_flops(1, 24, 32768, 128, 64, 64, -1) == pytest.approx(exact)
+    # nothing left to approximate: the hybrid term vanishes
+    assert R.attention_flops(1, 16, 16384, 64, 128, 128, 2) == pytest.approx(R.dense_flops(1, 16, 16384, 64))
+
+
+def test_routing_and_hybrid_bytes():
+    # per-block S1 read twice (2 x 403 MB) + Hbar + M
+    assert R.routing_bytes(1, 24, 32768, 128, 64) / 1e6 == pytest.approx(808.5, abs=1.0)
+    # order 2 writes Hbar (64 KB per head) instead of per-block S1
+    assert R.stats_bytes(1, 24, 32768, 128, 64, 2) / 1e6 == pytest.approx(416.8, abs=1.0)
