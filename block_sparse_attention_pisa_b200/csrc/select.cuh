@@ -12,10 +12,12 @@
 //   1. pool: stream the query blocks once (16-byte coalesced loads, two row
 //      halves per (block, 16-byte column) pair) and average their rows into
 //      qbar (fp32, shared memory);
-//   2. score: each thread takes two key blocks per pass and forms kSelectQB dot
-//      products against each (fp32 FMA; kbar read through the read-only cache --
-//      a head's kbar is shared by all its CTAs and stays in L2). Scores are
-//      stored as order-preserving uint32 keys;
+//   2. score: each warp takes 32 consecutive key blocks per pass (lane = key block).
+//      Their kbar rows (L2-resident: a head's kbar is shared by all its CTAs)
+//      stream through a per-warp shared-memory tile 32 dimensions at a time, with
+//      coalesced 16-byte loads (four rows per load instruction); each lane then forms
+//      kSelectQB fp32 dot products against its own row (conflict-free 16-byte shared
+//      reads, query rows broadcast). Scores are stored as order-preserving uint32 keys;
 //   3. top-k: one warp per row finds the k-th largest key bit by bit (a count of
 //      keys >= candidate per bit, starting below the row's common key prefix),
 //      then emits the selected block indices in ascending order with ballots;
@@ -28,6 +30,9 @@ namespace pisa {
 
 constexpr int kSelectQB = 8;         // query blocks per CTA
 constexpr int kSelectThreads = 256;
+constexpr int kSelectSlab = 32;                       // kbar dimensions per tile pass
+constexpr int kSelectTileLd = kSelectSlab + 4;        // padded tile row (floats)
+constexpr int kSelectTileFloats = 32 * kSelectTileLd;  // one warp's tile
 
 __host__ __device__ constexpr int select_score_ld(int nB) { return ((nB + 31) / 32) * 32 + 4; }
 
@@ -40,6 +45,7 @@ select_kernel(const bf16* __restrict__ Q, const float* __restrict__ kbar, const 
   float* sHalf = sQbar + kSelectQB * D;                                 // [QB][D] second-half row sums
   uint32_t* sKey = reinterpret_cast<uint32_t*>(sHalf + kSelectQB * D);  // [QB][ld]
   const int ld = select_score_ld(nB);
+  float* sTile = reinterpret_cast<float*>(sKey + kSelectQB * ld);        // [8 warps][32][TileLd]
 
   const size_t bh = blockIdx.y;
   const int i0 = blockIdx.x * kSelectQB;
@@ -82,46 +88,47 @@ select_kernel(const bf16* __restrict__ Q, const float* __restrict__ kbar, const 
   }
   __syncthreads();
 
-  // ---- 2. pooled scores: each thread two key blocks per pass ----
-  const float* kb_head = kbar + bh * size_t(nB) * D;
-  for (int j0 = tid; j0 < nB; j0 += 2 * kSelectThreads) {
-    const int j1 = j0 + kSelectThreads;
-    const bool has1 = j1 < nB;
-    float a0[kSelectQB], a1[kSelectQB];
+  // ---- 2. pooled scores: lane = key block, kbar rows through a per-warp tile ----
+  {
+    const float* kb_head = kbar + bh * size_t(nB) * D;
+    float* tile = sTile + warp * kSelectTileFloats;
+    for (int jb = warp * 32; jb < nB; jb += kSelectThreads) {
+      float acc[kSelectQB];
 #pragma unroll
-    for (int q = 0; q < kSelectQB; ++q) a0[q] = a1[q] = 0.f;
-    const float4* k0row = reinterpret_cast<const float4*>(kb_head + size_t(j0) * D);
-    const float4* k1row = reinterpret_cast<const float4*>(kb_head + size_t(has1 ? j1 : j0) * D);
-#pragma unroll 4
-    for (int a4 = 0; a4 < D / 4; ++a4) {
-      const float4 k0 = __ldg(k0row + a4);
-      const float4 k1 = __ldg(k1row + a4);
+      for (int q = 0; q < kSelectQB; ++q) acc[q] = 0.f;
+#pragma unroll 1
+      for (int d0 = 0; d0 < D; d0 += kSelectSlab) {
+        // rows (lane >> 3) + 4 i, 16-byte chunk (lane & 7): four whole 128-byte row slabs
+        // per load instruction
 #pragma unroll
-      for (int q = 0; q < kSelectQB; ++q) {
-        const float4 x = reinterpret_cast<const float4*>(sQbar + q * D)[a4];
-        a0[q] = fmaf(x.x, k0.x, a0[q]);
-        a0[q] = fmaf(x.y, k0.y, a0[q]);
-        a0[q] = fmaf(x.z, k0.z, a0[q]);
-        a0[q] = fmaf(x.w, k0.w, a0[q]);
-        a1[q] = fmaf(x.x, k1.x, a1[q]);
-        a1[q] = fmaf(x.y, k1.y, a1[q]);
-        a1[q] = fmaf(x.z, k1.z, a1[q]);
-        a1[q] = fmaf(x.w, k1.w, a1[q]);
+        for (int i = 0; i < 8; ++i) {
+          const int r = (lane >> 3) + 4 * i;
+          float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (jb + r < nB) x = __ldg(reinterpret_cast<const float4*>(kb_head + size_t(jb + r) * D + d0) + (lane & 7));
+          *reinterpret_cast<float4*>(tile + r * kSelectTileLd + (lane & 7) * 4) = x;
+        }
+        __syncwarp();
+        const float4* krow = reinterpret_cast<const float4*>(tile + lane * kSelectTileLd);
+#pragma unroll
+        for (int c = 0; c < kSelectSlab / 4; ++c) {
+          const float4 k = krow[c];
+#pragma unroll
+          for (int q = 0; q < kSelectQB; ++q) {
+            const float4 x = reinterpret_cast<const float4*>(sQbar + q * D + d0)[c];
+            acc[q] = fmaf(x.x, k.x, acc[q]);
+            acc[q] = fmaf(x.y, k.y, acc[q]);
+            acc[q] = fmaf(x.z, k.z, acc[q]);
+            acc[q] = fmaf(x.w, k.w, acc[q]);
+          }
+        }
+        __syncwarp();  // the tile is rewritten by the next slab
       }
-    }
-    if (route != nullptr) {
-      const float b0 = lambda * route[bh * size_t(nB) + j0];
-      const float b1 = has1 ? lambda * route[bh * size_t(nB) + j1] : 0.f;
+      const int j = jb + lane;
+      if (j < nB) {
+        const float bias = route != nullptr ? lambda * route[bh * size_t(nB) + j] : 0.f;
 #pragma unroll
-      for (int q = 0; q < kSelectQB; ++q) {
-        a0[q] += b0;
-        a1[q] += b1;
+        for (int q = 0; q < kSelectQB; ++q) sKey[q * ld + j] = float_order_key(acc[q] + bias + 0.f);  // -0 -> +0
       }
-    }
-#pragma unroll
-    for (int q = 0; q < kSelectQB; ++q) {
-      sKey[q * ld + j0] = float_order_key(a0[q] + 0.f);  // -0 -> +0
-      if (has1) sKey[q * ld + j1] = float_order_key(a1[q] + 0.f);
     }
   }
   __syncthreads();
@@ -174,7 +181,8 @@ select_kernel(const bf16* __restrict__ Q, const float* __restrict__ kbar, const 
 }
 
 inline size_t select_smem_bytes(int D, int nB) {
-  return size_t(2) * kSelectQB * D * sizeof(float) + size_t(kSelectQB) * select_score_ld(nB) * sizeof(uint32_t);
+  return size_t(2) * kSelectQB * D * sizeof(float) + size_t(kSelectQB) * select_score_ld(nB) * sizeof(uint32_t) +
+         size_t(kSelectThreads / 32) * kSelectTileFloats * sizeof(float);
 }
 
 }  // namespace pisa
