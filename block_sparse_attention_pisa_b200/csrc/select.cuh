@@ -14,8 +14,9 @@
 //      qbar (fp32, shared memory);
 //   2. score: each warp takes 32 consecutive key blocks per pass (lane = key block).
 //      Their kbar rows (L2-resident: a head's kbar is shared by all its CTAs)
-//      stream through a per-warp shared-memory tile 32 dimensions at a time, with
-//      coalesced 16-byte loads (four rows per load instruction); each lane then forms
+//      stream through two per-warp shared-memory tiles 16 dimensions at a time, with
+//      coalesced 16-byte cp.async copies (eight rows per instruction; the next slab is
+//      in flight while the current one is used); each lane then forms
 //      kSelectQB fp32 dot products against its own row (conflict-free 16-byte shared
 //      reads, query rows broadcast). Scores are stored as order-preserving uint32 keys;
 //   3. top-k: one warp per row finds the k-th largest key bit by bit (a count of
@@ -30,9 +31,9 @@ namespace pisa {
 
 constexpr int kSelectQB = 8;         // query blocks per CTA
 constexpr int kSelectThreads = 256;
-constexpr int kSelectSlab = 32;                       // kbar dimensions per tile pass
-constexpr int kSelectTileLd = kSelectSlab + 4;        // padded tile row (floats)
-constexpr int kSelectTileFloats = 32 * kSelectTileLd;  // one warp's tile
+constexpr int kSelectSlab = 16;                           // kbar dimensions per tile pass
+constexpr int kSelectTileLd = kSelectSlab + 4;            // padded tile row (floats)
+constexpr int kSelectTileFloats = 2 * 32 * kSelectTileLd;  // one warp's two tiles
 
 __host__ __device__ constexpr int select_score_ld(int nB) { return ((nB + 31) / 32) * 32 + 4; }
 
@@ -88,27 +89,43 @@ select_kernel(const bf16* __restrict__ Q, const float* __restrict__ kbar, const 
   }
   __syncthreads();
 
-  // ---- 2. pooled scores: lane = key block, kbar rows through a per-warp tile ----
+  // ---- 2. pooled scores: lane = key block, kbar rows through per-warp tiles ----
   {
     const float* kb_head = kbar + bh * size_t(nB) * D;
-    float* tile = sTile + warp * kSelectTileFloats;
+    float* tiles = sTile + warp * kSelectTileFloats;
+    const uint32_t tiles_u = smem_u32(tiles);
+    constexpr int NSLAB = D / kSelectSlab;
     for (int jb = warp * 32; jb < nB; jb += kSelectThreads) {
+      // rows (lane >> 2) + 8 i, 16-byte chunk (lane & 3) of the slab; rows past nB are
+      // zero-filled
+      auto issue = [&](int sl) {
+        const uint32_t dst = tiles_u + uint32_t((sl & 1) * 32 * kSelectTileLd) * 4u;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = (lane >> 2) + 8 * i;
+          const bool in = jb + r < nB;
+          const float* src = kb_head + size_t(in ? jb + r : 0) * D + sl * kSelectSlab + (lane & 3) * 4;
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst + uint32_t(r * kSelectTileLd + (lane & 3) * 4) * 4u),
+                       "l"(src), "r"(in ? 16u : 0u)
+                       : "memory");
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+      };
       float acc[kSelectQB];
 #pragma unroll
       for (int q = 0; q < kSelectQB; ++q) acc[q] = 0.f;
+      issue(0);
 #pragma unroll 1
-      for (int d0 = 0; d0 < D; d0 += kSelectSlab) {
-        // rows (lane >> 3) + 4 i, 16-byte chunk (lane & 7): four whole 128-byte row slabs
-        // per load instruction
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int r = (lane >> 3) + 4 * i;
-          float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (jb + r < nB) x = __ldg(reinterpret_cast<const float4*>(kb_head + size_t(jb + r) * D + d0) + (lane & 7));
-          *reinterpret_cast<float4*>(tile + r * kSelectTileLd + (lane & 7) * 4) = x;
+      for (int sl = 0; sl < NSLAB; ++sl) {
+        if (sl + 1 < NSLAB) {
+          issue(sl + 1);
+          asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+          asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
         __syncwarp();
-        const float4* krow = reinterpret_cast<const float4*>(tile + lane * kSelectTileLd);
+        const float4* krow = reinterpret_cast<const float4*>(tiles + (sl & 1) * 32 * kSelectTileLd + lane * kSelectTileLd);
+        const int d0 = sl * kSelectSlab;
 #pragma unroll
         for (int c = 0; c < kSelectSlab / 4; ++c) {
           const float4 k = krow[c];
@@ -121,7 +138,7 @@ select_kernel(const bf16* __restrict__ Q, const float* __restrict__ kbar, const 
             acc[q] = fmaf(x.w, k.w, acc[q]);
           }
         }
-        __syncwarp();  // the tile is rewritten by the next slab
+        __syncwarp();  // this tile is refilled two slabs later
       }
       const int j = jb + lane;
       if (j < nB) {
