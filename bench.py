@@ -3,12 +3,22 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload video] [--kernel fused|simt]
 
-One step = one pass of the whole path (block statistics, block selection,
-fused attention) over one batch of the named workload, inputs already resident
-in HBM. Default workload "video": B=1, H=24, N=32768 (8x64x64 latent grid),
-d=128, block 64, top-k 64 of 512 blocks (12.5% exact), order 1, seeded
-synthetic smooth tokens. Inputs (Q, K, V: 604 MB) are larger than L2, so no
-flush is needed between steps.
+One step = one pass of the whole path (block statistics, the covariance-aware
+routing statistic when the workload routes, block selection, fused attention)
+over one batch of the named workload, inputs already resident in HBM. Default
+workload "video": B=1, H=24, N=32768 (8x64x64 latent grid), d=128, block 64,
+top-k 64 of 512 blocks (12.5% exact), order 1, seeded synthetic smooth tokens.
+Other workloads: video_hybrid (order 2, global Hbar), video_routed (order 2 with
+covariance-aware routing), video_drop (keep-or-drop), image, dense (+ k8
+variants), long, long_hybrid. Inputs (Q, K, V: 604 MB at video) are larger than
+L2, so no flush is needed between steps.
+
+The JSON line reports the step throughput (algorithmic TFLOP/s), per-kernel
+times, the attention kernel's roofline against the measured sustained bf16 peak,
+the stats / select / routing kernels' GB/s against the measured HBM copy rate,
+the end-to-end rate through the host entry point (pinned host buffers, copies
+inside the timed region, pipelined over (batch, head) ranges), the CPU oracle on
+a bounded sample, and the SM clocks sampled during the timed region.
 
 N > 1 (torchrun, one process per GPU): every rank runs its own batch (weak
 scaling); the heads and batches are independent, so there is no collective in
