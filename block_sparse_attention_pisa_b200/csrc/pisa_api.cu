@@ -419,6 +419,6 @@ const char* pisa_status_string(pisa_status_t status) {
 
 const char* pisa_last_error(void) { return g_last_error.c_str(); }
 
-int32_t pisa_version(void) { return 100; }
+int32_t pisa_version(void) { return 200; }  // 0.2.0: orders -1 and 2, covariance-aware routing
 
 }  // extern "C"

@@ -148,9 +148,10 @@ pisa_status_t pisa_routing_norms(const void* S1, pisa_shape_t shape, float* Hbar
  * All exponents are taken relative to one running row maximum (a single online-softmax
  * accumulator). idx rows must hold topk distinct blocks in [0, nB) (the order inside a
  * row does not matter); out-of-range entries are ignored and flagged in the device
- * error word. S1 is the per-block bf16 S1 at order 1 and the fp32 Hbar at order 2 (both
- * from pisa_block_stats at the same order); it may be NULL at orders 0 and -1, and kbar
- * and S0 may be NULL at order -1. scale must be finite and > 0.
+ * error word. S1 is the per-block bf16 S1 at order 1 and the fp32 Hbar at order 2 (from
+ * pisa_block_stats at the same order, or the Hbar of pisa_routing_norms); it may be NULL
+ * at orders 0 and -1, and kbar and S0 may be NULL at order -1. scale must be finite and
+ * > 0.
  */
 pisa_status_t pisa_attention(const void* Q, const void* K, const void* V, const float* kbar,
                              const float* S0, const void* S1, const int32_t* idx,
