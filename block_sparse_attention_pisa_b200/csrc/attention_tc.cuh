@@ -45,9 +45,9 @@
 //   hand-off, O += A_j S1_j (TS-MMA, S1 MN-major): the first-order term as one
 //   long-K GEMM.
 // Hybrid order: the approximate stage runs at order 0 while each row also sums its
-//   alpha weights (s_t); at the end the converter warps write Hbar as a bf16
-//   operand into the (then idle) first ring stage, the row threads write
-//   A_H = bf16(s_t x_t), and one M128 x D x D MMA adds A_H Hbar to O.
+//   alpha weights (s_t); the row threads that sit out the approximate stage write
+//   Hbar as a bf16 operand into the (then idle) first ring stage, the others write
+//   A_H = bf16(s_t x_t) at the end, and one M128 x D x D MMA adds A_H Hbar to O.
 // Keep-or-drop: no approximate stage at all.
 // Denominator: sum of P plus sum n_j alpha_j, kept in fp32 registers. One running
 // row maximum covers both stages; the accumulator is rescaled only when the
@@ -131,8 +131,8 @@ struct TcCfg {
   static constexpr int B_OSYNC = B_AE + 2;        //       end of the exact stage / of a chunk (commit)
   static constexpr int B_ODONE = B_OSYNC + 1;     //       all MMAs done (commit)
   static constexpr int B_XD = B_ODONE + 1;        //       exact stage done, ring idle (commit; hybrid)
-  static constexpr int B_HF = B_XD + 1;           //       Hbar operand converted (2 warps; hybrid)
-  static constexpr int B_AH = B_HF + 1;           //       A_H = s x written (8 warps; hybrid)
+  static constexpr int B_HF = B_XD + 1;           //       Hbar operand converted (4 warps; hybrid)
+  static constexpr int B_AH = B_HF + 1;           //       A_H = s x written (4 warps; hybrid)
   static constexpr int NBARS = B_AH + 1;
   // shared memory (offsets from a 1024-byte aligned base)
   static constexpr int OFF_RING = 0;
@@ -277,7 +277,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     mbar_init(BAR(C::B_OSYNC), 1);
     mbar_init(BAR(C::B_ODONE), 1);
     mbar_init(BAR(C::B_XD), 1);
-    mbar_init(BAR(C::B_HF), 2);
+    mbar_init(BAR(C::B_HF), 4);
     mbar_init(BAR(C::B_AH), kApproxWarps);
     misc[1] = 0;
     mbar_init_fence();
@@ -586,23 +586,6 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       fence_proxy_async_smem();
       warp_arrive(BAR(C::B_CVF + s));
     }
-    if (hybrid && __all_sync(0xffffffffu, wait_bounded(BAR(C::B_XD), 0, abort_flag))) {
-      // Hbar fp32 [D][D] (row a = key dim, column c = value dim) -> bf16 MN-major
-      // operand in ring stage 0, laid out as a TMA 128-byte-swizzled load of 64-column
-      // panels would place it
-      const float* gh = p.hbar + size_t(bh) * D * D;
-      uint8_t* dh = base + C::OFF_RING;
-      for (int q = ct; q < D * (D / 8); q += 64) {
-        const int r = q / (D / 8), c16 = q % (D / 8);
-        const float4 h0 = __ldg(reinterpret_cast<const float4*>(gh + r * D + c16 * 8));
-        const float4 h1 = __ldg(reinterpret_cast<const float4*>(gh + r * D + c16 * 8 + 4));
-        const uint4 hv = make_uint4(pack_bf16x2(h0.x, h0.y), pack_bf16x2(h0.z, h0.w), pack_bf16x2(h1.x, h1.y),
-                                    pack_bf16x2(h1.z, h1.w));
-        *reinterpret_cast<uint4*>(dh + (c16 >> 3) * (D * 128) + r * 128 + (((c16 & 7) ^ (r & 7)) << 4)) = hv;
-      }
-      fence_proxy_async_smem();
-      warp_arrive(BAR(C::B_HF));
-    }
   } else {
     // ----------------------------------------------------------- row threads
     // Two threads per query row: half 0 (warps 4-7) and half 1 (warps 8-11) of a lane
@@ -738,6 +721,40 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       ok = pair_sync_and(pair_id, ok);
       if (hf == 1) {
         l = 0.f;
+        if (ok && hybrid) {
+          // Hbar fp32 [D][D] (row a = key dim, column c = value dim) -> bf16 MN-major
+          // operand in ring stage 0 (idle once the exact stage is done), laid out as a
+          // TMA 128-byte-swizzled load of 64-column panels would place it. Loads are
+          // issued in batches of four 16-byte output chunks per thread.
+          ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_XD), 0, abort_flag));
+          if (ok) {
+            const float* gh = p.hbar + size_t(bh) * D * D;
+            uint8_t* dh = base + C::OFF_RING;
+            constexpr int ITEMS = D * (D / 8) / 128, BATCH = 4;
+            static_assert(ITEMS % BATCH == 0, "Hbar conversion batches");
+#pragma unroll 1
+            for (int b0 = 0; b0 < ITEMS; b0 += BATCH) {
+              float4 f[BATCH][2];
+#pragma unroll
+              for (int i = 0; i < BATCH; ++i) {
+                const int q = r + (b0 + i) * 128;
+                const int row = q / (D / 8), c16 = q % (D / 8);
+                f[i][0] = __ldg(reinterpret_cast<const float4*>(gh + row * D + c16 * 8));
+                f[i][1] = __ldg(reinterpret_cast<const float4*>(gh + row * D + c16 * 8 + 4));
+              }
+#pragma unroll
+              for (int i = 0; i < BATCH; ++i) {
+                const int q = r + (b0 + i) * 128;
+                const int row = q / (D / 8), c16 = q % (D / 8);
+                *reinterpret_cast<uint4*>(dh + (c16 >> 3) * (D * 128) + row * 128 + (((c16 & 7) ^ (row & 7)) << 4)) =
+                    make_uint4(pack_bf16x2(f[i][0].x, f[i][0].y), pack_bf16x2(f[i][0].z, f[i][0].w),
+                               pack_bf16x2(f[i][1].x, f[i][1].y), pack_bf16x2(f[i][1].z, f[i][1].w));
+              }
+            }
+            fence_proxy_async_smem();
+            warp_arrive(BAR(C::B_HF));
+          }
+        }
       } else if (ok) {
         l += xs[128 + r];
         ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_OSYNC), 0, abort_flag));
