@@ -138,6 +138,37 @@ def _full_idx(B, H, nB, k=None):
     return np.broadcast_to(np.arange(k, dtype=np.int32), (B, H, nB, k)).copy()
 
 
+def pin_dense_textbook(orc, seed=21):
+    """oracle.dense_attention against scipy's softmax, scalar loops on a tiny case, and
+    large logit offsets (a per-row shift of the logits cannot change a softmax)."""
+    r = _rng(seed)
+    B, H, N, M, d = 1, 2, 9, 13, 5
+    Q = r.standard_normal((B, H, N, d))
+    K = r.standard_normal((B, H, M, d))
+    V = r.standard_normal((B, H, M, d))
+    scale = 0.7
+    err = float(np.abs(orc.dense_attention(Q, K, V, scale) - _textbook(Q, K, V, scale)).max())
+    # one row written out with scalar loops
+    out = orc.dense_attention(Q, K, V, scale)
+    for h in range(H):
+        for t in (0, N - 1):
+            z = [scale * sum(Q[0, h, t, a] * K[0, h, n, a] for a in range(d)) for n in range(M)]
+            w = [math.exp(v - max(z)) for v in z]
+            for c in range(d):
+                ref = sum(w[n] * V[0, h, n, c] for n in range(M)) / sum(w)
+                err = max(err, abs(out[0, h, t, c] - ref))
+    # logits near 700 overflow exp() unless the row maximum is taken out first; the
+    # rows get different offsets (q_t -> q_t + s_t u with u . k_n = const over n)
+    u = np.zeros(d)
+    u[0] = 1.0
+    K2 = K.copy()
+    K2[..., 0] = 50.0
+    Q2 = Q + (np.arange(N) * 2.0 + 14.0)[None, None, :, None] * u
+    err = max(err, float(np.abs(orc.dense_attention(Q2, K2, V, 1.0)
+                                - _textbook(Q2 - Q2[..., :1] * u, K2, V, 1.0)).max()))
+    return err
+
+
 def pin_all_selected_is_dense(orc, seed=5):
     r = _rng(seed)
     B, H, N, d, b = 1, 2, 45, 8, 8           # ragged last block

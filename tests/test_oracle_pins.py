@@ -29,6 +29,7 @@ def _pins(orc):
         ("stats_constant_values", P.pin_stats_constant_values, lambda e: e < TOL),
         ("select_bruteforce", P.pin_select_bruteforce, lambda e: e == 0),
         ("select_ties", P.pin_select_ties, lambda e: e == 0),
+        ("dense_textbook", P.pin_dense_textbook, lambda e: e < TOL),
         ("all_selected_is_dense", P.pin_all_selected_is_dense, lambda e: e < TOL),
         ("block_one_is_exact", P.pin_block_one_is_exact, lambda e: e < TOL),
         ("identical_keys_exact", P.pin_identical_keys_exact, lambda e: e < TOL),
@@ -64,7 +65,7 @@ def real_pins():
 
 @pytest.mark.parametrize("name", [
     "stats_bruteforce", "stats_covariance", "stats_constant_values", "select_bruteforce",
-    "select_ties", "all_selected_is_dense", "block_one_is_exact", "identical_keys_exact",
+    "select_ties", "dense_textbook", "all_selected_is_dense", "block_one_is_exact", "identical_keys_exact",
     "order0_pseudo_tokens", "first_order_key_form", "linear_in_values",
     "permutation_in_block", "order0_convex", "worked_example",
     "convergence_order0", "convergence_order1", "drop_is_masked_softmax", "hybrid_bruteforce",
@@ -109,6 +110,12 @@ MUTATIONS = {
     "routing weight sign flipped": ("scores + lam * np.asarray(route", "scores - lam * np.asarray(route"),
     "routing bias on the query axis": ("dtype=np.float64)[:, :, None, :]", "dtype=np.float64)[:, :, :, None]"),
     "bf16 rounding truncates": ("r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16", "r = (u >> 16) << 16"),
+    "dense scale missing": ("z = scale * np.matmul(Q, np.swapaxes(K, -1, -2))",
+                            "z = np.matmul(Q, np.swapaxes(K, -1, -2))"),
+    "dense max over the query axis": ("z = z - z.max(axis=-1, keepdims=True)",
+                                      "z = z - z.max(axis=-2, keepdims=True)"),
+    "dense normaliser over queries": ("np.matmul(p, V) / p.sum(axis=-1, keepdims=True)",
+                                      "np.matmul(p, V) / p.sum(axis=-2, keepdims=True)[..., :1]"),
     "bf16 ties away from even": ("r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16",
                                  "r = ((u + 0x8000) >> 16) << 16"),
 }
