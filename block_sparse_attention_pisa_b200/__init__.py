@@ -106,6 +106,53 @@ def _shape(x, block: int) -> Shape:
     return Shape(B, H, N, d, block)
 
 
+def _require(t, name: str, shape, dtype, device=None):
+    """Raise ValueError unless ``t`` is a contiguous tensor of exactly ``shape`` and
+    ``dtype`` (and, when ``device`` is given, on that CUDA device). Shapes and dtypes
+    are checked first, so a wrong buffer is named before any device question."""
+    import torch
+    if t is None:
+        raise ValueError(f"{name} is required here")
+    if not isinstance(t, torch.Tensor):
+        raise ValueError(f"{name} must be a torch tensor")
+    if tuple(t.shape) != tuple(int(x) for x in shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(int(x) for x in shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def _device_of(t):
+    """The CUDA device of the operands (``t`` must live on one)."""
+    if not t.is_cuda:
+        raise ValueError("the operands must be CUDA tensors")
+    return t.device
+
+
+def _stat_shapes(s: Shape, order: int):
+    """(kbar / S0 shape, first-order statistic shape or None) for one order."""
+    nB = num_blocks(s.N, s.block)
+    kb = (s.B, s.H, nB, s.d)
+    if order == ORDER_FIRST:
+        return kb, (s.B, s.H, nB, s.d, s.d)
+    if order == ORDER_HYBRID:
+        return kb, (s.B, s.H, s.d, s.d)
+    return kb, None
+
+
+def _first_order_dtype(order: int):
+    import torch
+    return torch.bfloat16 if order == ORDER_FIRST else torch.float32
+
+
+def _check_order(order: int):
+    if order not in (ORDER_DROP, ORDER_ZERO, ORDER_FIRST, ORDER_HYBRID):
+        raise ValueError(f"order={order} (must be -1, 0, 1 or 2)")
+
+
 def block_stats(K, V, block: int, order: int = 1, out=None):
     """kbar (fp32), S0 (fp32) and the first-order statistic of every key/value block:
     per-block S1 (bf16 [B, H, nB, d, d]) at order 1, the head's Hbar (fp32
@@ -113,18 +160,29 @@ def block_stats(K, V, block: int, order: int = 1, out=None):
     ``out`` = (kbar, S0, S1) preallocated outputs (optional)."""
     import torch
     s = _shape(K, block)
+    _check_order(order)
     nB = num_blocks(s.N, block)
+    kb_shape, s1_shape = _stat_shapes(s, order)
+    _require(K, "K", K.shape, torch.bfloat16)
+    _require(V, "V", K.shape, torch.bfloat16)
+    outs = []
     if out is not None:
         kbar, S0, S1 = out
-    else:
-        kbar = torch.empty((s.B, s.H, nB, s.d), device=K.device, dtype=torch.float32)
-        S0 = torch.empty_like(kbar)
-        if order == ORDER_FIRST:
-            S1 = torch.empty((s.B, s.H, nB, s.d, s.d), device=K.device, dtype=torch.bfloat16)
-        elif order == ORDER_HYBRID:
-            S1 = torch.empty((s.B, s.H, s.d, s.d), device=K.device, dtype=torch.float32)
+        outs = [(kbar, "kbar", kb_shape, torch.float32), (S0, "S0", kb_shape, torch.float32)]
+        if s1_shape is not None:
+            outs.append((S1, "S1", s1_shape, _first_order_dtype(order)))
         else:
             S1 = None
+        for t, name, shp, dt in outs:
+            _require(t, name, shp, dt)
+    dev = _device_of(K)
+    for t, name in [(V, "V")] + [(x, n) for x, n, _, _ in outs]:
+        if t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, expected {dev}")
+    if out is None:
+        kbar = torch.empty((s.B, s.H, nB, s.d), device=K.device, dtype=torch.float32)
+        S0 = torch.empty_like(kbar)
+        S1 = torch.empty(s1_shape, device=K.device, dtype=_first_order_dtype(order)) if s1_shape else None
     _check(lib().pisa_block_stats(_ptr(K), _ptr(V), s, order, _ptr(kbar), _ptr(S0), _ptr(S1),
                                   _stream(K)))
     return kbar, S0, S1
@@ -137,6 +195,16 @@ def select(Q, kbar, block: int, topk: int, out=None, route=None, lam: float = 0.
     import torch
     s = _shape(Q, block)
     nB = num_blocks(s.N, block)
+    _require(Q, "Q", Q.shape, torch.bfloat16)
+    _require(kbar, "kbar", (s.B, s.H, nB, s.d), torch.float32)
+    if route is not None:
+        _require(route, "route", (s.B, s.H, nB), torch.float32)
+    if out is not None:
+        _require(out, "idx", (s.B, s.H, nB, topk), torch.int32)
+    dev = _device_of(Q)
+    for t, name in ((kbar, "kbar"), (route, "route"), (out, "idx")):
+        if t is not None and t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, expected {dev}")
     idx = (torch.empty((s.B, s.H, nB, topk), device=Q.device, dtype=torch.int32)
            if out is None else out)
     _check(lib().pisa_select(_ptr(Q), _ptr(kbar), _ptr(route), float(lam), s, topk, _ptr(idx),
@@ -148,14 +216,22 @@ def routing_norms(S1, block: int, N: int, out=None):
     """(Hbar fp32 [B, H, d, d], M fp32 [B, H, nB]) from per-block bf16 S1 [B, H, nB, d, d]:
     the mean first-order matrix and each block's Frobenius deviation from it."""
     import torch
+    if S1.dim() != 5 or S1.shape[-1] != S1.shape[-2]:
+        raise ValueError("S1 must be [B, H, nB, d, d]")
     B, H, nB, d, _ = S1.shape
-    if not S1.is_contiguous():
-        raise ValueError("S1 must be contiguous")
     if nB != num_blocks(N, block):
         raise ValueError("S1 block count does not match N and block")
+    _require(S1, "S1", S1.shape, torch.bfloat16)
     s = Shape(B, H, N, d, block)
     if out is not None:
         Hbar, M = out
+        _require(Hbar, "Hbar", (B, H, d, d), torch.float32)
+        _require(M, "M", (B, H, nB), torch.float32)
+    dev = _device_of(S1)
+    if out is not None:
+        for t, name in ((Hbar, "Hbar"), (M, "M")):
+            if t.device != dev:
+                raise ValueError(f"{name} is on {t.device}, expected {dev}")
     else:
         Hbar = torch.empty((B, H, d, d), device=S1.device, dtype=torch.float32)
         M = torch.empty((B, H, nB), device=S1.device, dtype=torch.float32)
@@ -166,8 +242,31 @@ def routing_norms(S1, block: int, N: int, out=None):
 def _attention(fn, Q, K, V, kbar, S0, S1, idx, block, order, scale, out=None):
     import torch
     s = _shape(Q, block)
-    O = torch.empty_like(Q) if out is None else out
+    _check_order(order)
+    nB = num_blocks(s.N, block)
+    if idx is None or idx.dim() != 4:
+        raise ValueError("idx must be an int32 [B, H, nB, topk] tensor")
     topk = int(idx.shape[-1])
+    kb_shape, s1_shape = _stat_shapes(s, order)
+    checks = [(Q, "Q", Q.shape, torch.bfloat16), (K, "K", Q.shape, torch.bfloat16),
+              (V, "V", Q.shape, torch.bfloat16), (idx, "idx", (s.B, s.H, nB, topk), torch.int32)]
+    if out is not None:
+        checks.append((out, "O", Q.shape, torch.bfloat16))
+    if order != ORDER_DROP:
+        checks += [(kbar, "kbar", kb_shape, torch.float32), (S0, "S0", kb_shape, torch.float32)]
+    if s1_shape is not None:
+        checks.append((S1, "S1" if order == ORDER_FIRST else "Hbar (S1)", s1_shape, _first_order_dtype(order)))
+    for t, name, shp, dt in checks:
+        _require(t, name, shp, dt)
+    dev = _device_of(Q)
+    for t, name, _, _ in checks:
+        if t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, expected {dev}")
+    if order == ORDER_DROP:
+        kbar = S0 = S1 = None
+    elif s1_shape is None:
+        S1 = None
+    O = torch.empty_like(Q) if out is None else out
     _check(fn(_ptr(Q), _ptr(K), _ptr(V), _ptr(kbar), _ptr(S0), _ptr(S1), _ptr(idx), s, topk,
               order, float(scale), _ptr(O), _stream(Q)))
     return O
