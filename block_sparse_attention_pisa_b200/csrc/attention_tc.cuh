@@ -812,9 +812,13 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             const float x1 = ex2(__uint_as_float(sv[k + 1]) - m);
             const float n0 = (c * C::CHUNK + k == nB - 1) ? float(nlast) : float(BLK);
             const float n1 = (c * C::CHUNK + k + 1 == nB - 1) ? float(nlast) : float(BLK);
-            lsp[(k >> 1) & 3] = fmaf(n1, x1, fmaf(n0, x0, lsp[(k >> 1) & 3]));
-            if (hybrid) ssp[(k >> 1) & 1] += x0 + x1;
-            a0[k >> 1] = pack_bf16x2_int(x0, x1);
+            // the denominator (and the hybrid weight sum) take the bf16-rounded alpha that
+            // the numerator's MMAs multiply, so both sides weigh each block alike
+            const uint32_t w = pack_bf16x2_int(x0, x1);
+            const float r0 = bf16_lo(w), r1 = bf16_hi(w);
+            lsp[(k >> 1) & 3] = fmaf(n1, r1, fmaf(n0, r0, lsp[(k >> 1) & 3]));
+            if (hybrid) ssp[(k >> 1) & 1] += r0 + r1;
+            a0[k >> 1] = w;
           }
           l += (lsp[0] + lsp[1]) + (lsp[2] + lsp[3]);
           s_alpha += ssp[0] + ssp[1];

@@ -9,9 +9,14 @@ namespace pisa {
 
 using bf16 = __nv_bfloat16;
 
-// Device error word (one per device context): bit 0 = a bounded wait ran out,
-// bit 1 = an idx entry was out of range. Read and cleared by pisa_device_error().
+// Device error word (one per device, shared by every stream and caller): bit 0 = a
+// bounded wait ran out, bit 1 = an idx entry was out of range. pisa_device_error()
+// takes it with one atomic exchange (take_error_kernel), so a bit raised between two
+// readers is reported by the second and never lost.
 __device__ unsigned int g_pisa_error;
+__device__ unsigned int g_pisa_error_taken;  // the word as take_error_kernel found it
+
+__global__ void take_error_kernel() { g_pisa_error_taken = atomicExch(&g_pisa_error, 0u); }
 
 constexpr unsigned kErrTimeout = 1u;
 constexpr unsigned kErrBadIndex = 2u;

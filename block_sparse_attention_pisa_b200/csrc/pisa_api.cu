@@ -395,11 +395,17 @@ pisa_status_t pisa_attention_simt(const void* Q, const void* K, const void* V, c
 }
 
 pisa_status_t pisa_device_error(void* stream) {
-  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return fail(PISA_ERR_CUDA, "cudaStreamSynchronize: %s", cudaGetErrorString(e));
-  unsigned word = 0, zero = 0;
-  if ((e = cudaMemcpyFromSymbol(&word, pisa::g_pisa_error, sizeof(word))) != cudaSuccess ||
-      (e = cudaMemcpyToSymbol(pisa::g_pisa_error, &zero, sizeof(zero))) != cudaSuccess)
+  auto st = static_cast<cudaStream_t>(stream);
+  // one caller at a time: the exchanged word passes through one device variable
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  pisa::take_error_kernel<<<1, 1, 0, st>>>();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(PISA_ERR_CUDA, "take_error_kernel launch: %s", cudaGetErrorString(e));
+  unsigned word = 0;
+  if ((e = cudaMemcpyFromSymbolAsync(&word, pisa::g_pisa_error_taken, sizeof(word), 0, cudaMemcpyDeviceToHost, st)) !=
+          cudaSuccess ||
+      (e = cudaStreamSynchronize(st)) != cudaSuccess)
     return fail(PISA_ERR_CUDA, "device error word: %s", cudaGetErrorString(e));
   if (word & pisa::kErrTimeout) return fail(PISA_ERR_TIMEOUT, "a bounded device wait ran out (word=0x%x)", word);
   if (word & pisa::kErrBadIndex) return fail(PISA_ERR_INVALID_ARG, "idx held an out-of-range block (word=0x%x)", word);

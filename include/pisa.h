@@ -32,7 +32,7 @@
  *    a wait that runs out (or an out-of-range entry in `idx`) sets a device error word
  *    that pisa_device_error() reports as PISA_ERR_TIMEOUT / PISA_ERR_INVALID_ARG.
  *  - The calls are thread-safe with respect to one another; pisa_last_error() is per
- *    host thread.
+ *    host thread. The device error word is shared per device (see pisa_device_error).
  *
  * Orders (how the non-critical blocks U_i of a query block enter the softmax)
  * -------------------------------------------------------------------------
@@ -171,9 +171,16 @@ pisa_status_t pisa_attention_simt(const void* Q, const void* K, const void* V, c
                                   void* O, void* stream);
 
 /*
- * pisa_device_error -- synchronises `stream`, then reads and clears the device error
- * word that the kernels set. Returns PISA_OK, PISA_ERR_TIMEOUT (a bounded wait ran
- * out), PISA_ERR_INVALID_ARG (an idx entry was out of range) or PISA_ERR_CUDA.
+ * pisa_device_error -- takes the device error word that the kernels set, after all
+ * work already enqueued on `stream`, and synchronises `stream`. Returns PISA_OK,
+ * PISA_ERR_TIMEOUT (a bounded wait ran out), PISA_ERR_INVALID_ARG (an idx entry was out
+ * of range) or PISA_ERR_CUDA.
+ * The word is ONE PER DEVICE, shared by every stream and host thread that uses the
+ * library on the current device: a bit raised by a kernel on any stream is reported by
+ * the first pisa_device_error() that takes the word after the bit was raised, whatever
+ * stream that call names, and is cleared by it. The take is one atomic exchange on the
+ * device (read and clear cannot interleave with a kernel's raise), so no bit is lost; a
+ * caller that needs per-launch attribution serialises its launches with this call.
  */
 pisa_status_t pisa_device_error(void* stream);
 

@@ -37,11 +37,33 @@ def assert_close(out, ref, what=""):
     return mx, rel
 
 
-def compare_idx(gpu_idx: np.ndarray, ref_idx: np.ndarray, near: np.ndarray):
+# (label, rows, oracle near-tie rows, GPU rows differing, of which at near-ties), one
+# entry per index comparison of the session; printed by the terminal summary hook
+NEAR_TIE_LOG = []
+
+
+def compare_idx(gpu_idx: np.ndarray, ref_idx: np.ndarray, near: np.ndarray, label: str = ""):
     """Rows must match exactly unless the oracle recorded a near-tie there.
-    Returns (mismatched rows, of which near-ties)."""
+    Returns (mismatched rows, of which near-ties, the mismatch mask) and records the
+    counts for the session's near-tie report."""
     bad = np.any(gpu_idx != ref_idx, axis=-1)
+    NEAR_TIE_LOG.append((label, int(bad.size), int(near.sum()), int(bad.sum()), int((bad & near).sum())))
     return int(bad.sum()), int((bad & near).sum()), bad
+
+
+def sampled_query_blocks(wl, count: int = 32, seed: int = 0):
+    """Query blocks for a sampled oracle check of a large launch: the first and last
+    blocks, and blocks spread over the sequence. At b = 64 both query blocks of each
+    chosen 128-row tile are taken (the fused kernel computes two query blocks per tile)."""
+    rng = np.random.default_rng(seed)
+    def spread(n, k):        # 0, n - 1 and k - 2 others
+        inner = rng.choice(np.arange(1, n - 1), size=max(0, min(n - 2, k - 2)), replace=False) if n > 2 else []
+        return sorted({0, n - 1} | set(int(x) for x in inner))
+    if wl.block == 64:
+        qbs = [q for t in spread(-(-wl.nB // 2), count // 2) for q in (2 * t, 2 * t + 1) if q < wl.nB]
+    else:
+        qbs = spread(wl.nB, count)
+    return qbs
 
 
 def oracle_stats(Kf, Vf, wl: W.Workload):

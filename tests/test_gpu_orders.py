@@ -54,7 +54,8 @@ def test_small_pipeline(wl, order, fn):
     np.testing.assert_allclose(kbar.cpu().numpy(), ref["kbar"], rtol=1e-5, atol=1e-5)
     PT.check_first_order_stat(S1, ref["S1"], order)
     idx = P.select(dq, kbar, wl.block, wl.topk)
-    bad, near_bad, _ = PT.compare_idx(idx.cpu().numpy(), ref["idx"], ref["near"])
+    bad, near_bad, _ = PT.compare_idx(idx.cpu().numpy(), ref["idx"], ref["near"],
+                                      f"order {order} N{wl.N} d{wl.d} b{wl.block} ({fn})")
     assert bad == near_bad, f"{bad} index rows differ, {near_bad} of them at near-ties"
     oidx = torch.from_numpy(ref["idx"]).cuda()
     run = P.attention if fn == "fused" else P.attention_simt
@@ -95,7 +96,7 @@ def test_image_workload(order):
     ref = PT.oracle_pipeline(*host, wl)
     PT.check_first_order_stat(S1, ref["S1"], order)
     idx = P.select(dq, kbar, wl.block, wl.topk)
-    bad, near_bad, bad_rows = PT.compare_idx(idx.cpu().numpy(), ref["idx"], ref["near"])
+    bad, near_bad, bad_rows = PT.compare_idx(idx.cpu().numpy(), ref["idx"], ref["near"], f"image order {order}")
     assert bad == near_bad
     O = P.attention(dq, dk, dv, kbar, S0, S1, idx, wl.block, order, wl.scale)
     out = PT.bf16_to_f64(O)
@@ -105,7 +106,8 @@ def test_image_workload(order):
 
 @pytest.mark.parametrize("name", ["video_hybrid", "video_drop", "long_hybrid"])
 def test_large_workload_sampled(name):
-    """Full-size launch; the oracle checks three heads on sampled query blocks."""
+    """Full-size launch; the oracle checks three heads on 32 sampled query blocks each
+    (at b = 64 both query blocks of 16 of the 128-row tiles, first and last included)."""
     wl = W.get(name)
     q, k, v = W.make_inputs(wl)
     dq, dk, dv = (PT.to_device(a) for a in (q, k, v))
@@ -114,14 +116,14 @@ def test_large_workload_sampled(name):
     O = P.attention(dq, dk, dv, kbar, S0, S1, idx, wl.block, wl.order, wl.scale)
     torch.cuda.synchronize()
     heads = [0, wl.H // 2, wl.H - 1]
-    qbs = sorted({0, 1, wl.nB // 3, wl.nB // 2, wl.nB - 2, wl.nB - 1})
+    qbs = PT.sampled_query_blocks(wl, 32)
     Qf, Kf, Vf = (PT.to_f64(a[:, heads]) for a in (q, k, v))
     rk, r0, r1 = PT.oracle_stats(Kf, Vf, wl)
     np.testing.assert_allclose(kbar[:, heads].cpu().numpy(), rk, rtol=1e-5, atol=1e-5)
     if wl.order == 2:
         PT.check_first_order_stat(S1[:, heads], r1, 2)
     ridx, near, _ = oracle.select(Qf, rk, wl.block, wl.topk)
-    bad, near_bad, bad_rows = PT.compare_idx(idx[:, heads].cpu().numpy(), ridx, near)
+    bad, near_bad, bad_rows = PT.compare_idx(idx[:, heads].cpu().numpy(), ridx, near, f"{name} (3 heads)")
     assert bad == near_bad, f"{bad} index rows differ, {near_bad} at near-ties"
     ref = oracle.attention(Qf, Kf, Vf, rk, r0, r1, ridx, wl.block, wl.order, wl.scale,
                            query_blocks=qbs)

@@ -61,6 +61,8 @@ SMALL = [
     W.get("tiny").with_(d=128, block=128, N=1000, H=3, topk=2, scale=0.09),
     W.get("tiny").with_(N=512, topk=8),                       # all selected: dense attention
     W.get("tiny").with_(N=512, topk=1, H=2, B=2),
+    W.get("tiny").with_(d=128, N=330, block=64, topk=2, order=0),   # order 0 at d = 128, b = 64
+    W.get("tiny").with_(d=128, N=4096, block=64, topk=5, H=2, order=0),  # two approximate chunks
 ]
 
 
@@ -72,7 +74,8 @@ def test_small_pipeline(wl, fn):
     kbar, S0, S1 = _check_stats(wl, dev, host)
     ref = PT.oracle_pipeline(*host, wl)
     idx = P.select(dq, kbar, wl.block, wl.topk)
-    bad, near_bad, _ = PT.compare_idx(idx.cpu().numpy(), ref["idx"], ref["near"])
+    bad, near_bad, _ = PT.compare_idx(idx.cpu().numpy(), ref["idx"], ref["near"],
+                                      f"small N{wl.N} d{wl.d} b{wl.block} k{wl.topk} ({fn})")
     assert bad == near_bad, f"{bad} index rows differ, {near_bad} of them at near-ties"
     # the attention is checked on the oracle's own selection
     oidx = torch.from_numpy(ref["idx"]).cuda()
@@ -125,7 +128,7 @@ def test_full_workload(name):
     kbar, S0, S1 = _check_stats(wl, dev, host)
     ref = PT.oracle_pipeline(*host, wl)
     idx = P.select(dq, kbar, wl.block, wl.topk)
-    bad, near_bad, bad_rows = PT.compare_idx(idx.cpu().numpy(), ref["idx"], ref["near"])
+    bad, near_bad, bad_rows = PT.compare_idx(idx.cpu().numpy(), ref["idx"], ref["near"], name)
     assert bad == near_bad, f"{bad} index rows differ, {near_bad} at near-ties"
     O = P.attention(dq, dk, dv, kbar, S0, S1, idx, wl.block, wl.order, wl.scale)
     out = PT.bf16_to_f64(O)
@@ -139,7 +142,8 @@ def test_full_workload(name):
 
 @pytest.mark.parametrize("name", ["video", "long"])
 def test_large_workload_sampled(name):
-    """Full-size launch; the oracle checks three heads on sampled query blocks."""
+    """Full-size launch; the oracle checks three heads on 32 sampled query blocks each
+    (at b = 64 both query blocks of 16 of the 128-row tiles, first and last included)."""
     wl = W.get(name)
     q, k, v = W.make_inputs(wl)
     dq, dk, dv = (PT.to_device(a) for a in (q, k, v))
@@ -148,7 +152,7 @@ def test_large_workload_sampled(name):
     O = P.attention(dq, dk, dv, kbar, S0, S1, idx, wl.block, wl.order, wl.scale)
     torch.cuda.synchronize()
     heads = [0, wl.H // 2, wl.H - 1]
-    qbs = sorted({0, 1, wl.nB // 3, wl.nB // 2, wl.nB - 2, wl.nB - 1})
+    qbs = PT.sampled_query_blocks(wl, 32)
     sub = wl.with_(H=len(heads))
     Qf, Kf, Vf = (PT.to_f64(a[:, heads]) for a in (q, k, v))
     rk, r0, r1 = oracle.block_stats(Kf, Vf, wl.block, wl.order)
@@ -158,7 +162,7 @@ def test_large_workload_sampled(name):
     assert np.all(np.abs(g1 - r1) <= 2.0 ** -8 * np.abs(r1) + 1e-3)
     ridx, near, _ = oracle.select(Qf, rk, wl.block, wl.topk)
     gidx = idx[:, heads].cpu().numpy()
-    bad, near_bad, bad_rows = PT.compare_idx(gidx, ridx, near)
+    bad, near_bad, bad_rows = PT.compare_idx(gidx, ridx, near, f"{name} (3 heads)")
     assert bad == near_bad, f"{bad} index rows differ, {near_bad} at near-ties"
     ref = oracle.attention(Qf, Kf, Vf, rk, r0, r1, ridx, wl.block, wl.order, wl.scale,
                            query_blocks=qbs)
@@ -191,6 +195,23 @@ def test_out_of_range_index_is_flagged_not_faulted():
         run(dq, dk, dv, kbar, S0, S1, idx, wl.block, wl.order, wl.scale)
         with pytest.raises(P.PisaError, match="INVALID_ARG"):
             P.device_error()
+
+
+def test_device_error_word_is_shared_per_device():
+    """A bit raised by a kernel on one stream is reported by a device_error call on another
+    stream (the word is one per device), and that call clears it."""
+    wl = W.get("tiny")
+    (dq, dk, dv), _ = _inputs(wl)
+    kbar, S0, S1 = P.block_stats(dk, dv, wl.block, wl.order)
+    idx = P.select(dq, kbar, wl.block, wl.topk)
+    idx[0, 0, 2, 1] = -3
+    P.attention(dq, dk, dv, kbar, S0, S1, idx, wl.block, wl.order, wl.scale)
+    torch.cuda.synchronize()
+    other = torch.cuda.Stream()
+    with torch.cuda.stream(other):
+        with pytest.raises(P.PisaError, match="INVALID_ARG"):
+            P.device_error()
+    P.device_error()          # taken by the first reader: nothing left
 
 
 def test_host_entry_point_matches_device():

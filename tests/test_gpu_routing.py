@@ -70,7 +70,7 @@ def test_routed_hybrid_pipeline(wl):
     ref_M, ref_H = _check_routing(Hbar, M, r1, S1)
     idx = P.select(dq, kbar, wl.block, wl.topk, route=M, lam=LAM)
     ridx, near, _ = oracle.select(Qf, rk, wl.block, wl.topk, route=ref_M, lam=LAM)
-    bad, near_bad, _ = PT.compare_idx(idx.cpu().numpy(), ridx, near)
+    bad, near_bad, _ = PT.compare_idx(idx.cpu().numpy(), ridx, near, f"routed N{wl.N} d{wl.d} b{wl.block}")
     assert bad == near_bad, f"{bad} index rows differ, {near_bad} of them at near-ties"
     O = P.attention(dq, dk, dv, kbar, S0, Hbar, torch.from_numpy(ridx).cuda(), wl.block, 2, wl.scale)
     ref = oracle.attention(Qf, Kf, Vf, rk, r0, ref_H, ridx, wl.block, 2, wl.scale)
@@ -108,5 +108,5 @@ def test_routing_full_size(name):
     sub = lambda t: t[bi:bi + 1, heads]  # noqa: E731
     ref_M, ref_H = _check_routing(sub(Hbar), sub(M), r1, sub(S1))
     ridx, near, _ = oracle.select(Qf, rk, wl.block, wl.topk, route=ref_M, lam=lam)
-    bad, near_bad, _ = PT.compare_idx(sub(idx).cpu().numpy(), ridx, near)
+    bad, near_bad, _ = PT.compare_idx(sub(idx).cpu().numpy(), ridx, near, f"{name} routed (2 heads)")
     assert bad == near_bad, f"{bad} index rows differ, {near_bad} at near-ties"
