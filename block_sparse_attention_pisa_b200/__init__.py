@@ -21,7 +21,7 @@ ORDER_DROP, ORDER_ZERO, ORDER_FIRST, ORDER_HYBRID = -1, 0, 1, 2
 
 __all__ = [
     "ORDER_DROP", "ORDER_ZERO", "ORDER_FIRST", "ORDER_HYBRID", "PisaError", "Shape", "lib", "block_stats", "select", "attention", "attention_simt",
-    "pisa", "pisa_host", "head_chunks", "device_error", "num_blocks", "LIB_PATH", "SYMBOLS", "routing_norms",
+    "pisa", "pisa_host", "host_workspace_bytes", "head_chunks", "device_error", "num_blocks", "LIB_PATH", "SYMBOLS", "routing_norms",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpisa.so")
@@ -30,6 +30,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpisa.so"
 SYMBOLS = (
     "pisa_block_stats", "pisa_select", "pisa_routing_norms", "pisa_attention", "pisa_attention_simt",
     "pisa_device_error", "pisa_status_string", "pisa_last_error", "pisa_version",
+    "pisa_run_host_workspace", "pisa_run_host",
 )
 
 STATUS = {0: "PISA_OK", 1: "PISA_ERR_INVALID_ARG", 2: "PISA_ERR_UNSUPPORTED",
@@ -66,6 +67,8 @@ def lib():
     attn = [vp, vp, vp, vp, vp, vp, vp, Shape, i32, i32, f32, vp, vp]
     L.pisa_attention.argtypes = attn
     L.pisa_attention_simt.argtypes = attn
+    L.pisa_run_host_workspace.argtypes = [Shape, i32, i32, f32, i32, ctypes.POINTER(ctypes.c_size_t)]
+    L.pisa_run_host.argtypes = [vp, vp, vp, Shape, i32, i32, f32, f32, i32, vp, ctypes.c_size_t, vp, vp]
     L.pisa_device_error.argtypes = [vp]
     L.pisa_status_string.argtypes = [ctypes.c_int]
     L.pisa_status_string.restype = ctypes.c_char_p
@@ -73,7 +76,7 @@ def lib():
     L.pisa_last_error.restype = ctypes.c_char_p
     L.pisa_version.argtypes = []
     for name in ("pisa_block_stats", "pisa_select", "pisa_routing_norms", "pisa_attention", "pisa_attention_simt",
-                 "pisa_device_error", "pisa_version"):
+                 "pisa_device_error", "pisa_version", "pisa_run_host_workspace", "pisa_run_host"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -309,54 +312,44 @@ def head_chunks(BH: int, chunks: int):
     return [(edges[c], edges[c + 1]) for c in range(chunks) if edges[c + 1] > edges[c]]
 
 
-def pisa_host(Q, K, V, block: int, topk: int, order: int = 1, scale: float | None = None,
-              device="cuda", route_lambda: float = 0.0, chunks: int = 8):
-    """The whole path on HOST tensors [B, H, N, d]: copies Q, K, V to the device, runs it,
-    and copies the output back. Returns O on the host.
+def host_workspace_bytes(shape: Shape, topk: int, order: int, route_lambda: float = 0.0, chunks: int = 8) -> int:
+    """Device workspace (bytes) that ``pisa_host`` needs for this problem."""
+    n = ctypes.c_size_t(0)
+    _check(lib().pisa_run_host_workspace(shape, int(topk), int(order), float(route_lambda), int(chunks),
+                                         ctypes.byref(n)))
+    return int(n.value)
 
-    (batch, head) pairs are independent in every step, so the call is pipelined over
-    `chunks` ranges of them: the host-to-device copy of range c + 1 and the
-    device-to-host copy of range c - 1 run on their own streams while range c
-    computes. With pinned host tensors the copies are asynchronous and overlap the
-    kernels; the result is identical to running the whole batch at once."""
+
+def pisa_host(Q, K, V, block: int, topk: int, order: int = 1, scale: float | None = None,
+              device="cuda", route_lambda: float = 0.0, chunks: int = 8, out=None):
+    """The whole path on HOST tensors [B, H, N, d] through the C ABI's ``pisa_run_host``:
+    the library copies Q, K, V to the device, runs the path and copies O back, pipelined
+    over ``chunks`` ranges of (batch, head) pairs (copies of one range overlap the kernels
+    of another; the result equals the whole-batch device path bit for bit). Pinned host
+    tensors let the copies run asynchronously. Returns O on the host (``out`` if given).
+    The device workspace is allocated here with torch."""
     import torch
-    if Q.dim() != 4 or not (Q.is_contiguous() and K.is_contiguous() and V.is_contiguous()):
-        raise ValueError("expected contiguous [B, H, N, d] host tensors")
-    B, H, N, d = Q.shape
-    BH = B * H
+    if scale is None:
+        scale = Q.shape[-1] ** -0.5
+    s = _shape(Q, block)
+    for t, name in ((Q, "Q"), (K, "K"), (V, "V")):
+        _require(t, name, Q.shape, torch.bfloat16)
+        if t.is_cuda:
+            raise ValueError(f"{name} must be a host tensor (pisa_host copies it to the device)")
+    if out is None:
+        out = torch.empty(Q.shape, dtype=Q.dtype, pin_memory=Q.is_pinned())
+    _require(out, "O", Q.shape, torch.bfloat16)
+    if out.is_cuda:
+        raise ValueError("O must be a host tensor")
     dev = torch.device(device)
     if dev.index is None:
         dev = torch.device("cuda", torch.cuda.current_device())
-    flat = [t.view(BH, N, d) for t in (Q, K, V)]
-    dbuf = [torch.empty((BH, N, d), device=dev, dtype=t.dtype) for t in (Q, K, V)]
-    dO = torch.empty((BH, N, d), device=dev, dtype=Q.dtype)
-    out = torch.empty(Q.shape, dtype=Q.dtype, pin_memory=Q.is_pinned())
-    out_flat = out.view(BH, N, d)
-    compute = torch.cuda.current_stream(dev)
-    h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ranges = head_chunks(BH, chunks)
-    landed = [torch.cuda.Event() for _ in ranges]
-    done = [torch.cuda.Event() for _ in ranges]
-    h2d.wait_stream(compute)  # the device buffers are fresh allocations of this stream
-    with torch.cuda.stream(h2d):
-        for c, (a, b) in enumerate(ranges):
-            for src, dst in zip(flat, dbuf):
-                dst[a:b].copy_(src[a:b], non_blocking=True)
-            landed[c].record(h2d)
-    for c, (a, b) in enumerate(ranges):
-        compute.wait_event(landed[c])
-        q, k, v = (t[a:b].view(1, b - a, N, d) for t in dbuf)
-        with torch.cuda.stream(compute):
-            pisa(q, k, v, block, topk, order, scale, route_lambda, out=dO[a:b].view(1, b - a, N, d))
-        done[c].record(compute)
-        d2h.wait_event(done[c])
-        with torch.cuda.stream(d2h):
-            out_flat[a:b].copy_(dO[a:b], non_blocking=True)
-    compute.wait_stream(d2h)
-    for t in dbuf + [dO]:
-        t.record_stream(h2d)
-        t.record_stream(d2h)
-    compute.synchronize()
+    with torch.cuda.device(dev):
+        nbytes = host_workspace_bytes(s, topk, order, route_lambda, chunks)
+        ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+        stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+        _check(lib().pisa_run_host(_ptr(Q), _ptr(K), _ptr(V), s, int(topk), int(order), float(scale),
+                                   float(route_lambda), int(chunks), _ptr(ws), nbytes, _ptr(out), stream))
     return out
 
 

@@ -15,6 +15,7 @@
 #include "routing.cuh"
 #include "attention_simt.cuh"
 #include "attention_tc.cuh"
+#include "host_pipeline.cuh"
 
 using pisa::bf16;
 
@@ -392,6 +393,157 @@ pisa_status_t pisa_attention_simt(const void* Q, const void* K, const void* V, c
   auto o = static_cast<bf16*>(O);
   if (shape.d == 128) return launch_attention_simt<128>(shape, q, k, v, kbar, S0, s1, idx, topk, order, scale, o, st);
   return launch_attention_simt<64>(shape, q, k, v, kbar, S0, s1, idx, topk, order, scale, o, st);
+}
+
+pisa_status_t pisa_run_host_workspace(pisa_shape_t shape, int32_t topk, int32_t order, float route_lambda,
+                                       int32_t chunks, size_t* bytes) {
+  if (bytes == nullptr) return fail(PISA_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = 0;
+  bool empty = false;
+  PISA_TRY(check_shape(shape, &empty));
+  if (empty) return ok();
+  PISA_TRY(check_order(order));
+  PISA_TRY(check_topk(shape, topk));
+  if (chunks < 1) return fail(PISA_ERR_INVALID_ARG, "chunks=%d (must be >= 1)", chunks);
+  if (!std::isfinite(route_lambda) || route_lambda < 0.f)
+    return fail(PISA_ERR_INVALID_ARG, "route_lambda=%g (must be finite and >= 0)", double(route_lambda));
+  PISA_TRY(check_support(shape));
+  *bytes = pisa_host::workspace_bytes(shape, topk, order, route_lambda > 0.f, chunks);
+  return ok();
+}
+
+pisa_status_t pisa_run_host(const void* Q, const void* K, const void* V, pisa_shape_t shape, int32_t topk,
+                            int32_t order, float scale, float route_lambda, int32_t chunks, void* workspace,
+                            size_t workspace_bytes, void* O, void* stream) {
+  size_t need = 0;
+  PISA_TRY(pisa_run_host_workspace(shape, topk, order, route_lambda, chunks, &need));
+  if (need == 0) return ok();  // empty problem: nothing touched
+  const void* host[4] = {Q, K, V, O};
+  const char* names[4] = {"Q", "K", "V", "O"};
+  for (int i = 0; i < 4; ++i)
+    if (host[i] == nullptr) return fail(PISA_ERR_INVALID_ARG, "%s is NULL", names[i]);
+  if (!std::isfinite(scale) || !(scale > 0.f))
+    return fail(PISA_ERR_INVALID_ARG, "scale=%g (must be finite and > 0)", double(scale));
+  if (workspace == nullptr) return fail(PISA_ERR_INVALID_ARG, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(workspace) % pisa_host::kAlign)
+    return fail(PISA_ERR_INVALID_ARG, "workspace is not %zu-byte aligned", pisa_host::kAlign);
+  if (workspace_bytes < need)
+    return fail(PISA_ERR_INVALID_ARG, "workspace holds %zu bytes, %zu needed", workspace_bytes, need);
+  int sms = 0;
+  PISA_TRY(check_device(&sms));
+  for (int i = 0; i < 4; ++i) {
+    cudaPointerAttributes at{};
+    if (cudaPointerGetAttributes(&at, host[i]) == cudaSuccess && at.type == cudaMemoryTypeDevice)
+      return fail(PISA_ERR_INVALID_ARG, "%s is device memory; pisa_run_host takes host buffers", names[i]);
+    cudaGetLastError();  // an unregistered host pointer may leave an error behind
+  }
+
+  const int64_t BH = int64_t(shape.B) * shape.H;
+  const int nc = int(chunks < BH ? chunks : BH);
+  const int slots = nc < pisa_host::kSlots ? nc : pisa_host::kSlots;
+  const int64_t nB = num_blocks(shape);
+  const bool routed = route_lambda > 0.f;
+  const pisa_host::SlotLayout L =
+      pisa_host::slot_layout(pisa_host::range_size(BH, nc), shape.N, shape.d, nB, topk, order, routed);
+  const size_t row_bytes = size_t(shape.N) * shape.d * 2;  // one (batch, head) slice of Q, K, V or O
+  auto cs = static_cast<cudaStream_t>(stream);
+  cudaStream_t in_s = nullptr, out_s = nullptr;
+  std::vector<cudaEvent_t> ev;  // entry, then landed / computed / drained per range
+  pisa_status_t st = PISA_OK;
+  cudaError_t e = cudaSuccess;
+  auto cuda_fail = [&](const char* what) { return fail(PISA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e)); };
+  auto event = [&](cudaEvent_t* out) {
+    e = cudaEventCreateWithFlags(out, cudaEventDisableTiming);
+    if (e == cudaSuccess) ev.push_back(*out);
+    return e == cudaSuccess;
+  };
+  cudaEvent_t entry = nullptr;
+  std::vector<cudaEvent_t> landed(nc), computed(nc), drained(nc);
+  do {
+    if ((e = cudaStreamCreateWithFlags(&in_s, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaStreamCreateWithFlags(&out_s, cudaStreamNonBlocking)) != cudaSuccess) {
+      st = cuda_fail("cudaStreamCreateWithFlags");
+      break;
+    }
+    // the copy streams start after whatever the caller's stream already holds (earlier
+    // users of the workspace)
+    if (!event(&entry) || (e = cudaEventRecord(entry, cs)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(in_s, entry, 0)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(out_s, entry, 0)) != cudaSuccess) {
+      st = cuda_fail("entry event");
+      break;
+    }
+    for (int c = 0; c < nc && st == PISA_OK; ++c) {
+      const int64_t a = BH * c / nc, b = BH * (c + 1) / nc, n = b - a;
+      uint8_t* base = static_cast<uint8_t*>(workspace) + size_t(c % slots) * L.bytes;
+      if (!event(&landed[c]) || !event(&computed[c]) || !event(&drained[c])) {
+        st = cuda_fail("cudaEventCreate");
+        break;
+      }
+      // copy in, once the slot's previous range has been copied out
+      if (c >= slots && (e = cudaStreamWaitEvent(in_s, drained[c - slots], 0)) != cudaSuccess) {
+        st = cuda_fail("cudaStreamWaitEvent");
+        break;
+      }
+      const size_t off = size_t(a) * row_bytes, len = size_t(n) * row_bytes;
+      const size_t dst[3] = {L.q, L.k, L.v};
+      for (int t = 0; t < 3 && e == cudaSuccess; ++t)
+        e = cudaMemcpyAsync(base + dst[t], static_cast<const uint8_t*>(host[t]) + off, len, cudaMemcpyHostToDevice,
+                            in_s);
+      if (e != cudaSuccess || (e = cudaEventRecord(landed[c], in_s)) != cudaSuccess ||
+          (e = cudaStreamWaitEvent(cs, landed[c], 0)) != cudaSuccess) {
+        st = cuda_fail("copy-in");
+        break;
+      }
+      // the path on the caller's stream, for this range as a [1, n, N, d] problem
+      pisa_shape_t rs{1, int32_t(n), shape.N, shape.d, shape.block};
+      float* kbar = reinterpret_cast<float*>(base + L.kbar);
+      float* S0 = reinterpret_cast<float*>(base + L.s0);
+      void* S1 = base + L.s1;
+      int32_t* idx = reinterpret_cast<int32_t*>(base + L.idx);
+      const int stats_order = routed ? PISA_ORDER_FIRST : order;
+      const void* first = order == PISA_ORDER_FIRST || order == PISA_ORDER_HYBRID ? S1 : nullptr;
+      const float* route = nullptr;
+      if ((st = pisa_block_stats(base + L.k, base + L.v, rs, stats_order, kbar, S0,
+                                 stats_order >= PISA_ORDER_FIRST ? S1 : nullptr, cs)) != PISA_OK)
+        break;
+      if (routed) {
+        float* hbar = reinterpret_cast<float*>(base + L.hbar);
+        float* M = reinterpret_cast<float*>(base + L.m);
+        if ((st = pisa_routing_norms(S1, rs, hbar, M, cs)) != PISA_OK) break;
+        route = M;
+        if (order == PISA_ORDER_HYBRID) first = hbar;
+      }
+      if ((st = pisa_select(base + L.q, kbar, route, route_lambda, rs, topk, idx, cs)) != PISA_OK) break;
+      if ((st = pisa_attention(base + L.q, base + L.k, base + L.v, kbar, S0, first, idx, rs, topk, order, scale,
+                               base + L.o, cs)) != PISA_OK)
+        break;
+      // copy out, once the range's kernels are done
+      if ((e = cudaEventRecord(computed[c], cs)) != cudaSuccess ||
+          (e = cudaStreamWaitEvent(out_s, computed[c], 0)) != cudaSuccess ||
+          (e = cudaMemcpyAsync(static_cast<uint8_t*>(O) + off, base + L.o, len, cudaMemcpyDeviceToHost, out_s)) !=
+              cudaSuccess ||
+          (e = cudaEventRecord(drained[c], out_s)) != cudaSuccess) {
+        st = cuda_fail("copy-out");
+        break;
+      }
+    }
+  } while (false);
+  // whatever happened, nothing may still run on the workspace or the host buffers when
+  // the call returns
+  for (int i = 0; i < 3; ++i) {
+    cudaStream_t s = i == 0 ? in_s : (i == 1 ? out_s : cs);
+    if (i < 2 && s == nullptr) continue;  // a copy stream that was never created
+    cudaError_t se = cudaStreamSynchronize(s);
+    if (se != cudaSuccess && st == PISA_OK) {
+      e = se;
+      st = cuda_fail("cudaStreamSynchronize");
+    }
+  }
+  for (cudaEvent_t x : ev) cudaEventDestroy(x);
+  if (in_s) cudaStreamDestroy(in_s);
+  if (out_s) cudaStreamDestroy(out_s);
+  return st;
 }
 
 pisa_status_t pisa_device_error(void* stream) {

@@ -49,6 +49,7 @@
 #ifndef PISA_H_
 #define PISA_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -169,6 +170,40 @@ pisa_status_t pisa_attention_simt(const void* Q, const void* K, const void* V, c
                                   const float* S0, const void* S1, const int32_t* idx,
                                   pisa_shape_t shape, int32_t topk, int32_t order, float scale,
                                   void* O, void* stream);
+
+/*
+ * pisa_run_host_workspace -- bytes of device workspace that pisa_run_host needs for
+ * this problem: *bytes = 0 for an empty problem. Same argument checks as pisa_run_host
+ * (no device is touched). The figure is about min(3, chunks) ranges of
+ * ceil(B*H / chunks) (batch, head) pairs, each holding its Q, K, V, O and statistics.
+ */
+pisa_status_t pisa_run_host_workspace(pisa_shape_t shape, int32_t topk, int32_t order, float route_lambda,
+                                      int32_t chunks, size_t* bytes);
+
+/*
+ * pisa_run_host -- the whole path on HOST buffers: pisa_block_stats, (with
+ * route_lambda > 0) pisa_routing_norms, pisa_select and pisa_attention, as one call.
+ *
+ * Section 2 of the explainer, "Hardware implementation": a precompute step, routing,
+ * then the fused kernel. Every step is independent across (batch, head) pairs, so the
+ * call splits the B*H pairs into `chunks` contiguous ranges and pipelines them through
+ * the workspace on three streams: the host-to-device copy of a range, the kernels of
+ * the previous one (on `stream`) and the device-to-host copy of the one before overlap.
+ * The result is bit for bit that of the four device calls on the whole batch.
+ * Q, K, V: HOST bf16 [B, H, N, d] (page-locked memory lets the copies overlap the
+ * kernels; pageable memory works, with less overlap); O: HOST bf16 [B, H, N, d],
+ * written; topk, order, scale as in pisa_attention; route_lambda: 0 for plain
+ * relevance, > 0 for covariance-aware routing with that weight (order 1 then attends
+ * with the per-block S1, order 2 with the routing call's Hbar); chunks >= 1.
+ * workspace: DEVICE memory owned by the caller, 256-byte aligned, of at least the
+ * size pisa_run_host_workspace reports for the same arguments; its contents are
+ * scratch. The call BLOCKS until O holds the whole result and nothing runs on the
+ * workspace or the host buffers any more. Device pointers passed as Q, K, V or O are
+ * rejected with PISA_ERR_INVALID_ARG.
+ */
+pisa_status_t pisa_run_host(const void* Q, const void* K, const void* V, pisa_shape_t shape, int32_t topk,
+                            int32_t order, float scale, float route_lambda, int32_t chunks, void* workspace,
+                            size_t workspace_bytes, void* O, void* stream);
 
 /*
  * pisa_device_error -- takes the device error word that the kernels set, after all

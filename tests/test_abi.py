@@ -179,3 +179,58 @@ def test_binding_raises_on_missing_library(tmp_path, monkeypatch):
     monkeypatch.setattr(P, "_lib", None)
     with pytest.raises(RuntimeError, match="missing"):
         P.lib()
+
+
+def _ws(L, s=None, topk=2, order=1, lam=0.0, chunks=8):
+    n = ctypes.c_size_t(123)
+    st = L.pisa_run_host_workspace(s or shape(), topk, order, lam, chunks, ctypes.byref(n))
+    return st, n.value
+
+
+def test_host_workspace_size(L):
+    """3 slots of ceil(B*H / chunks) pairs: Q, K, V, O, kbar, S0, S1 (or Hbar), routing
+    buffers and idx, each rounded up to 256 bytes."""
+    up = lambda x: -(-x // 256) * 256  # noqa: E731
+    B, H, N, d, b, k = 1, 24, 32768, 128, 64, 64
+    nB = N // b
+    R = 3                               # 24 pairs in 8 chunks
+    act = up(R * N * d * 2)
+    common = 4 * act + 2 * up(R * nB * d * 4) + up(R * nB * k * 4)
+    st, n1 = _ws(L, shape(B, H, N, d, b), k, 1)
+    assert st == OK and n1 == 3 * (common + up(R * nB * d * d * 2))
+    st, n2 = _ws(L, shape(B, H, N, d, b), k, 2)
+    assert st == OK and n2 == 3 * (common + up(R * d * d * 4))
+    st, nr = _ws(L, shape(B, H, N, d, b), k, 2, lam=0.01)
+    assert st == OK and nr == 3 * (common + up(R * nB * d * d * 2) + up(R * d * d * 4) + up(R * nB * 4))
+    st, n0 = _ws(L, shape(B, H, N, d, b), k, -1, chunks=1)
+    assert st == OK and n0 == 4 * up(24 * N * d * 2) + 2 * up(24 * nB * d * 4) + up(24 * nB * k * 4)
+    assert _ws(L, shape(N=0)) == (OK, 0)
+    assert _ws(L, chunks=0)[0] == INVALID
+    assert _ws(L, lam=-1.0)[0] == INVALID
+    assert _ws(L, order=5)[0] == INVALID
+    assert _ws(L, topk=9)[0] == INVALID
+    assert L.pisa_run_host_workspace(shape(), 2, 1, 0.0, 8, None) == INVALID
+
+
+def run_host(L, s=None, topk=2, order=1, scale=0.1, lam=0.0, chunks=2, ws=FAKE, nbytes=None, **ptrs):
+    p = {k: FAKE for k in ("Q", "K", "V", "O")}
+    p.update(ptrs)
+    if nbytes is None:
+        nbytes = _ws(L, s, topk, order, lam, chunks)[1]
+    return L.pisa_run_host(vp(p["Q"]), vp(p["K"]), vp(p["V"]), s or shape(), topk, order, scale, lam, chunks,
+                           vp(ws), nbytes, vp(p["O"]), None)
+
+
+def test_host_entry_arguments(L):
+    for name in ("Q", "K", "V", "O"):
+        assert run_host(L, **{name: 0}) == INVALID, name
+    assert run_host(L, ws=0) == INVALID
+    assert run_host(L, ws=FAKE + 16) == INVALID          # workspace must be 256-byte aligned
+    assert b"256" in L.pisa_last_error()
+    assert run_host(L, nbytes=100) == INVALID
+    assert b"needed" in L.pisa_last_error()
+    assert run_host(L, scale=0.0) == INVALID
+    assert run_host(L, chunks=0) == INVALID
+    assert run_host(L, s=shape(B=0), Q=0, K=0, V=0, O=0, ws=0, nbytes=0) == OK
+    _no_device()
+    _passes_validation(run_host(L, Q=MISALIGNED), L)     # host buffers need no alignment

@@ -214,23 +214,43 @@ def test_device_error_word_is_shared_per_device():
     P.device_error()          # taken by the first reader: nothing left
 
 
-def test_host_entry_point_matches_device():
+@pytest.mark.parametrize("order,lam", [(1, 0.0), (2, 0.0), (-1, 0.0), (0, 0.0), (2, 0.02), (1, 0.02)])
+def test_host_entry_point_matches_device(order, lam):
+    """pisa_run_host (host buffers in and out, through the C ABI) gives the bits of the
+    device calls on the whole batch, for every order, with and without routing."""
     wl = W.get("image").with_(B=1, H=2)
     q, k, v = W.make_inputs(wl)
     hq, hk, hv = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in (q, k, v))
-    Oh = P.pisa_host(hq, hk, hv, wl.block, wl.topk, wl.order, wl.scale)
-    Od, _ = P.pisa(hq.cuda(), hk.cuda(), hv.cuda(), wl.block, wl.topk, wl.order, wl.scale)
+    Oh = P.pisa_host(hq, hk, hv, wl.block, wl.topk, order, wl.scale, route_lambda=lam)
+    Od, _ = P.pisa(hq.cuda(), hk.cuda(), hv.cuda(), wl.block, wl.topk, order, wl.scale, route_lambda=lam)
     assert torch.equal(Oh.view(torch.int16), Od.cpu().view(torch.int16))
 
 
 def test_host_entry_point_pipelined_over_heads():
     """The host entry point splits (batch, head) pairs into ranges that copy and compute
-    on separate streams; every chunking gives the device path's bits."""
+    on separate streams through three workspace slots; every chunking gives the device
+    path's bits, with page-locked and with pageable host memory."""
     wl = W.get("image").with_(B=2, H=3)
     q, k, v = W.make_inputs(wl)
     hq, hk, hv = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in (q, k, v))
     Od, _ = P.pisa(hq.cuda(), hk.cuda(), hv.cuda(), wl.block, wl.topk, wl.order, wl.scale)
     ref = Od.cpu().view(torch.int16)
-    for chunks in (1, 4, 6, 16):
+    for chunks in (1, 2, 4, 6, 16):
         Oh = P.pisa_host(hq, hk, hv, wl.block, wl.topk, wl.order, wl.scale, chunks=chunks)
         assert torch.equal(Oh.view(torch.int16), ref), chunks
+    pq, pk, pv = (t.clone() for t in (hq, hk, hv))       # pageable copies
+    assert not pq.is_pinned()
+    Oh = P.pisa_host(pq, pk, pv, wl.block, wl.topk, wl.order, wl.scale, chunks=4)
+    assert torch.equal(Oh.view(torch.int16), ref)
+
+
+def test_host_entry_point_rejects_device_buffers():
+    wl = W.get("tiny")
+    q, k, v = (PT.to_device(a) for a in W.make_inputs(wl))
+    s = P.Shape(wl.B, wl.H, wl.N, wl.d, wl.block)
+    n = P.host_workspace_bytes(s, wl.topk, wl.order)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    O = torch.empty_like(q)
+    st = P.lib().pisa_run_host(P._ptr(q), P._ptr(k), P._ptr(v), s, wl.topk, wl.order, wl.scale, 0.0, 2,
+                               P._ptr(ws), n, P._ptr(O), None)
+    assert st == 1 and b"device memory" in P.lib().pisa_last_error()
