@@ -26,6 +26,7 @@ from .pisa import (  # noqa: F401
     block_stats,
     pooled_queries,
     select,
+    select_grouped,
     attention,
     dense_attention,
     global_first_order,

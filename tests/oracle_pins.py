@@ -528,3 +528,76 @@ def pin_routed_select_bruteforce(orc, seed=20, trials=30):
                     best, best_set = tot, sub
             bad += list(idx[0, 0, i]) != list(best_set)
     return bad
+
+
+# ----------------------------------------------------------------------------
+# selection amortisation: one proxy query per group of query blocks
+# ----------------------------------------------------------------------------
+def _best_subset(scores, among, k):
+    """Subset of `among` (size k) with the largest total score; ties -> the
+    lexicographically smallest subset (itertools.combinations order)."""
+    best, best_set = -math.inf, None
+    for sub in itertools.combinations(sorted(among), k):
+        tot = sum(scores[j] for j in sub)
+        if tot > best + 1e-12:
+            best, best_set = tot, sub
+    return list(best_set)
+
+
+def pin_grouped_bruteforce(orc, seed=22, trials=24):
+    """Grouped selection by scalar loops: the proxy is the mean of every real query row
+    of the group, its candidate list the best `c` blocks by exhaustive subset search,
+    and each member's row the best `k` of those candidates for its own pooled query
+    (ragged N, planted ties, optional routing bias). Returns #mismatched rows."""
+    r = _rng(seed)
+    bad = 0
+    for t in range(trials):
+        b = int(r.integers(1, 4))
+        nB = int(r.integers(4, 9))
+        N = b * nB - int(r.integers(0, b))
+        nB = -(-N // b)
+        d = int(r.integers(1, 4))
+        g = int(r.integers(1, 4))
+        k = int(r.integers(1, nB + 1))
+        c = int(r.integers(k, nB + 1))
+        Q = r.standard_normal((1, 1, N, d))
+        kbar = r.standard_normal((1, 1, nB, d))
+        if t % 3 == 0:
+            kbar[0, 0, nB - 1] = kbar[0, 0, 0]
+        lam = float(r.uniform(0.2, 2.0)) if t % 2 else 0.0
+        M = np.abs(r.standard_normal((1, 1, nB)))
+        idx, _ = orc.select_grouped(Q, kbar, b, k, g, c, route=M if lam else None, lam=lam)
+        bias = [lam * M[0, 0, j] for j in range(nB)]
+        for m in range(-(-nB // g)):
+            rows = list(range(m * g * b, min((m + 1) * g * b, N)))
+            proxy = [sum(Q[0, 0, s, a] for s in rows) / len(rows) for a in range(d)]
+            psc = [sum(proxy[a] * kbar[0, 0, j, a] for a in range(d)) + bias[j] for j in range(nB)]
+            cand = _best_subset(psc, range(nB), c)
+            for i in range(m * g, min((m + 1) * g, nB)):
+                qrows = list(range(i * b, min(i * b + b, N)))
+                qb = [sum(Q[0, 0, s, a] for s in qrows) / len(qrows) for a in range(d)]
+                msc = [sum(qb[a] * kbar[0, 0, j, a] for a in range(d)) + bias[j] for j in range(nB)]
+                bad += list(idx[0, 0, i]) != _best_subset(msc, cand, k)
+    return bad
+
+
+def pin_grouped_special_cases(orc, seed=23):
+    """Group 1 with any candidate count, and any group with candidates = nB, reduce to
+    plain selection; candidates = topk (the reuse mode) gives every member of a group
+    the same row. Returns #violations."""
+    r = _rng(seed)
+    B, H, N, d, b = 1, 2, 77, 5, 6
+    nB = -(-N // b)
+    Q = r.standard_normal((B, H, N, d))
+    kbar = r.standard_normal((B, H, nB, d))
+    plain, _, _ = orc.select(Q, kbar, b, 4)
+    bad = 0
+    for c in (4, 7, nB):
+        bad += int(np.any(orc.select_grouped(Q, kbar, b, 4, 1, c)[0] != plain))
+    for g in (2, 3, 5):
+        bad += int(np.any(orc.select_grouped(Q, kbar, b, 4, g, nB)[0] != plain))
+        reuse, _ = orc.select_grouped(Q, kbar, b, 4, g, 4)
+        for m in range(-(-nB // g)):
+            members = reuse[:, :, m * g:min((m + 1) * g, nB)]
+            bad += int(np.any(members != members[:, :, :1]))
+    return bad

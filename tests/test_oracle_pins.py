@@ -46,6 +46,8 @@ def _pins(orc):
         ("round_to_bf16", P.pin_round_to_bf16, lambda e: e == 0),
         ("routing_norms_bruteforce", P.pin_routing_norms_bruteforce, lambda e: e < TOL),
         ("routed_select_bruteforce", P.pin_routed_select_bruteforce, lambda e: e == 0),
+        ("grouped_bruteforce", P.pin_grouped_bruteforce, lambda e: e == 0),
+        ("grouped_special_cases", P.pin_grouped_special_cases, lambda e: e == 0),
     ]:
         try:
             v = fn(orc)
@@ -70,7 +72,8 @@ def real_pins():
     "permutation_in_block", "order0_convex", "worked_example",
     "convergence_order0", "convergence_order1", "drop_is_masked_softmax", "hybrid_bruteforce",
     "hybrid_shared_first_order", "hybrid_all_selected_is_dense", "round_to_bf16",
-    "routing_norms_bruteforce", "routed_select_bruteforce"])
+    "routing_norms_bruteforce", "routed_select_bruteforce", "grouped_bruteforce",
+    "grouped_special_cases"])
 def test_pin(real_pins, name):
     value, ok = real_pins[name]
     assert ok, f"{name}: {value}"
@@ -116,6 +119,11 @@ MUTATIONS = {
                                       "z = z - z.max(axis=-2, keepdims=True)"),
     "dense normaliser over queries": ("np.matmul(p, V) / p.sum(axis=-1, keepdims=True)",
                                       "np.matmul(p, V) / p.sum(axis=-2, keepdims=True)[..., :1]"),
+    "proxy from the group's first block only": ("proxy = Q[b, h, s:e].sum(axis=0) / (e - s)",
+                                                "proxy = qbar[b, h, m * group]"),
+    "members not refined to the candidates": ("_top(row, topk, among=cand)", "_top(row, topk)"),
+    "group span one token short": ("span = group * block", "span = group * block - 1"),
+    "candidates ranked lowest first": ("order = np.lexsort((cols, -vals))", "order = np.lexsort((cols, vals))"),
     "bf16 ties away from even": ("r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16",
                                  "r = ((u + 0x8000) >> 16) << 16"),
 }
