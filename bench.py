@@ -164,8 +164,15 @@ def oracle_sample(wl, budget_s: float = 15.0, min_blocks: int = 2):
             S1 = oracle.round_to_bf16(S1).mean(axis=2)
     elif wl.order == 2:
         S1 = oracle.global_first_order(S1)
-    idx, _, _ = oracle.select(Qf, kbar, wl.block, wl.topk, route=route, lam=wl.route_lambda)
-    t_pre = time.perf_counter() - t0
+    t_stats = time.perf_counter() - t0
+    t1 = time.perf_counter()
+    if wl.select_group > 1 or wl.select_cand:
+        idx, _ = oracle.select_grouped(Qf, kbar, wl.block, wl.topk, wl.select_group, wl.select_cand or wl.nB,
+                                       route=route, lam=wl.route_lambda)
+    else:
+        idx, _, _ = oracle.select(Qf, kbar, wl.block, wl.topk, route=route, lam=wl.route_lambda)
+    # with index reuse the selection belongs to an earlier call: it is not in the step
+    t_pre = t_stats + (0.0 if wl.reuse_idx else time.perf_counter() - t1)
     # query blocks spread over the sequence, run until the budget is spent
     order = np.random.default_rng(0).permutation(wl.nB)
     done, t1 = 0, time.perf_counter()
@@ -177,7 +184,7 @@ def oracle_sample(wl, budget_s: float = 15.0, min_blocks: int = 2):
     frac_q = done / wl.nB
     flops = (R.attention_flops(1, 1, wl.N, wl.d, wl.block, wl.topk, wl.order) * frac_q
              + R.stats_flops(1, 1, wl.N, wl.d, wl.block, 1 if routed else wl.order)
-             + R.select_flops(1, 1, wl.N, wl.d, wl.block))
+             + _select_flops(wl.with_(B=1, H=1)))
     secs = t_pre + t_attn
     threads = _blas_threads()
     desc = (f"oracle fp64 on head 0 of {wl.name}: full stats + select, attention on {done} of "
@@ -209,7 +216,11 @@ def near_tie_report(wl, q, k, v, gpu_idx):
             Qf, Kf, Vf = (W.bf16_bits_to_f32(a[b:b + 1, h:h + 1]).astype(np.float64) for a in (q, k, v))
             kbar, _, S1 = oracle.block_stats(Kf, Vf, wl.block, 1 if routed else 0)
             route = oracle.routing_norms(S1) if routed else None
-            ridx, near, _ = oracle.select(Qf, kbar, wl.block, wl.topk, route=route, lam=wl.route_lambda)
+            if wl.select_group > 1 or wl.select_cand:
+                ridx, near = oracle.select_grouped(Qf, kbar, wl.block, wl.topk, wl.select_group,
+                                                   wl.select_cand or wl.nB, route=route, lam=wl.route_lambda)
+            else:
+                ridx, near, _ = oracle.select(Qf, kbar, wl.block, wl.topk, route=route, lam=wl.route_lambda)
             bad = np.any(gpu_idx[b:b + 1, h:h + 1] != ridx, axis=-1)
             rows += bad.size
             flagged += int(near.sum())
@@ -287,8 +298,19 @@ def _captured_traffic(wl):
     return d["dram_bytes_per_full_launch"] if h == d["sources_sha256"] else None
 
 
+def _select_flops(wl):
+    if wl.reuse_idx:          # the indices come from an earlier call
+        return 0.0
+    cand = wl.select_cand if wl.select_cand else 0
+    if wl.select_cand == wl.topk and wl.select_group > 1:     # reuse mode: no member scores
+        return R.select_flops(wl.B, wl.H, wl.N, wl.d, wl.block, wl.select_group, wl.nB) - \
+            2.0 * wl.B * wl.H * wl.d * wl.nB * wl.nB
+    return R.select_flops(wl.B, wl.H, wl.N, wl.d, wl.block, wl.select_group, cand)
+
+
 def _step_flops(wl):
-    flops = R.step_flops(wl.B, wl.H, wl.N, wl.d, wl.block, wl.topk, wl.order)
+    flops = (R.attention_flops(wl.B, wl.H, wl.N, wl.d, wl.block, wl.topk, wl.order)
+             + R.stats_flops(wl.B, wl.H, wl.N, wl.d, wl.block, wl.order) + _select_flops(wl))
     if wl.route_lambda > 0 and wl.order != 1:   # per-block S1 is formed for the routing norms
         flops += R.stats_flops(wl.B, wl.H, wl.N, wl.d, wl.block, 1) - R.stats_flops(
             wl.B, wl.H, wl.N, wl.d, wl.block, wl.order)
@@ -306,6 +328,9 @@ def _config(wl, ws, shard="batch"):
     return {"workload": _workload_desc(wl), "global_batch": wl.B * (1 if shard == "heads" else ws), "seq_len": wl.N,
             "heads": wl.H, "head_dim": wl.d, "block": wl.block, "topk": wl.topk,
             "keep": wl.topk / wl.nB, "order": wl.order, "route_lambda": wl.route_lambda,
+            "selection": ("indices of an earlier call reused (no selection in the step)" if wl.reuse_idx else
+                          f"one proxy per {wl.select_group} query blocks, {wl.select_cand or wl.nB} candidates"
+                          if (wl.select_group > 1 or wl.select_cand) else "per query block"),
             "l2": "inputs larger than L2 (Q+K+V %.0f MB per GPU), no flush" % (3 * wl.B * wl.H * wl.N * wl.d * 2 / 1e6),
             "parallelism": par}
 
@@ -358,6 +383,7 @@ def run_ours(args):
     O = torch.empty_like(Q)
     attn = P.attention if args.kernel == "fused" else P.attention_simt
     stream = torch.cuda.current_stream(dev)
+    sel_opts = dict(group=wl.select_group, candidates=wl.select_cand or None)
 
     def step(ev=None):
         if ev is not None:
@@ -369,13 +395,19 @@ def run_ours(args):
             P.routing_norms(S1, wl.block, wl.N, out=(Hbar, M))
         if ev is not None:
             ev[2].record(stream)
-        P.select(Q, kbar, wl.block, wl.topk, out=idx, route=M, lam=wl.route_lambda)
+        if not wl.reuse_idx:
+            P.select(Q, kbar, wl.block, wl.topk, out=idx, route=M, lam=wl.route_lambda, **sel_opts)
         if ev is not None:
             ev[3].record(stream)
         attn(Q, K, V, kbar, S0, first, idx, wl.block, wl.order, wl.scale, out=O)
         if ev is not None:
             ev[4].record(stream)
 
+    if wl.reuse_idx:
+        # index reuse: the indices of an earlier call (here: one full selection before
+        # the timed region) serve every step, whose path is stats + attention
+        P.block_stats(K, V, wl.block, stats_order, out=(kbar, S0, S1))
+        P.select(Q, kbar, wl.block, wl.topk, out=idx, route=M, lam=wl.route_lambda)
     for _ in range(args.warmup):
         step()
     P.device_error()
@@ -409,7 +441,8 @@ def run_ours(args):
     att_tf = att_flops / (k_ms["attention"] * 1e-3) / 1e12
     dense_tf = R.dense_flops(wl.B, wl.H, wl.N, wl.d) / (k_ms["attention"] * 1e-3) / 1e12
     st_gbs = R.stats_bytes(wl.B, wl.H, wl.N, wl.d, wl.block, stats_order) / (k_ms["stats"] * 1e-3) / 1e9
-    se_gbs = R.select_bytes(wl.B, wl.H, wl.N, wl.d, wl.block, wl.topk) / (k_ms["select"] * 1e-3) / 1e9
+    se_gbs = (None if wl.reuse_idx else
+              R.select_bytes(wl.B, wl.H, wl.N, wl.d, wl.block, wl.topk) / (k_ms["select"] * 1e-3) / 1e9)
     pk = _peaks()
     # the attention kernel runs in a timed region well under a few seconds: the burst
     # bf16 peak is its denominator (the sustained figure is for seconds-long loops)
@@ -417,11 +450,11 @@ def run_ours(args):
 
     # end to end through the public host API: pinned host Q, K, V in, O out
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not wl.reuse_idx:   # one host call cannot reuse an earlier call's indices
         hq, hk, hv = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in (q, k, v))
         for _ in range(2):
             P.pisa_host(hq, hk, hv, wl.block, wl.topk, wl.order, wl.scale, device=dev,
-                        route_lambda=wl.route_lambda)
+                        route_lambda=wl.route_lambda, group=wl.select_group, candidates=wl.select_cand)
         n_e2e = max(2, min(args.steps, 5))
         if pg:
             pg.barrier()
@@ -432,7 +465,7 @@ def run_ours(args):
         e0.record(stream)
         for _ in range(n_e2e):
             P.pisa_host(hq, hk, hv, wl.block, wl.topk, wl.order, wl.scale, device=dev,
-                        route_lambda=wl.route_lambda)
+                        route_lambda=wl.route_lambda, group=wl.select_group, candidates=wl.select_cand)
         e1.record(stream)
         torch.cuda.synchronize()
         wall = (time.perf_counter() - t0) * 1e3 / n_e2e
@@ -470,7 +503,7 @@ def run_ours(args):
         "attention_effective_tflops": att_tf,
         "attention_dense_equivalent_tflops": dense_tf,
         "stats_gbs": st_gbs, "stats_hbm_frac": st_gbs / pk["hbm"],
-        "select_gbs": se_gbs, "select_hbm_frac": se_gbs / pk["hbm"],
+        "select_gbs": se_gbs, "select_hbm_frac": None if se_gbs is None else se_gbs / pk["hbm"],
         **({"routing_gbs": R.routing_bytes(wl.B, wl.H, wl.N, wl.d, wl.block) / (k_ms["routing"] * 1e-3) / 1e9}
            if routed else {}),
         "e2e": e2e, "cpu_baseline": cpu, "near_ties": near,

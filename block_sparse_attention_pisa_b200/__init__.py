@@ -20,7 +20,7 @@ import os
 ORDER_DROP, ORDER_ZERO, ORDER_FIRST, ORDER_HYBRID = -1, 0, 1, 2
 
 __all__ = [
-    "ORDER_DROP", "ORDER_ZERO", "ORDER_FIRST", "ORDER_HYBRID", "PisaError", "Shape", "lib", "block_stats", "select", "attention", "attention_simt",
+    "ORDER_DROP", "ORDER_ZERO", "ORDER_FIRST", "ORDER_HYBRID", "PisaError", "Shape", "HostOptions", "lib", "block_stats", "select", "attention", "attention_simt",
     "pisa", "pisa_host", "host_workspace_bytes", "head_chunks", "device_error", "num_blocks", "LIB_PATH", "SYMBOLS", "routing_norms",
 ]
 
@@ -30,7 +30,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpisa.so"
 SYMBOLS = (
     "pisa_block_stats", "pisa_select", "pisa_routing_norms", "pisa_attention", "pisa_attention_simt",
     "pisa_device_error", "pisa_status_string", "pisa_last_error", "pisa_version",
-    "pisa_run_host_workspace", "pisa_run_host",
+    "pisa_run_host_workspace", "pisa_run_host", "pisa_select_grouped",
 )
 
 STATUS = {0: "PISA_OK", 1: "PISA_ERR_INVALID_ARG", 2: "PISA_ERR_UNSUPPORTED",
@@ -48,6 +48,12 @@ class Shape(ctypes.Structure):
                 ("d", ctypes.c_int32), ("block", ctypes.c_int32)]
 
 
+class HostOptions(ctypes.Structure):
+    """pisa_host_options_t: routing weight, grouped selection and pipeline ranges (0: default)."""
+    _fields_ = [("route_lambda", ctypes.c_float), ("group", ctypes.c_int32),
+                ("candidates", ctypes.c_int32), ("chunks", ctypes.c_int32)]
+
+
 _lib = None
 
 
@@ -63,12 +69,14 @@ def lib():
     vp, i32, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
     L.pisa_block_stats.argtypes = [vp, vp, Shape, i32, vp, vp, vp, vp]
     L.pisa_select.argtypes = [vp, vp, vp, f32, Shape, i32, vp, vp]
+    L.pisa_select_grouped.argtypes = [vp, vp, vp, f32, Shape, i32, i32, i32, vp, vp]
     L.pisa_routing_norms.argtypes = [vp, Shape, vp, vp, vp]
     attn = [vp, vp, vp, vp, vp, vp, vp, Shape, i32, i32, f32, vp, vp]
     L.pisa_attention.argtypes = attn
     L.pisa_attention_simt.argtypes = attn
-    L.pisa_run_host_workspace.argtypes = [Shape, i32, i32, f32, i32, ctypes.POINTER(ctypes.c_size_t)]
-    L.pisa_run_host.argtypes = [vp, vp, vp, Shape, i32, i32, f32, f32, i32, vp, ctypes.c_size_t, vp, vp]
+    opts = ctypes.POINTER(HostOptions)
+    L.pisa_run_host_workspace.argtypes = [Shape, i32, i32, opts, ctypes.POINTER(ctypes.c_size_t)]
+    L.pisa_run_host.argtypes = [vp, vp, vp, Shape, i32, i32, f32, opts, vp, ctypes.c_size_t, vp, vp]
     L.pisa_device_error.argtypes = [vp]
     L.pisa_status_string.argtypes = [ctypes.c_int]
     L.pisa_status_string.restype = ctypes.c_char_p
@@ -76,7 +84,8 @@ def lib():
     L.pisa_last_error.restype = ctypes.c_char_p
     L.pisa_version.argtypes = []
     for name in ("pisa_block_stats", "pisa_select", "pisa_routing_norms", "pisa_attention", "pisa_attention_simt",
-                 "pisa_device_error", "pisa_version", "pisa_run_host_workspace", "pisa_run_host"):
+                 "pisa_device_error", "pisa_version", "pisa_run_host_workspace", "pisa_run_host",
+                 "pisa_select_grouped"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -191,10 +200,14 @@ def block_stats(K, V, block: int, order: int = 1, out=None):
     return kbar, S0, S1
 
 
-def select(Q, kbar, block: int, topk: int, out=None, route=None, lam: float = 0.0):
+def select(Q, kbar, block: int, topk: int, out=None, route=None, lam: float = 0.0,
+           group: int = 1, candidates: int | None = None):
     """int32 [B, H, nB, topk]: critical blocks of every query block (ascending).
     ``route`` (fp32 [B, H, nB], from ``routing_norms``) and ``lam`` add the
-    covariance term lam * M_j to every score."""
+    covariance term lam * M_j to every score. With ``group`` > 1 (or ``candidates``
+    below nB) the selection is grouped: one proxy query per ``group`` query blocks keeps
+    ``candidates`` key blocks, and each member keeps its best ``topk`` of them
+    (``candidates`` = topk hands the proxy's list to every member)."""
     import torch
     s = _shape(Q, block)
     nB = num_blocks(s.N, block)
@@ -210,8 +223,13 @@ def select(Q, kbar, block: int, topk: int, out=None, route=None, lam: float = 0.
             raise ValueError(f"{name} is on {t.device}, expected {dev}")
     idx = (torch.empty((s.B, s.H, nB, topk), device=Q.device, dtype=torch.int32)
            if out is None else out)
-    _check(lib().pisa_select(_ptr(Q), _ptr(kbar), _ptr(route), float(lam), s, topk, _ptr(idx),
-                             _stream(Q)))
+    if group == 1 and (candidates is None or candidates == nB):
+        _check(lib().pisa_select(_ptr(Q), _ptr(kbar), _ptr(route), float(lam), s, topk, _ptr(idx),
+                                 _stream(Q)))
+    else:
+        cand = nB if candidates is None else int(candidates)
+        _check(lib().pisa_select_grouped(_ptr(Q), _ptr(kbar), _ptr(route), float(lam), s, topk, int(group),
+                                         cand, _ptr(idx), _stream(Q)))
     return idx
 
 
@@ -287,21 +305,22 @@ def attention_simt(Q, K, V, kbar, S0, S1, idx, block: int, order: int, scale: fl
 
 
 def pisa(Q, K, V, block: int, topk: int, order: int = 1, scale: float | None = None,
-         route_lambda: float = 0.0, out=None):
+         route_lambda: float = 0.0, out=None, group: int = 1, candidates: int | None = None):
     """The whole path on device tensors: stats -> select -> attention. Returns (O, idx).
     With ``route_lambda`` > 0 the selection is covariance-aware: stats at order 1 ->
     routing norms -> routed select -> attention (at order 2 with the routing call's
-    Hbar)."""
+    Hbar). ``group`` / ``candidates`` select with grouped proxies (see ``select``)."""
     if scale is None:
         scale = Q.shape[-1] ** -0.5
+    sel = dict(group=group, candidates=candidates)
     if route_lambda > 0.0:
         kbar, S0, S1 = block_stats(K, V, block, ORDER_FIRST)
         Hbar, M = routing_norms(S1, block, Q.shape[2])
-        idx = select(Q, kbar, block, topk, route=M, lam=route_lambda)
+        idx = select(Q, kbar, block, topk, route=M, lam=route_lambda, **sel)
         first = Hbar if order == ORDER_HYBRID else (S1 if order == ORDER_FIRST else None)
         return attention(Q, K, V, kbar, S0, first, idx, block, order, scale, out=out), idx
     kbar, S0, S1 = block_stats(K, V, block, order)
-    idx = select(Q, kbar, block, topk)
+    idx = select(Q, kbar, block, topk, **sel)
     return attention(Q, K, V, kbar, S0, S1, idx, block, order, scale, out=out), idx
 
 
@@ -312,22 +331,25 @@ def head_chunks(BH: int, chunks: int):
     return [(edges[c], edges[c + 1]) for c in range(chunks) if edges[c + 1] > edges[c]]
 
 
-def host_workspace_bytes(shape: Shape, topk: int, order: int, route_lambda: float = 0.0, chunks: int = 8) -> int:
+def host_workspace_bytes(shape: Shape, topk: int, order: int, route_lambda: float = 0.0, chunks: int = 8,
+                         group: int = 1, candidates: int = 0) -> int:
     """Device workspace (bytes) that ``pisa_host`` needs for this problem."""
     n = ctypes.c_size_t(0)
-    _check(lib().pisa_run_host_workspace(shape, int(topk), int(order), float(route_lambda), int(chunks),
-                                         ctypes.byref(n)))
+    o = HostOptions(float(route_lambda), int(group), int(candidates), int(chunks))
+    _check(lib().pisa_run_host_workspace(shape, int(topk), int(order), ctypes.byref(o), ctypes.byref(n)))
     return int(n.value)
 
 
 def pisa_host(Q, K, V, block: int, topk: int, order: int = 1, scale: float | None = None,
-              device="cuda", route_lambda: float = 0.0, chunks: int = 8, out=None):
+              device="cuda", route_lambda: float = 0.0, chunks: int = 8, out=None,
+              group: int = 1, candidates: int = 0):
     """The whole path on HOST tensors [B, H, N, d] through the C ABI's ``pisa_run_host``:
     the library copies Q, K, V to the device, runs the path and copies O back, pipelined
     over ``chunks`` ranges of (batch, head) pairs (copies of one range overlap the kernels
     of another; the result equals the whole-batch device path bit for bit). Pinned host
-    tensors let the copies run asynchronously. Returns O on the host (``out`` if given).
-    The device workspace is allocated here with torch."""
+    tensors let the copies run asynchronously. ``group`` / ``candidates`` select with
+    grouped proxies as ``select`` does. Returns O on the host (``out`` if given). The
+    device workspace is allocated here with torch."""
     import torch
     if scale is None:
         scale = Q.shape[-1] ** -0.5
@@ -344,12 +366,14 @@ def pisa_host(Q, K, V, block: int, topk: int, order: int = 1, scale: float | Non
     dev = torch.device(device)
     if dev.index is None:
         dev = torch.device("cuda", torch.cuda.current_device())
+    o = HostOptions(float(route_lambda), int(group), int(candidates or 0), int(chunks))
     with torch.cuda.device(dev):
-        nbytes = host_workspace_bytes(s, topk, order, route_lambda, chunks)
-        ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+        nbytes = ctypes.c_size_t(0)
+        _check(lib().pisa_run_host_workspace(s, int(topk), int(order), ctypes.byref(o), ctypes.byref(nbytes)))
+        ws = torch.empty(max(nbytes.value, 1), dtype=torch.uint8, device=dev)
         stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
         _check(lib().pisa_run_host(_ptr(Q), _ptr(K), _ptr(V), s, int(topk), int(order), float(scale),
-                                   float(route_lambda), int(chunks), _ptr(ws), nbytes, _ptr(out), stream))
+                                   ctypes.byref(o), _ptr(ws), nbytes.value, _ptr(out), stream))
     return out
 
 

@@ -159,13 +159,39 @@ pisa_status_t launch_stats(const pisa_shape_t& s, const bf16* K, const bf16* V, 
 
 template <int D>
 pisa_status_t launch_select(const pisa_shape_t& s, const bf16* Q, const float* kbar, const float* route,
-                            float lambda, int topk, int32_t* idx, cudaStream_t st) {
+                            float lambda, int topk, int group, int cand, int32_t* idx, int sms, cudaStream_t st) {
   auto k = pisa::select_kernel<D>;
   const int nB = int(num_blocks(s));
-  const size_t smem = pisa::select_smem_bytes(D, nB);
+  pisa::SelParams p{};
+  p.Q = Q;
+  p.kbar = kbar;
+  p.route = route;
+  p.lambda = lambda;
+  p.idx = idx;
+  p.N = s.N;
+  p.nB = nB;
+  p.block = s.block;
+  p.topk = topk;
+  p.group = group;
+  p.cand = cand;
+  p.QB = group * (pisa::kSelQB / group > 1 ? pisa::kSelQB / group : 1);
+  p.tiles_per_head = (nB + p.QB - 1) / p.QB;
+  const int64_t tiles = int64_t(s.B) * s.H * p.tiles_per_head;
+  if (tiles > (int64_t(1) << 30)) return fail(PISA_ERR_UNSUPPORTED, "too many select tiles (%lld)", (long long)tiles);
+  p.total_tiles = int(tiles);
+  p.ld = pisa::select_key_ld(nB);
+  // ring: up to two tiles' stages, as many as fit next to the rest of shared memory
+  constexpr int kMaxSmem = 227 * 1024 - 128;  // minus the base-alignment slack
+  const int spt = p.QB * (s.block / pisa::kSelStageRows);
+  int ring = 2 * spt;
+  while (ring > 2 && pisa::select_smem(D, nB, ring).bytes > kMaxSmem) --ring;
+  if (pisa::select_smem(D, nB, ring).bytes > kMaxSmem)
+    return fail(PISA_ERR_UNSUPPORTED, "select shared memory for nB=%d exceeds the limit", nB);
+  p.ring = ring;
+  const size_t smem = size_t(pisa::select_smem(D, nB, ring).bytes) + 128;
   PISA_TRY(set_smem(k, smem));
-  dim3 grid((nB + pisa::kSelectQB - 1) / pisa::kSelectQB, s.B * s.H);
-  k<<<grid, pisa::kSelectThreads, smem, st>>>(Q, kbar, route, lambda, s.N, nB, s.block, topk, idx);
+  const int grid = int(tiles < sms ? tiles : sms);
+  k<<<grid, pisa::kSelThreads, smem, st>>>(p);
   return check_launch("select_kernel");
 }
 
@@ -316,8 +342,9 @@ pisa_status_t pisa_block_stats(const void* K, const void* V, pisa_shape_t shape,
   return launch_stats<64, 128>(shape, k, v, order, kbar, S0, S1, st);
 }
 
-pisa_status_t pisa_select(const void* Q, const float* kbar, const float* route, float lambda, pisa_shape_t shape,
-                          int32_t topk, int32_t* idx, void* stream) {
+pisa_status_t pisa_select_grouped(const void* Q, const float* kbar, const float* route, float lambda,
+                                  pisa_shape_t shape, int32_t topk, int32_t group, int32_t candidates, int32_t* idx,
+                                  void* stream) {
   bool empty = false;
   PISA_TRY(check_shape(shape, &empty));
   if (empty) return ok();
@@ -330,13 +357,27 @@ pisa_status_t pisa_select(const void* Q, const float* kbar, const float* route, 
       return fail(PISA_ERR_INVALID_ARG, "lambda=%g (must be finite and >= 0)", double(lambda));
   }
   PISA_TRY(check_topk(shape, topk));
+  if (group < 1 || group > pisa::kSelMaxGroup)
+    return fail(PISA_ERR_INVALID_ARG, "group=%d outside [1, %d]", group, pisa::kSelMaxGroup);
+  if (candidates < topk || candidates > num_blocks(shape))
+    return fail(PISA_ERR_INVALID_ARG, "candidates=%d outside [topk=%d, nB=%lld]", candidates, topk,
+                (long long)num_blocks(shape));
   PISA_TRY(check_support(shape));
   int sms = 0;
   PISA_TRY(check_device(&sms));
   auto st = static_cast<cudaStream_t>(stream);
   auto q = static_cast<const bf16*>(Q);
-  if (shape.d == 128) return launch_select<128>(shape, q, kbar, route, lambda, topk, idx, st);
-  return launch_select<64>(shape, q, kbar, route, lambda, topk, idx, st);
+  if (shape.d == 128) return launch_select<128>(shape, q, kbar, route, lambda, topk, group, candidates, idx, sms, st);
+  return launch_select<64>(shape, q, kbar, route, lambda, topk, group, candidates, idx, sms, st);
+}
+
+pisa_status_t pisa_select(const void* Q, const float* kbar, const float* route, float lambda, pisa_shape_t shape,
+                          int32_t topk, int32_t* idx, void* stream) {
+  bool empty = false;
+  PISA_TRY(check_shape(shape, &empty));
+  if (empty) return ok();
+  // plain selection: every query block is its own proxy and every key block a candidate
+  return pisa_select_grouped(Q, kbar, route, lambda, shape, topk, 1, int32_t(num_blocks(shape)), idx, stream);
 }
 
 pisa_status_t pisa_routing_norms(const void* S1, pisa_shape_t shape, float* Hbar, float* M, void* stream) {
@@ -395,8 +436,36 @@ pisa_status_t pisa_attention_simt(const void* Q, const void* K, const void* V, c
   return launch_attention_simt<64>(shape, q, k, v, kbar, S0, s1, idx, topk, order, scale, o, st);
 }
 
-pisa_status_t pisa_run_host_workspace(pisa_shape_t shape, int32_t topk, int32_t order, float route_lambda,
-                                       int32_t chunks, size_t* bytes) {
+}  // extern "C"
+
+namespace {
+
+// options with their defaults filled in, checked against the problem
+pisa_status_t host_options(const pisa_shape_t& s, int32_t topk, const pisa_host_options_t* in,
+                           pisa_host_options_t* out) {
+  pisa_host_options_t o{0.f, 1, 0, 8};
+  if (in != nullptr) o = *in;
+  if (o.group == 0) o.group = 1;
+  if (o.chunks == 0) o.chunks = 8;
+  const int32_t nB = int32_t(num_blocks(s));
+  if (o.candidates == 0) o.candidates = nB;
+  if (!std::isfinite(o.route_lambda) || o.route_lambda < 0.f)
+    return fail(PISA_ERR_INVALID_ARG, "route_lambda=%g (must be finite and >= 0)", double(o.route_lambda));
+  if (o.chunks < 1) return fail(PISA_ERR_INVALID_ARG, "chunks=%d (must be >= 1)", o.chunks);
+  if (o.group < 1 || o.group > pisa::kSelMaxGroup)
+    return fail(PISA_ERR_INVALID_ARG, "group=%d outside [1, %d]", o.group, pisa::kSelMaxGroup);
+  if (o.candidates < topk || o.candidates > nB)
+    return fail(PISA_ERR_INVALID_ARG, "candidates=%d outside [topk=%d, nB=%d]", o.candidates, topk, nB);
+  *out = o;
+  return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+pisa_status_t pisa_run_host_workspace(pisa_shape_t shape, int32_t topk, int32_t order,
+                                      const pisa_host_options_t* options, size_t* bytes) {
   if (bytes == nullptr) return fail(PISA_ERR_INVALID_ARG, "bytes is NULL");
   *bytes = 0;
   bool empty = false;
@@ -404,20 +473,23 @@ pisa_status_t pisa_run_host_workspace(pisa_shape_t shape, int32_t topk, int32_t 
   if (empty) return ok();
   PISA_TRY(check_order(order));
   PISA_TRY(check_topk(shape, topk));
-  if (chunks < 1) return fail(PISA_ERR_INVALID_ARG, "chunks=%d (must be >= 1)", chunks);
-  if (!std::isfinite(route_lambda) || route_lambda < 0.f)
-    return fail(PISA_ERR_INVALID_ARG, "route_lambda=%g (must be finite and >= 0)", double(route_lambda));
+  pisa_host_options_t o;
+  PISA_TRY(host_options(shape, topk, options, &o));
   PISA_TRY(check_support(shape));
-  *bytes = pisa_host::workspace_bytes(shape, topk, order, route_lambda > 0.f, chunks);
+  *bytes = pisa_host::workspace_bytes(shape, topk, order, o.route_lambda > 0.f, o.chunks);
   return ok();
 }
 
 pisa_status_t pisa_run_host(const void* Q, const void* K, const void* V, pisa_shape_t shape, int32_t topk,
-                            int32_t order, float scale, float route_lambda, int32_t chunks, void* workspace,
+                            int32_t order, float scale, const pisa_host_options_t* options, void* workspace,
                             size_t workspace_bytes, void* O, void* stream) {
   size_t need = 0;
-  PISA_TRY(pisa_run_host_workspace(shape, topk, order, route_lambda, chunks, &need));
+  PISA_TRY(pisa_run_host_workspace(shape, topk, order, options, &need));
   if (need == 0) return ok();  // empty problem: nothing touched
+  pisa_host_options_t opt;
+  PISA_TRY(host_options(shape, topk, options, &opt));
+  const float route_lambda = opt.route_lambda;
+  const int32_t chunks = opt.chunks;
   const void* host[4] = {Q, K, V, O};
   const char* names[4] = {"Q", "K", "V", "O"};
   for (int i = 0; i < 4; ++i)
@@ -514,7 +586,9 @@ pisa_status_t pisa_run_host(const void* Q, const void* K, const void* V, pisa_sh
         route = M;
         if (order == PISA_ORDER_HYBRID) first = hbar;
       }
-      if ((st = pisa_select(base + L.q, kbar, route, route_lambda, rs, topk, idx, cs)) != PISA_OK) break;
+      if ((st = pisa_select_grouped(base + L.q, kbar, route, route_lambda, rs, topk, opt.group, opt.candidates, idx,
+                                    cs)) != PISA_OK)
+        break;
       if ((st = pisa_attention(base + L.q, base + L.k, base + L.v, kbar, S0, first, idx, rs, topk, order, scale,
                                base + L.o, cs)) != PISA_OK)
         break;

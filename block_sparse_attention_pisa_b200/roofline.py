@@ -12,7 +12,8 @@ Per-unit figures:
   (2*nB*d*4) + S1 written (nB*d*d*2 at order 1) or Hbar written (d*d*4 at
   order 2); flops = 2*n*d*d per block for K^T V (orders 1 and 2).
 * select: bytes = Q read (N*d*2) + kbar read (nB*d*4) + idx written
-  (nB*k*4); flops = 2*d per (query block, key block) pooled score.
+  (nB*k*4); flops = 2*d per (query block, key block) pooled score; grouped:
+  2*d per (proxy, key block) + 2*d per (member block, candidate).
 * routing (covariance-aware): bytes = per-block S1 read twice (2*nB*d*d*2:
   once for Hbar, once for the deviations) + Hbar written and read (2*d*d*4)
   + M written (nB*4).
@@ -74,9 +75,16 @@ def routing_bytes(B, H, N, d, block) -> float:
     return float(B * H * (2 * nB * d * d * 2 + 2 * d * d * 4 + nB * 4))
 
 
-def select_flops(B, H, N, d, block) -> float:
+def select_flops(B, H, N, d, block, group: int = 1, cand: int = 0) -> float:
+    """Pooled-score flops: 2 d per (query block, key block) for plain selection; with
+    grouped proxies 2 d per (proxy, key block) plus 2 d per (member, candidate) (none
+    when the candidate list is handed over unchanged)."""
     nB = num_blocks(N, block)
-    return float(B * H * 2.0 * nB * nB * d)
+    if group == 1 and cand in (0, nB):
+        return float(B * H * 2.0 * nB * nB * d)
+    ng = -(-nB // group)
+    c = nB if cand == 0 else cand
+    return float(B * H * 2.0 * d * (ng * nB + nB * c))
 
 
 def step_flops(B, H, N, d, block, topk, order) -> float:

@@ -117,6 +117,24 @@ pisa_status_t pisa_select(const void* Q, const float* kbar, const float* route, 
                           pisa_shape_t shape, int32_t topk, int32_t* idx, void* stream);
 
 /*
+ * pisa_select_grouped -- pisa_select with one proxy query per group of query blocks.
+ *
+ * PIVOT page ("PIVOT slashes sparse-attention indexer cost 4x and cuts latency 1.6x"),
+ * "Two observations behind PIVOT": neighbouring queries pick nearly the same blocks, so
+ * `group` consecutive query blocks [m*group, (m+1)*group) share a proxy query, the mean
+ * of all their real rows. The proxy is scored against every key block (qbar . kbar_j,
+ * plus lambda * M_j with `route`) and keeps its `candidates` best as a candidate list;
+ * each member query block then keeps the topk candidates with its own best pooled
+ * scores. candidates == topk is the reuse mode (every member takes the proxy's list);
+ * group == 1 with candidates == nB is pisa_select. Ties go to the lower block index,
+ * rows are written ascending. 1 <= group <= 8; topk <= candidates <= nB; other
+ * arguments as pisa_select.
+ */
+pisa_status_t pisa_select_grouped(const void* Q, const float* kbar, const float* route, float lambda,
+                                  pisa_shape_t shape, int32_t topk, int32_t group, int32_t candidates, int32_t* idx,
+                                  void* stream);
+
+/*
  * pisa_routing_norms -- the covariance-aware routing statistic.
  *
  * Section 2, "Covariance-aware routing": the selection score of a block carries the
@@ -171,30 +189,38 @@ pisa_status_t pisa_attention_simt(const void* Q, const void* K, const void* V, c
                                   pisa_shape_t shape, int32_t topk, int32_t order, float scale,
                                   void* O, void* stream);
 
+/* Options of the host-buffer entry point (NULL: all defaults). */
+typedef struct {
+  float route_lambda;  /* 0 (default): plain relevance; > 0: covariance-aware routing weight */
+  int32_t group;       /* query blocks per proxy query for the selection (default / 0: 1)     */
+  int32_t candidates;  /* proxy candidate-list length (default / 0: every key block)           */
+  int32_t chunks;      /* (batch, head) ranges pipelined through the workspace (default / 0: 8) */
+} pisa_host_options_t;
+
 /*
  * pisa_run_host_workspace -- bytes of device workspace that pisa_run_host needs for
  * this problem: *bytes = 0 for an empty problem. Same argument checks as pisa_run_host
  * (no device is touched). The figure is about min(3, chunks) ranges of
  * ceil(B*H / chunks) (batch, head) pairs, each holding its Q, K, V, O and statistics.
  */
-pisa_status_t pisa_run_host_workspace(pisa_shape_t shape, int32_t topk, int32_t order, float route_lambda,
-                                      int32_t chunks, size_t* bytes);
+pisa_status_t pisa_run_host_workspace(pisa_shape_t shape, int32_t topk, int32_t order,
+                                      const pisa_host_options_t* options, size_t* bytes);
 
 /*
  * pisa_run_host -- the whole path on HOST buffers: pisa_block_stats, (with
- * route_lambda > 0) pisa_routing_norms, pisa_select and pisa_attention, as one call.
+ * route_lambda > 0) pisa_routing_norms, pisa_select (pisa_select_grouped with a group
+ * or a candidate count) and pisa_attention, as one call.
  *
  * Section 2 of the explainer, "Hardware implementation": a precompute step, routing,
  * then the fused kernel. Every step is independent across (batch, head) pairs, so the
  * call splits the B*H pairs into `chunks` contiguous ranges and pipelines them through
  * the workspace on three streams: the host-to-device copy of a range, the kernels of
  * the previous one (on `stream`) and the device-to-host copy of the one before overlap.
- * The result is bit for bit that of the four device calls on the whole batch.
+ * The result is bit for bit that of the device calls on the whole batch.
  * Q, K, V: HOST bf16 [B, H, N, d] (page-locked memory lets the copies overlap the
  * kernels; pageable memory works, with less overlap); O: HOST bf16 [B, H, N, d],
- * written; topk, order, scale as in pisa_attention; route_lambda: 0 for plain
- * relevance, > 0 for covariance-aware routing with that weight (order 1 then attends
- * with the per-block S1, order 2 with the routing call's Hbar); chunks >= 1.
+ * written; topk, order, scale as in pisa_attention. With route_lambda > 0, order 1
+ * attends with the per-block S1 and order 2 with the routing call's Hbar.
  * workspace: DEVICE memory owned by the caller, 256-byte aligned, of at least the
  * size pisa_run_host_workspace reports for the same arguments; its contents are
  * scratch. The call BLOCKS until O holds the whole result and nothing runs on the
@@ -202,7 +228,7 @@ pisa_status_t pisa_run_host_workspace(pisa_shape_t shape, int32_t topk, int32_t 
  * rejected with PISA_ERR_INVALID_ARG.
  */
 pisa_status_t pisa_run_host(const void* Q, const void* K, const void* V, pisa_shape_t shape, int32_t topk,
-                            int32_t order, float scale, float route_lambda, int32_t chunks, void* workspace,
+                            int32_t order, float scale, const pisa_host_options_t* options, void* workspace,
                             size_t workspace_bytes, void* O, void* stream);
 
 /*

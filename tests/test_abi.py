@@ -181,9 +181,13 @@ def test_binding_raises_on_missing_library(tmp_path, monkeypatch):
         P.lib()
 
 
-def _ws(L, s=None, topk=2, order=1, lam=0.0, chunks=8):
+def _opts(lam=0.0, chunks=8, group=1, cand=0):
+    return ctypes.byref(P.HostOptions(lam, group, cand, chunks))
+
+
+def _ws(L, s=None, topk=2, order=1, lam=0.0, chunks=8, group=1, cand=0):
     n = ctypes.c_size_t(123)
-    st = L.pisa_run_host_workspace(s or shape(), topk, order, lam, chunks, ctypes.byref(n))
+    st = L.pisa_run_host_workspace(s or shape(), topk, order, _opts(lam, chunks, group, cand), ctypes.byref(n))
     return st, n.value
 
 
@@ -205,11 +209,18 @@ def test_host_workspace_size(L):
     st, n0 = _ws(L, shape(B, H, N, d, b), k, -1, chunks=1)
     assert st == OK and n0 == 4 * up(24 * N * d * 2) + 2 * up(24 * nB * d * 4) + up(24 * nB * k * 4)
     assert _ws(L, shape(N=0)) == (OK, 0)
-    assert _ws(L, chunks=0)[0] == INVALID
+    assert _ws(L, chunks=-1)[0] == INVALID
+    assert _ws(L, chunks=0) == _ws(L, chunks=8)             # 0: the default
     assert _ws(L, lam=-1.0)[0] == INVALID
     assert _ws(L, order=5)[0] == INVALID
     assert _ws(L, topk=9)[0] == INVALID
-    assert L.pisa_run_host_workspace(shape(), 2, 1, 0.0, 8, None) == INVALID
+    assert L.pisa_run_host_workspace(shape(), 2, 1, None, None) == INVALID
+    n = ctypes.c_size_t(0)
+    assert L.pisa_run_host_workspace(shape(), 2, 1, None, ctypes.byref(n)) == OK   # NULL options: defaults
+    assert n.value == _ws(L)[1]
+    assert _ws(L, group=9)[0] == INVALID
+    assert _ws(L, cand=1)[0] == INVALID             # fewer candidates than topk
+    assert _ws(L, group=4, cand=3)[0] == OK
 
 
 def run_host(L, s=None, topk=2, order=1, scale=0.1, lam=0.0, chunks=2, ws=FAKE, nbytes=None, **ptrs):
@@ -217,8 +228,8 @@ def run_host(L, s=None, topk=2, order=1, scale=0.1, lam=0.0, chunks=2, ws=FAKE, 
     p.update(ptrs)
     if nbytes is None:
         nbytes = _ws(L, s, topk, order, lam, chunks)[1]
-    return L.pisa_run_host(vp(p["Q"]), vp(p["K"]), vp(p["V"]), s or shape(), topk, order, scale, lam, chunks,
-                           vp(ws), nbytes, vp(p["O"]), None)
+    return L.pisa_run_host(vp(p["Q"]), vp(p["K"]), vp(p["V"]), s or shape(), topk, order, scale,
+                           _opts(lam, chunks), vp(ws), nbytes, vp(p["O"]), None)
 
 
 def test_host_entry_arguments(L):
@@ -230,7 +241,24 @@ def test_host_entry_arguments(L):
     assert run_host(L, nbytes=100) == INVALID
     assert b"needed" in L.pisa_last_error()
     assert run_host(L, scale=0.0) == INVALID
-    assert run_host(L, chunks=0) == INVALID
+    assert run_host(L, chunks=-2) == INVALID
     assert run_host(L, s=shape(B=0), Q=0, K=0, V=0, O=0, ws=0, nbytes=0) == OK
     _no_device()
     _passes_validation(run_host(L, Q=MISALIGNED), L)     # host buffers need no alignment
+
+
+def sel_grouped(L, s=None, Q=FAKE, kbar=FAKE, topk=2, group=2, cand=3, idx=FAKE, route=0, lam=0.0):
+    return L.pisa_select_grouped(vp(Q), vp(kbar), vp(route), lam, s or shape(), topk, group, cand, vp(idx), None)
+
+
+def test_grouped_select_arguments(L):
+    assert sel_grouped(L, group=0) == INVALID
+    assert sel_grouped(L, group=9) == INVALID
+    assert sel_grouped(L, cand=1) == INVALID        # fewer candidates than topk
+    assert sel_grouped(L, cand=5) == INVALID        # more candidates than nB = 4
+    assert sel_grouped(L, idx=MISALIGNED) == INVALID
+    assert sel_grouped(L, s=shape(d=96)) == UNSUPPORTED
+    assert sel_grouped(L, s=shape(N=0), Q=0, kbar=0, idx=0) == OK
+    _no_device()
+    _passes_validation(sel_grouped(L), L)
+    _passes_validation(sel_grouped(L, group=8, cand=2), L)

@@ -214,15 +214,18 @@ def test_device_error_word_is_shared_per_device():
     P.device_error()          # taken by the first reader: nothing left
 
 
-@pytest.mark.parametrize("order,lam", [(1, 0.0), (2, 0.0), (-1, 0.0), (0, 0.0), (2, 0.02), (1, 0.02)])
-def test_host_entry_point_matches_device(order, lam):
+@pytest.mark.parametrize("order,lam,group,cand", [(1, 0.0, 1, 0), (2, 0.0, 1, 0), (-1, 0.0, 1, 0), (0, 0.0, 1, 0),
+                                                  (2, 0.02, 1, 0), (1, 0.02, 1, 0), (2, 0.0, 4, 32), (1, 0.02, 2, 16)])
+def test_host_entry_point_matches_device(order, lam, group, cand):
     """pisa_run_host (host buffers in and out, through the C ABI) gives the bits of the
-    device calls on the whole batch, for every order, with and without routing."""
+    device calls on the whole batch, for every order, with and without routing and with
+    grouped selection."""
     wl = W.get("image").with_(B=1, H=2)
     q, k, v = W.make_inputs(wl)
     hq, hk, hv = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in (q, k, v))
-    Oh = P.pisa_host(hq, hk, hv, wl.block, wl.topk, order, wl.scale, route_lambda=lam)
-    Od, _ = P.pisa(hq.cuda(), hk.cuda(), hv.cuda(), wl.block, wl.topk, order, wl.scale, route_lambda=lam)
+    Oh = P.pisa_host(hq, hk, hv, wl.block, wl.topk, order, wl.scale, route_lambda=lam, group=group, candidates=cand)
+    Od, _ = P.pisa(hq.cuda(), hk.cuda(), hv.cuda(), wl.block, wl.topk, order, wl.scale, route_lambda=lam,
+                   group=group, candidates=cand or None)
     assert torch.equal(Oh.view(torch.int16), Od.cpu().view(torch.int16))
 
 
@@ -251,6 +254,6 @@ def test_host_entry_point_rejects_device_buffers():
     n = P.host_workspace_bytes(s, wl.topk, wl.order)
     ws = torch.empty(n, dtype=torch.uint8, device="cuda")
     O = torch.empty_like(q)
-    st = P.lib().pisa_run_host(P._ptr(q), P._ptr(k), P._ptr(v), s, wl.topk, wl.order, wl.scale, 0.0, 2,
+    st = P.lib().pisa_run_host(P._ptr(q), P._ptr(k), P._ptr(v), s, wl.topk, wl.order, wl.scale, None,
                                P._ptr(ws), n, P._ptr(O), None)
     assert st == 1 and b"device memory" in P.lib().pisa_last_error()

@@ -60,6 +60,9 @@ class Workload:
     grid: tuple = ()     # token grid for the smooth generators
     seed: int = 0
     route_lambda: float = 0.0   # covariance-aware routing weight (0: plain relevance)
+    select_group: int = 1       # query blocks per proxy query (1: every block is its own)
+    select_cand: int = 0        # proxy candidate-list length (0: every key block)
+    reuse_idx: bool = False     # the step reuses the indices of an earlier call
 
     @property
     def nB(self) -> int:
@@ -94,6 +97,12 @@ WORKLOADS["long_hybrid"] = WORKLOADS["long"].with_(name="long_hybrid", order=2)
 # the hybrid order with covariance-aware routing; the weight puts lambda * std(M_j)
 # at about half the spread between a row's best and k-th pooled score
 WORKLOADS["video_routed"] = WORKLOADS["video"].with_(name="video_routed", order=2, route_lambda=0.015)
+# selection amortisation at the hybrid order: one proxy per 4 query blocks keeping 2k
+# candidates refined per member (grouped proxies), and indices reused from an earlier
+# call with no selection in the step (index reuse across layers)
+WORKLOADS["video_grouped"] = WORKLOADS["video"].with_(name="video_grouped", order=2, select_group=4,
+                                                      select_cand=128)
+WORKLOADS["video_reuse"] = WORKLOADS["video"].with_(name="video_reuse", order=2, reuse_idx=True)
 
 
 def get(name: str) -> Workload:
