@@ -8,8 +8,9 @@
 // 2 hybrid order with the global correction (x_t Hbar) sum_U alpha_{t,j}.
 // One CTA per (query block, head), one thread per query row; blocks are visited
 // in ascending order and the accumulator is rescaled whenever the running row
-// maximum grows. Used to cross-check the fused kernel on sizes where the CPU
-// oracle is slow, and as the path for shapes the fused kernel does not cover.
+// maximum grows. It is reached only through its own entry point
+// (pisa_attention_simt): an independent GPU cross-check of the fused kernel on
+// sizes where the CPU oracle is slow. pisa_attention never routes to it.
 #pragma once
 
 #include "common.cuh"

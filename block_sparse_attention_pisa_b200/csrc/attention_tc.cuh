@@ -173,25 +173,6 @@ __device__ __forceinline__ uint32_t hmul2_bf16(uint32_t a, uint32_t b) {
   return *reinterpret_cast<uint32_t*>(&z);
 }
 
-// bounded wait that ignores the abort flag: used only to drain copies / MMAs
-// already in flight before the CTA releases its shared and tensor memory
-__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitCycles) {
-      flag_error(kErrTimeout);
-      return;
-    }
-  }
-}
-
-// one arrival per warp: every lane has finished its part (its tensor-memory stores
-// waited for, its shared-memory writes fenced) before lane 0 arrives
-__device__ __forceinline__ void warp_arrive(uint32_t bar) {
-  __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-}
-
 // named barrier of the two warps of one TMEM lane quarter (64 threads); returns the
 // AND of `ok` over them, so that both warps of a pair take the same exits
 __device__ __forceinline__ bool pair_sync_and(int id, bool ok) {

@@ -15,6 +15,7 @@
 #include "routing.cuh"
 #include "attention_simt.cuh"
 #include "attention_tc.cuh"
+#include "stats_tc.cuh"
 #include "host_pipeline.cuh"
 
 using pisa::bf16;
@@ -142,18 +143,47 @@ pisa_status_t launch_stats_mode(const pisa_shape_t& s, const bf16* K, const bf16
   return check_launch("stats_pipe_kernel");
 }
 
+pisa_status_t make_map(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box1);
+
+// d = 128, orders 1 and 2: the tensor-core statistics kernel (persistent, one CTA per SM)
+template <int BLK, int MODE>
+pisa_status_t launch_stats_tc(const pisa_shape_t& s, const bf16* K, const bf16* V, float* kbar, float* S0, bf16* S1,
+                              float* Hbar, int sms, cudaStream_t st) {
+  using C = pisa::StatsTcCfg<BLK, MODE>;
+  const int nB = int(num_blocks(s));
+  const uint64_t BH = uint64_t(s.B) * s.H;
+  CUtensorMap mK, mV, mS;
+  PISA_TRY(make_map(&mK, K, 128, uint64_t(s.N), BH, BLK));
+  PISA_TRY(make_map(&mV, V, 128, uint64_t(s.N), BH, BLK));
+  if (MODE == pisa::kStatsS1) PISA_TRY(make_map(&mS, S1, 128, 128, BH * nB, 128));
+  else mS = mK;  // never used in Hbar mode
+  auto k = pisa::stats_tc_kernel<BLK, MODE>;
+  PISA_TRY(set_smem(k, C::SMEM));
+  const int uph = (nB + C::UNIT - 1) / C::UNIT;
+  const int64_t total = int64_t(BH) * uph;
+  if (total > (int64_t(1) << 30)) return fail(PISA_ERR_UNSUPPORTED, "too many statistics units");
+  const int grid = int(total < sms ? total : sms);
+  k<<<grid, C::kThreads, C::SMEM, st>>>(mK, mV, mS, s.N, nB, uph, int(total), kbar, S0, Hbar);
+  return check_launch("stats_tc_kernel");
+}
+
 template <int D, int BLK>
 pisa_status_t launch_stats(const pisa_shape_t& s, const bf16* K, const bf16* V, int order, float* kbar,
-                           float* S0, void* S1, cudaStream_t st) {
+                           float* S0, void* S1, int sms, cudaStream_t st) {
   if (order == PISA_ORDER_HYBRID) {
     // Hbar is accumulated with atomics: zero it first, on the same stream
     const size_t bytes = size_t(s.B) * s.H * D * D * sizeof(float);
     cudaError_t e = cudaMemsetAsync(S1, 0, bytes, st);
     if (e != cudaSuccess) return fail(PISA_ERR_CUDA, "cudaMemsetAsync(Hbar): %s", cudaGetErrorString(e));
+    if (D == 128)
+      return launch_stats_tc<BLK, pisa::kStatsHbar>(s, K, V, kbar, S0, nullptr, static_cast<float*>(S1), sms, st);
     return launch_stats_mode<D, BLK, pisa::kStatsHbar>(s, K, V, kbar, S0, nullptr, static_cast<float*>(S1), st);
   }
-  if (order == PISA_ORDER_FIRST)
+  if (order == PISA_ORDER_FIRST) {
+    if (D == 128)
+      return launch_stats_tc<BLK, pisa::kStatsS1>(s, K, V, kbar, S0, static_cast<bf16*>(S1), nullptr, sms, st);
     return launch_stats_mode<D, BLK, pisa::kStatsS1>(s, K, V, kbar, S0, static_cast<bf16*>(S1), nullptr, st);
+  }
   return launch_stats_mode<D, BLK, pisa::kStatsSums>(s, K, V, kbar, S0, nullptr, nullptr, st);
 }
 
@@ -336,10 +366,10 @@ pisa_status_t pisa_block_stats(const void* K, const void* V, pisa_shape_t shape,
   auto st = static_cast<cudaStream_t>(stream);
   auto k = static_cast<const bf16*>(K);
   auto v = static_cast<const bf16*>(V);
-  if (shape.d == 128 && shape.block == 64) return launch_stats<128, 64>(shape, k, v, order, kbar, S0, S1, st);
-  if (shape.d == 128 && shape.block == 128) return launch_stats<128, 128>(shape, k, v, order, kbar, S0, S1, st);
-  if (shape.d == 64 && shape.block == 64) return launch_stats<64, 64>(shape, k, v, order, kbar, S0, S1, st);
-  return launch_stats<64, 128>(shape, k, v, order, kbar, S0, S1, st);
+  if (shape.d == 128 && shape.block == 64) return launch_stats<128, 64>(shape, k, v, order, kbar, S0, S1, sms, st);
+  if (shape.d == 128 && shape.block == 128) return launch_stats<128, 128>(shape, k, v, order, kbar, S0, S1, sms, st);
+  if (shape.d == 64 && shape.block == 64) return launch_stats<64, 64>(shape, k, v, order, kbar, S0, S1, sms, st);
+  return launch_stats<64, 128>(shape, k, v, order, kbar, S0, S1, sms, st);
 }
 
 pisa_status_t pisa_select_grouped(const void* Q, const float* kbar, const float* route, float lambda,

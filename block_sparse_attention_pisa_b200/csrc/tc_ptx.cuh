@@ -80,6 +80,25 @@ __device__ __forceinline__ bool wait_poll(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// bounded wait that ignores the abort flag: used only to drain copies / MMAs
+// already in flight before the CTA releases its shared and tensor memory
+__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitCycles) {
+      flag_error(kErrTimeout);
+      return;
+    }
+  }
+}
+
+// one arrival per warp: every lane has finished its part (its tensor-memory stores
+// waited for, its shared-memory writes fenced) before lane 0 arrives
+__device__ __forceinline__ void warp_arrive(uint32_t bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
                                             int c2) {
