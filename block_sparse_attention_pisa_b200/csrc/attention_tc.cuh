@@ -23,16 +23,22 @@
 //   warps 2-3   build the block lists, then convert fp32 kbar / S0 chunks of 32
 //               blocks into bf16 swizzled shared-memory operands;
 //   warps 4-11  two threads per query row (= TMEM lane): warps w and w + 4 share a
-//               lane quarter. In the exact stage each takes half of the row's score
+//               lane quarter. Exact stage at b = 64: two independent groups, warps 4-7
+//               taking the even exact blocks and warps 8-11 the odd ones, each thread
+//               all of its row's scores of its block, with its own accumulator O_g,
+//               running maximum and denominator; one group's exponentials overlap the
+//               other's hand-offs, and the two accumulators are merged once at the end.
+//               Exact stage at b = 128: each thread takes half of the row's score
 //               columns and half of O's columns, and a pair agrees on its running
 //               maximum through shared memory at one named barrier per block. The
 //               approximate stage runs on warps 4-7 alone with full-width operands
 //               (its hand-offs are short; fewer warps to wait for pays more there).
 // Tensor memory (512 columns): O accumulator (D), the tile's queries Q (D/2; the A
-// operand of Q K^T and Q Kbar^T), then either a ring of exact score buffers S
-// (P overwrites its own S) or, in the approximate stage, two pooled-score buffers
-// Sbar (the bf16 alpha operand overwrites its own Sbar) and four A_j =
-// (alpha_j * scale) (.) q operand slots used in pairs.
+// operand of Q K^T and Q Kbar^T), then, in the exact stage, the second group's
+// accumulator O_1 (D, b = 64 only) and a ring of exact score buffers S (P overwrites
+// its own S), or, in the approximate stage, two pooled-score buffers Sbar (the bf16
+// alpha operand overwrites its own Sbar) and four A_j = (alpha_j * scale) (.) q
+// operand slots used in pairs.
 //
 // Exact stage, per block j in the union of the tile's selections:
 //   S = Q K_j^T (TS-MMA), P = exp(x.k - m) (zero for rows whose query block
@@ -58,7 +64,8 @@
 // tensor-pipe time: per exact block once for K_j and V_j (one barrier) and once
 // for P; per pair of approximated blocks once (the row threads signal a pair only
 // after writing both A operands and seeing both S1 tiles land). The exact scores
-// run NSB - 2 blocks ahead of the softmax (three at d = 128, b = 64). Hand-off
+// run NSB - 1 blocks ahead of the softmax with two groups (two at d = 128, b = 64),
+// NSB - 2 otherwise. Hand-off
 // barriers count one arrival per warp. Every wait is bounded by clock64; on timeout
 // a CTA raises the device error word, drains its copies and MMAs, frees TMEM and
 // exits. The two warps of a row pair leave together: their named barriers AND-reduce
@@ -101,7 +108,13 @@ struct TcCfg {
   // exact score buffers. At d = 128 as many as the columns after Q hold (the approximate
   // stage's operand slots reuse the same columns later): five at b = 64 measured 1-2%
   // faster than four. At d = 64 a deeper ring measured slower (b = 128: 3.20 vs 3.14 ms).
-  static constexpr int NSB = (D == 128) ? (512 - (D + D / 2)) / BLK : ((BLK == 64) ? 4 : 2);
+  // At b = 64 the exact stage runs as two independent groups of row warps (warps 4-7 take
+  // the even exact blocks, warps 8-11 the odd ones), each with its own accumulator O_g,
+  // running maximum and denominator; the two are merged before the approximate stage.
+  static constexpr bool GROUPS = (BLK == 64);
+  static constexpr int O1_COL = D + D / 2;              // second exact accumulator (GROUPS)
+  static constexpr int SX_COL = GROUPS ? O1_COL + D : D + D / 2;  // exact score buffers
+  static constexpr int NSB = GROUPS ? (512 - SX_COL) / BLK : ((D == 128) ? (512 - (D + D / 2)) / BLK : 2);
   static constexpr int MAXB = 2048;
   static constexpr int MAXC = MAXB / CHUNK;
   // tensor-memory columns
@@ -111,7 +124,8 @@ struct TcCfg {
   static constexpr int A_COL0 = R_COL + 2 * CHUNK;
   static constexpr int A_COLS = D / 2;
   static constexpr int TMEM_COLS = 512;
-  static_assert(R_COL + NSB * BLK <= TMEM_COLS, "exact score buffers exceed TMEM");
+  static_assert(SX_COL + NSB * BLK <= TMEM_COLS, "exact score buffers exceed TMEM");
+  static_assert(!GROUPS || NSB >= 3, "two groups need three score buffers");
   static_assert(A_COL0 + NA * A_COLS <= TMEM_COLS, "operand ring exceeds TMEM");
   static_assert(STAGE >= BLK * D * 2 && STAGE >= D * D * 2, "stage too small");
   // barriers
@@ -133,7 +147,8 @@ struct TcCfg {
   static constexpr int B_XD = B_ODONE + 1;        //       exact stage done, ring idle (commit; hybrid)
   static constexpr int B_HF = B_XD + 1;           //       Hbar operand converted (4 warps; hybrid)
   static constexpr int B_AH = B_HF + 1;           //       A_H = s x written (4 warps; hybrid)
-  static constexpr int NBARS = B_AH + 1;
+  static constexpr int B_MG = B_AH + 1;           //       group accumulators merged (8 row warps; GROUPS)
+  static constexpr int NBARS = B_MG + 1;
   // shared memory (offsets from a 1024-byte aligned base)
   static constexpr int OFF_RING = 0;
   static constexpr int OFF_CV = OFF_RING + NS * STAGE;
@@ -242,7 +257,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     for (int s = 0; s < C::NTF; ++s) mbar_init(BAR(C::B_TF + s), 1);
     for (int s = 0; s < C::NSB; ++s) {
       mbar_init(BAR(C::B_SF + s), 1);
-      mbar_init(BAR(C::B_PF + s), kRowWarps);
+      mbar_init(BAR(C::B_PF + s), C::GROUPS ? kRowWarps / 2 : kRowWarps);  // a group, or both halves
       mbar_init(BAR(C::B_PV + s), 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -260,6 +275,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     mbar_init(BAR(C::B_XD), 1);
     mbar_init(BAR(C::B_HF), 4);
     mbar_init(BAR(C::B_AH), kApproxWarps);
+    mbar_init(BAR(C::B_MG), kRowWarps);
     misc[1] = 0;
     mbar_init_fence();
   }
@@ -397,6 +413,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       constexpr uint32_t idSB = idesc_bf16(128, C::CHUNK, false);  // Sbar = Q Kbar^T
       constexpr uint32_t idO = idesc_bf16(128, D, true);           // O += {P V, alpha S0, A S1}
       uint32_t o_acc = 0;
+      uint32_t g_acc[2] = {0u, 0u};  // GROUPS: each group's accumulator holds a product
       bool ok = wait_poll(BAR(C::B_Q), 0, abort_flag);
       tc_fence_after();
       auto pv = [&](int e) -> bool {
@@ -405,12 +422,24 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         tc_fence_after();
         const int sv = (C::TPB * e + C::TPB - 1) % C::NS;
         const uint32_t vb = base_u + C::OFF_RING + sv * C::STAGE + (C::KV_PACKED ? BLK * D * 2 : 0);
-        // P of keys [16k, 16k + 16): half (k / (BLK/32)) of the row packed it at the
-        // start of its own score columns
+        if constexpr (C::GROUPS) {
+          // P of keys [16k, 16k + 16) at the start of block e's score columns; O of the
+          // block's group
+          const uint32_t oc = (e & 1) ? C::O1_COL : C::O_COL;
 #pragma unroll
-        for (int k = 0; k < BLK / 16; ++k)
-          umma_ts(tmem + C::O_COL, tmem + C::R_COL + sb * BLK + (k / (BLK / 32)) * (BLK / 2) + (k % (BLK / 32)) * 8,
-                  sdesc_sw128(vb + k * 2048, BLK * 128, 1024), idO, (o_acc | uint32_t(k)) ? 1u : 0u);
+          for (int k = 0; k < BLK / 16; ++k)
+            umma_ts(tmem + oc, tmem + C::SX_COL + sb * BLK + k * 8, sdesc_sw128(vb + k * 2048, BLK * 128, 1024), idO,
+                    (g_acc[e & 1] | uint32_t(k)) ? 1u : 0u);
+          g_acc[e & 1] = 1;
+        } else {
+          // P of keys [16k, 16k + 16): half (k / (BLK/32)) of the row packed it at the
+          // start of its own score columns
+#pragma unroll
+          for (int k = 0; k < BLK / 16; ++k)
+            umma_ts(tmem + C::O_COL,
+                    tmem + C::SX_COL + sb * BLK + (k / (BLK / 32)) * (BLK / 2) + (k % (BLK / 32)) * 8,
+                    sdesc_sw128(vb + k * 2048, BLK * 128, 1024), idO, (o_acc | uint32_t(k)) ? 1u : 0u);
+        }
         o_acc = 1;
         umma_commit(BAR(C::B_SE + sv));
         umma_commit(BAR(C::B_PV + sb));
@@ -426,14 +455,15 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         const uint32_t kb = base_u + C::OFF_RING + sk * C::STAGE;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          umma_ts(tmem + C::R_COL + sb * BLK, tmem + C::Q_COL + k * 8,
+          umma_ts(tmem + C::SX_COL + sb * BLK, tmem + C::Q_COL + k * 8,
                   sdesc_sw128(kb + (k >> 2) * (BLK * 128) + (k & 3) * 32, 16, 1024), idS, k ? 1u : 0u);
         if (!C::KV_PACKED) umma_commit(BAR(C::B_SE + sk));  // a packed stage is released after P V
         umma_commit(BAR(C::B_SF + sb));
         return true;
       };
       // the scores run kLook blocks ahead of the row threads' softmax
-      constexpr int kLook = C::NSB >= 3 ? C::NSB - 2 : 1;
+      // (two groups: one block further, since the two groups' blocks alternate)
+      constexpr int kLook = C::GROUPS ? C::NSB - 1 : (C::NSB >= 3 ? C::NSB - 2 : 1);
       for (int e = 0; e < kLook && e < n_exact && ok; ++e) ok = qk(e);
       for (int e = 0; e < n_exact && ok; ++e) {
         ok = pv(e);
@@ -443,8 +473,12 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       if (hybrid) umma_commit(BAR(C::B_XD));
 
       if (ok && n_active > 0) {
-        // the pooled-score and operand columns reuse the exact score buffers
-        ok = wait_poll(BAR(C::B_PV + (n_exact - 1) % C::NSB), ((n_exact - 1) / C::NSB) & 1, abort_flag);
+        // the pooled-score and operand columns reuse the exact score buffers (and, with two
+        // groups, the second accumulator, which the row threads have merged first)
+        if constexpr (C::GROUPS)
+          ok = wait_poll(BAR(C::B_MG), 0, abort_flag);
+        else
+          ok = wait_poll(BAR(C::B_PV + (n_exact - 1) % C::NSB), ((n_exact - 1) / C::NSB) & 1, abort_flag);
         auto sbar = [&](int ac) -> bool {
           const int b = ac & 1;
           if (!wait_poll(BAR(C::B_CVF + b), (ac >> 1) & 1, abort_flag)) return false;
@@ -618,80 +652,188 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     float s_alpha = 0.f;  // hybrid order: this half's sum of alpha weights (same frame as l)
 
     // ------------------------------------------------ exact stage
-    for (int e = 0; e < n_exact; ++e) {
-      const int j = exact_list[e], sb = e % C::NSB;
-      const bool sel = (mymask[j >> 5] >> (j & 31)) & 1u;  // uniform per warp
-      const int nmine = min(HK, N - j * BLK - hf * HK);     // this half's real keys (may be <= 0)
-      if (ok) ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SF + sb), (e / C::NSB) & 1, abort_flag));
-      uint32_t s[HK];
-      const uint32_t sa = tmem + lrow + C::R_COL + sb * BLK + hf * HK;
-      float pm = -INFINITY;
-      if (ok) {
-        tc_fence_after();
-#pragma unroll
-        for (int ch = 0; ch < HK / 16; ++ch) tmem_ld16(sa + ch * 16, *reinterpret_cast<uint32_t(*)[16]>(&s[ch * 16]));
-#pragma unroll
-        for (int ch = 0; ch < HK / 16; ++ch) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&s[ch * 16]));
-        if (nmine < HK) {  // ragged last block: keys past N take no weight
-#pragma unroll
-          for (int k = 0; k < HK; ++k)
-            if (k >= nmine) s[k] = __float_as_uint(-INFINITY);
-        }
+    if constexpr (C::GROUPS) {
+      // Group hf takes the exact blocks e = hf, hf + 2, ...: all BLK scores of its row,
+      // its own accumulator O_hf, running maximum m and denominator l. No exchange with the
+      // other group per block; one merge at the end.
+      const uint32_t oc = hf ? C::O1_COL : C::O_COL;
+      for (int e = hf; e < n_exact; e += 2) {
+        const int j = exact_list[e], sb = e % C::NSB;
+        const bool sel = (mymask[j >> 5] >> (j & 31)) & 1u;  // uniform per warp
+        const int nreal = min(BLK, N - j * BLK);              // real keys of the block
+        ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SF + sb), (e / C::NSB) & 1, abort_flag));
+        if (!ok) break;
+        const uint32_t sa = tmem + lrow + C::SX_COL + sb * BLK;
+        uint32_t pk[BLK / 2];
+        float rsp[4] = {0.f, 0.f, 0.f, 0.f};
         if (sel) {
-          // raw-score maximum (the positive scale commutes with it); independent partial
-          // maxima, because one warp per scheduler cannot hide a serial chain
+          tc_fence_after();
+          uint32_t sc[BLK];
+#pragma unroll
+          for (int ch = 0; ch < BLK / 16; ++ch)
+            tmem_ld16(sa + ch * 16, *reinterpret_cast<uint32_t(*)[16]>(&sc[ch * 16]));
+#pragma unroll
+          for (int ch = 0; ch < BLK / 16; ++ch) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&sc[ch * 16]));
+          if (nreal < BLK) {  // ragged last block: keys past N take no weight
+#pragma unroll
+            for (int k = 0; k < BLK; ++k)
+              if (k >= nreal) sc[k] = __float_as_uint(-INFINITY);
+          }
           float mxp[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) mxp[i] = -INFINITY;
 #pragma unroll
-          for (int k = 0; k < HK; ++k) mxp[k & 7] = fmaxf(mxp[k & 7], __uint_as_float(s[k]));
-          pm = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
-                     fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+          for (int k = 0; k < BLK; ++k) mxp[k & 7] = fmaxf(mxp[k & 7], __uint_as_float(sc[k]));
+          const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                                 fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]))) * sl2;
+          const bool grow_max = mx > m + 8.f;
+          const bool need_o = grow_max && m != -INFINITY;
+          if (__any_sync(0xffffffffu, need_o)) {
+            // the group's previous product must be in O_hf before it is rescaled
+            if (e >= 2)
+              ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_PV + (e - 2) % C::NSB), ((e - 2) / C::NSB) & 1,
+                                                        abort_flag));
+            if (ok) {
+              tc_fence_after();
+              const float f = need_o ? ex2(m - mx) : 1.f;
+              rescale_row<D>(tmem + lrow + oc, f);
+              l *= f;
+            }
+          }
+          if (!ok) break;
+          if (grow_max) m = mx;
+          const float negm = -m;
+#pragma unroll
+          for (int i = 0; i < BLK / 2; ++i) {
+            const float p0 = ex2(fmaf(__uint_as_float(sc[2 * i]), sl2, negm));
+            const float p1 = ex2(fmaf(__uint_as_float(sc[2 * i + 1]), sl2, negm));
+            rsp[i & 3] += p0 + p1;
+            pk[i] = pack_bf16x2_int(p0, p1);
+          }
+        } else {
+          // rows whose query block did not select j take no exact weight
+#pragma unroll
+          for (int i = 0; i < BLK / 2; ++i) pk[i] = 0u;
         }
+#pragma unroll
+        for (int ch = 0; ch < BLK / 32; ++ch)
+          tmem_st16(sa + ch * 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[ch * 16]));
+        l += (rsp[0] + rsp[1]) + (rsp[2] + rsp[3]);
+        tmem_wait_st();
+        tc_fence_before();
+        warp_arrive(BAR(C::B_PF + sb));
       }
-      xmax[((e & 1) * 2 + hf) * 128 + r] = pm;
+      // merge: O_0 <- f_0 O_0 + f_1 O_1 against the common maximum, each group over its own
+      // half of the columns, once every product of both groups is in
+      xmax[hf * 128 + r] = m;
+      xmax[256 + hf * 128 + r] = l;
       ok = pair_sync_and(pair_id, ok);
-      if (!ok) break;
-      const float mx = fmaxf(pm, xmax[((e & 1) * 2 + (hf ^ 1)) * 128 + r]) * sl2;
-      const bool grow_max = mx > m + 8.f;          // false for rows that did not select j
-      const bool need_o = grow_max && m != -INFINITY;
-      if (__any_sync(0xffffffffu, need_o)) {
-        if (e >= 1)
-          ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_PV + (e - 1) % C::NSB), ((e - 1) / C::NSB) & 1,
-                                                    abort_flag));
+      const float m_o = xmax[(hf ^ 1) * 128 + r], l_o = xmax[256 + (hf ^ 1) * 128 + r];
+      const float mm = fmaxf(m, m_o);
+      const float m0 = hf ? m_o : m, m1 = hf ? m : m_o;
+      const float f0 = m0 == -INFINITY ? 0.f : ex2(m0 - mm);
+      const float f1 = m1 == -INFINITY ? 0.f : ex2(m1 - mm);
+      if (ok && n_exact >= 2) {  // with a single exact block O_1 holds no product
+        ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_OSYNC), 0, abort_flag));
         if (ok) {
           tc_fence_after();
-          const float f = need_o ? ex2(m - mx) : 1.f;
-          rescale_row<HD>(tmem + lrow + C::O_COL + hf * HD, f);
-          l *= f;
+#pragma unroll 1
+          for (int ch = 0; ch < (D / 2) / 16; ++ch) {
+            uint32_t a[16], b[16];
+            tmem_ld16(tmem + lrow + C::O_COL + hf * (D / 2) + ch * 16, a);
+            tmem_ld16(tmem + lrow + C::O1_COL + hf * (D / 2) + ch * 16, b);
+            tmem_wait_ld(a);
+            tmem_wait_ld(b);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              a[i] = __float_as_uint(fmaf(__uint_as_float(a[i]), f0, __uint_as_float(b[i]) * f1));
+            tmem_st16(tmem + lrow + C::O_COL + hf * (D / 2) + ch * 16, a);
+          }
+          tmem_wait_st();
         }
       }
-      if (grow_max) m = mx;
-      float rsp[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[HK / 2];
-      if (sel) {
-        const float negm = -m;
-#pragma unroll
-        for (int i = 0; i < HK / 2; ++i) {
-          const float p0 = ex2(fmaf(__uint_as_float(s[2 * i]), sl2, negm));
-          const float p1 = ex2(fmaf(__uint_as_float(s[2 * i + 1]), sl2, negm));
-          rsp[i & 3] += p0 + p1;
-          pk[i] = pack_bf16x2_int(p0, p1);
-        }
-      } else {
-        // rows whose query block did not select j take no exact weight (m may still be
-        // -inf for them, so no exponential is evaluated)
-#pragma unroll
-        for (int i = 0; i < HK / 2; ++i) pk[i] = 0u;
-      }
-#pragma unroll
-      for (int ch = 0; ch < HK / 32; ++ch) tmem_st16(sa + ch * 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[ch * 16]));
-      l += (rsp[0] + rsp[1]) + (rsp[2] + rsp[3]);
-      tmem_wait_st();
       tc_fence_before();
-      warp_arrive(BAR(C::B_PF + sb));
+      warp_arrive(BAR(C::B_MG));
+      // from here on: one accumulator O_0 with maximum mm; the whole denominator with half 0
+      l = hf ? 0.f : (hf ? l_o : l) * f0 + (hf ? l : l_o) * f1;
+      m = mm;
+      ok = pair_sync_and(pair_id, ok);
+    } else {
+      for (int e = 0; e < n_exact; ++e) {
+        const int j = exact_list[e], sb = e % C::NSB;
+        const bool sel = (mymask[j >> 5] >> (j & 31)) & 1u;  // uniform per warp
+        const int nmine = min(HK, N - j * BLK - hf * HK);     // this half's real keys (may be <= 0)
+        if (ok) ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SF + sb), (e / C::NSB) & 1, abort_flag));
+        uint32_t s[HK];
+        const uint32_t sa = tmem + lrow + C::SX_COL + sb * BLK + hf * HK;
+        float pm = -INFINITY;
+        if (ok) {
+          tc_fence_after();
+  #pragma unroll
+          for (int ch = 0; ch < HK / 16; ++ch) tmem_ld16(sa + ch * 16, *reinterpret_cast<uint32_t(*)[16]>(&s[ch * 16]));
+  #pragma unroll
+          for (int ch = 0; ch < HK / 16; ++ch) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[16]>(&s[ch * 16]));
+          if (nmine < HK) {  // ragged last block: keys past N take no weight
+  #pragma unroll
+            for (int k = 0; k < HK; ++k)
+              if (k >= nmine) s[k] = __float_as_uint(-INFINITY);
+          }
+          if (sel) {
+            // raw-score maximum (the positive scale commutes with it); independent partial
+            // maxima, because one warp per scheduler cannot hide a serial chain
+            float mxp[8];
+  #pragma unroll
+            for (int i = 0; i < 8; ++i) mxp[i] = -INFINITY;
+  #pragma unroll
+            for (int k = 0; k < HK; ++k) mxp[k & 7] = fmaxf(mxp[k & 7], __uint_as_float(s[k]));
+            pm = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                       fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+          }
+        }
+        xmax[((e & 1) * 2 + hf) * 128 + r] = pm;
+        ok = pair_sync_and(pair_id, ok);
+        if (!ok) break;
+        const float mx = fmaxf(pm, xmax[((e & 1) * 2 + (hf ^ 1)) * 128 + r]) * sl2;
+        const bool grow_max = mx > m + 8.f;          // false for rows that did not select j
+        const bool need_o = grow_max && m != -INFINITY;
+        if (__any_sync(0xffffffffu, need_o)) {
+          if (e >= 1)
+            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_PV + (e - 1) % C::NSB), ((e - 1) / C::NSB) & 1,
+                                                      abort_flag));
+          if (ok) {
+            tc_fence_after();
+            const float f = need_o ? ex2(m - mx) : 1.f;
+            rescale_row<HD>(tmem + lrow + C::O_COL + hf * HD, f);
+            l *= f;
+          }
+        }
+        if (grow_max) m = mx;
+        float rsp[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t pk[HK / 2];
+        if (sel) {
+          const float negm = -m;
+  #pragma unroll
+          for (int i = 0; i < HK / 2; ++i) {
+            const float p0 = ex2(fmaf(__uint_as_float(s[2 * i]), sl2, negm));
+            const float p1 = ex2(fmaf(__uint_as_float(s[2 * i + 1]), sl2, negm));
+            rsp[i & 3] += p0 + p1;
+            pk[i] = pack_bf16x2_int(p0, p1);
+          }
+        } else {
+          // rows whose query block did not select j take no exact weight (m may still be
+          // -inf for them, so no exponential is evaluated)
+  #pragma unroll
+          for (int i = 0; i < HK / 2; ++i) pk[i] = 0u;
+        }
+  #pragma unroll
+        for (int ch = 0; ch < HK / 32; ++ch) tmem_st16(sa + ch * 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[ch * 16]));
+        l += (rsp[0] + rsp[1]) + (rsp[2] + rsp[3]);
+        tmem_wait_st();
+        tc_fence_before();
+        warp_arrive(BAR(C::B_PF + sb));
+      }
+      ok = pair_sync_and(pair_id, ok);
     }
-    ok = pair_sync_and(pair_id, ok);
 
     // ------------------------------------------------ approximate stage
     // Half 0 of each row runs it alone on full-width operands (O, alpha, A_j, A_H): the
