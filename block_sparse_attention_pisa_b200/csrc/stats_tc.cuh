@@ -263,11 +263,14 @@ stats_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     const uint32_t lrow = uint32_t(quarter * 32) << 16;
     const int a = et;
     bool ok = true;
-    for (int u = 0; u < nunits && ok; ++u) {
+    // S1 mode: the four warps meet at two named barriers per unit; a warp whose wait ran
+    // out keeps meeting them (skipping the work), so that no warp is left waiting
+    for (int u = 0; u < nunits && (ok || MODE != 2); ++u) {
       const int ab = u & 1;
-      ok = __all_sync(0xffffffffu, wait_bounded(SBAR(C::B_AFULL + ab), (u >> 1) & 1, abort_flag)) &&
-           __all_sync(0xffffffffu, wait_bounded(SBAR(C::B_SFULL + ab), (u >> 1) & 1, abort_flag));
-      if (!ok) break;
+      if (ok)
+        ok = __all_sync(0xffffffffu, wait_bounded(SBAR(C::B_AFULL + ab), (u >> 1) & 1, abort_flag)) &&
+             __all_sync(0xffffffffu, wait_bounded(SBAR(C::B_SFULL + ab), (u >> 1) & 1, abort_flag));
+      if (MODE == 2 && !ok) break;
       tc_fence_after();
       int bh, j;
       block_of(u * C::UNIT, &bh, &j);
@@ -279,7 +282,7 @@ stats_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         if (et == 0) bulk_wait_read<1>();
         epi_sync();
 #pragma unroll
-        for (int ch = 0; ch < D / 16; ++ch) {
+        for (int ch = 0; ch < D / 16 && ok; ++ch) {
           uint32_t r[16];
           tmem_ld16(tmem + lrow + ab * D + ch * 16, r);
           tmem_wait_ld(r);
@@ -297,10 +300,10 @@ stats_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
           *reinterpret_cast<uint4*>(rowp + (((q0 + 1) ^ (a & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
         }
         tc_fence_before();
-        warp_arrive(SBAR(C::B_AEMPTY + ab));  // accumulator and stats slot are free
+        if (ok) warp_arrive(SBAR(C::B_AEMPTY + ab));  // accumulator and stats slot are free
         fence_proxy_async_smem();
         epi_sync();
-        if (et == 0) {
+        if (et == 0 && *abort_flag == 0) {
 #pragma unroll
           for (int p = 0; p < D / 64; ++p) tma_store_3d(&tmS1, stg + p * (D * 128), p * 64, 0, bh * nB + j);
           bulk_commit();
