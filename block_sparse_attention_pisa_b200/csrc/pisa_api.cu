@@ -207,21 +207,14 @@ pisa_status_t launch_select(const pisa_shape_t& s, const bf16* Q, const float* k
   p.QB = group * (pisa::kSelQB / group > 1 ? pisa::kSelQB / group : 1);
   p.tiles_per_head = (nB + p.QB - 1) / p.QB;
   const int64_t tiles = int64_t(s.B) * s.H * p.tiles_per_head;
-  if (tiles > (int64_t(1) << 30)) return fail(PISA_ERR_UNSUPPORTED, "too many select tiles (%lld)", (long long)tiles);
-  p.total_tiles = int(tiles);
+  if (tiles > (int64_t(1) << 31) - 1)
+    return fail(PISA_ERR_UNSUPPORTED, "too many select tiles (%lld)", (long long)tiles);
   p.ld = pisa::select_key_ld(nB);
-  // ring: up to two tiles' stages, as many as fit next to the rest of shared memory
-  constexpr int kMaxSmem = 227 * 1024 - 128;  // minus the base-alignment slack
-  const int spt = p.QB * (s.block / pisa::kSelStageRows);
-  int ring = 2 * spt;
-  while (ring > 2 && pisa::select_smem(D, nB, ring).bytes > kMaxSmem) --ring;
-  if (pisa::select_smem(D, nB, ring).bytes > kMaxSmem)
-    return fail(PISA_ERR_UNSUPPORTED, "select shared memory for nB=%d exceeds the limit", nB);
-  p.ring = ring;
-  const size_t smem = size_t(pisa::select_smem(D, nB, ring).bytes) + 128;
+  const size_t smem = size_t(pisa::select_smem(D, nB, group > 1 || cand < nB).bytes);
+  if (smem > size_t(227 * 1024)) return fail(PISA_ERR_UNSUPPORTED, "select shared memory for nB=%d exceeds the limit", nB);
   PISA_TRY(set_smem(k, smem));
-  const int grid = int(tiles < sms ? tiles : sms);
-  k<<<grid, pisa::kSelThreads, smem, st>>>(p);
+  (void)sms;
+  k<<<unsigned(tiles), pisa::kSelThreads, smem, st>>>(p);
   return check_launch("select_kernel");
 }
 

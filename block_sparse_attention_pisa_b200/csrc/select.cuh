@@ -14,27 +14,24 @@
 // query block then keeps the topk best of those candidates by its own pooled score
 // (cand = topk hands the proxy's list to every member unchanged: the reuse mode).
 //
-// Kernel layout: persistent CTAs (one per SM), each walking its tiles of QB query blocks
-// (QB = 8 for plain selection; a whole number of groups otherwise). Per tile:
-//   1. pool: the tile's query rows stream through a shared-memory ring of 64-row stages
-//      filled by bulk copies (cp.async.bulk, completion on an mbarrier per stage). Warp
-//      r sums query block r alone (16-byte shared reads, packed f32x2 adds, one shuffle
-//      reduction), then refills the ring slot it just read with the stage `ring` stages
-//      ahead -- the next tile's rows land while this tile is scored;
+// Kernel layout: one CTA (256 threads, two per SM) per tile of QB query blocks of one
+// head (QB = 8 for plain selection; a whole number of groups otherwise):
+//   1. pool: warp r sums query block r alone: batches of 16 independent 16-byte loads
+//      per lane (every load of a batch in flight before the first add), packed f32x2
+//      adds, one shuffle reduction, no CTA barrier;
 //   2. score: rows (pooled queries, or proxies) against key blocks. Each lane owns two
 //      key blocks of 32-block groups spread over the warps and every row of the tile;
-//      kbar streams through per-warp padded slabs (8 dimensions, cp.async, double
-//      buffered, conflict-free 16-byte reads) and the products accumulate as packed
-//      f32x2 FMAs in even / odd dimension pairs. Scores become order-preserving uint32
-//      keys in shared memory;
+//      kbar streams through per-warp padded slabs (8 dimensions, cp.async, three
+//      buffers: two slabs in flight while one is used; conflict-free 16-byte reads) and
+//      the products accumulate as packed f32x2 FMAs in even / odd dimension pairs.
+//      Scores become order-preserving uint32 keys in shared memory;
 //   3. top-k: one warp per row finds the k-th largest key bit by bit (starting below
 //      the row's common prefix) and emits the winners in ascending block order with
 //      ballots; among keys equal to the threshold the lowest indices are taken;
 //   4. grouped selection only: proxies first keep `cand` candidates (steps 2-3 over all
 //      key blocks), then the members are scored against their group's candidates
 //      (kbar rows gathered by index) and keep topk of them.
-// Every mbarrier wait is bounded (about a second); a wait that runs out raises the
-// device error word and the CTA stops issuing work.
+// Two CTAs share an SM, so one CTA's pooling (HBM) overlaps the other's scoring (FMA).
 #pragma once
 
 #include "common.cuh"
@@ -45,11 +42,11 @@ constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kSelQB = 8;                   // query blocks per tile (plain selection)
 constexpr int kSelMaxGroup = 8;             // query blocks per proxy, at most
-constexpr int kSelStageRows = 64;           // query rows per ring stage
 constexpr int kSelSlab = 8;                 // kbar dimensions per slab
 constexpr int kSelSlabLd = 12;              // padded slab row (floats): conflict-free 16-byte reads
 constexpr int kSelSlabBuf = 2 * 32 * kSelSlabLd;  // one slab buffer: two 32-row groups (floats)
-constexpr long long kSelWaitCycles = 2000000000LL;
+constexpr int kSelSlabBufs = 3;             // slab buffers per warp (two in flight)
+constexpr int kSelPoolBatch = 16;           // 16-byte query loads in flight per lane
 
 struct SelParams {
   const bf16* Q;
@@ -61,36 +58,32 @@ struct SelParams {
   int group;           // query blocks per proxy (1: each query block is its own)
   int cand;            // candidate list length (nB with group 1: plain selection)
   int QB;              // query blocks per tile (a multiple of group)
-  int tiles_per_head, total_tiles;
-  int ring;            // ring stages
+  int tiles_per_head;
   int ld;              // key row stride (uint32)
 };
 
 __host__ __device__ constexpr int select_key_ld(int nB) { return ((nB + 31) / 32) * 32 + 4; }
 
-// shared-memory carve-up (byte offsets; the ring comes first, 128-byte aligned)
+// shared-memory carve-up (byte offsets)
 struct SelSmem {
-  int ring_off, bar_off, qsum_off, qmean_off, proxy_off, key_off, cand_off, slab_off, misc_off, bytes;
+  int qsum_off, qmean_off, proxy_off, key_off, cand_off, slab_off, bytes;
 };
 
-__host__ __device__ inline SelSmem select_smem(int D, int nB, int ring) {
+// (the proxy rows and candidate lists exist only for grouped selection)
+__host__ __device__ inline SelSmem select_smem(int D, int nB, bool grouped) {
   SelSmem s{};
   int off = 0;
-  auto take = [&](int bytes, int align) {
-    off = (off + align - 1) / align * align;
+  auto take = [&](int bytes) {
     const int at = off;
-    off += bytes;
+    off += (bytes + 15) / 16 * 16;
     return at;
   };
-  s.ring_off = take(ring * kSelStageRows * D * 2, 128);
-  s.bar_off = take(ring * 8, 8);
-  s.qsum_off = take(kSelQB * D * 4, 16);
-  s.qmean_off = take(kSelQB * D * 4, 16);
-  s.proxy_off = take(kSelQB * D * 4, 16);
-  s.key_off = take(kSelQB * select_key_ld(nB) * 4, 16);
-  s.cand_off = take(kSelQB * ((nB + 7) / 8 * 8) * 2, 16);
-  s.slab_off = take(kSelWarps * 2 * kSelSlabBuf * 4, 16);
-  s.misc_off = take(16, 16);
+  s.qsum_off = take(kSelQB * D * 4);
+  s.qmean_off = take(kSelQB * D * 4);
+  s.proxy_off = take(grouped ? kSelQB * D * 4 : 0);
+  s.key_off = take(kSelQB * select_key_ld(nB) * 4);
+  s.cand_off = take(grouped ? kSelQB * ((nB + 7) / 8 * 8) * 2 : 0);
+  s.slab_off = take(kSelWarps * kSelSlabBufs * kSelSlabBuf * 4);
   s.bytes = off;
   return s;
 }
@@ -114,41 +107,6 @@ __device__ __forceinline__ void fma2(uint64_t& acc, uint64_t a, uint64_t b) {
   asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
 }
 
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// bounded wait: false (and the device error word raised) when it runs out
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-  if (mbar_try(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (!mbar_try(bar, parity)) {
-    if (clock64() - t0 > kSelWaitCycles) {
-      flag_error(kErrTimeout);
-      return false;
-    }
-  }
-  return true;
-}
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-      "l"(src), "r"(bytes), "r"(bar)
-      : "memory");
-}
 __device__ __forceinline__ void cp16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
@@ -226,26 +184,27 @@ __device__ void score_rows(int nrows, const float* rows, const float* kb_head, c
       dst[i] = uint32_t((gg * 32 + rr) * kSelSlabLd + cc * 4) * 4u;
       nbytes[i] = in ? 16u : 0u;
     }
+    // slab sl lives in buffer sl % 3; two slabs are in flight while one is used (an
+    // empty commit group keeps the group count uniform at the tail)
     auto issue = [&](int sl) {
-      const uint32_t b = slab_u + uint32_t((sl & 1) * kSelSlabBuf) * 4u;
+      if (sl < NSL) {
+        const uint32_t b = slab_u + uint32_t((sl % kSelSlabBufs) * kSelSlabBuf) * 4u;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) cp16(b + dst[i], src[i] + sl * kSelSlab, nbytes[i]);
+        for (int i = 0; i < 4; ++i) cp16(b + dst[i], src[i] + sl * kSelSlab, nbytes[i]);
+      }
       asm volatile("cp.async.commit_group;" ::: "memory");
     };
     uint64_t acc[R][2];
 #pragma unroll
     for (int r = 0; r < R; ++r) acc[r][0] = acc[r][1] = 0ull;
     issue(0);
+    issue(1);
 #pragma unroll 1
     for (int sl = 0; sl < NSL; ++sl) {
-      if (sl + 1 < NSL) {
-        issue(sl + 1);
-        asm volatile("cp.async.wait_group 1;" ::: "memory");
-      } else {
-        asm volatile("cp.async.wait_group 0;" ::: "memory");
-      }
+      issue(sl + 2);
+      asm volatile("cp.async.wait_group 2;" ::: "memory");
       __syncwarp();
-      const float* buf = slab + (sl & 1) * kSelSlabBuf;
+      const float* buf = slab + (sl % kSelSlabBufs) * kSelSlabBuf;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         const uint4 k0 = *reinterpret_cast<const uint4*>(buf + lane * kSelSlabLd + 4 * c);
@@ -262,7 +221,7 @@ __device__ void score_rows(int nrows, const float* rows, const float* kb_head, c
           fma2(acc[r][1], xb, k1b);
         }
       }
-      __syncwarp();  // this buffer is refilled two slabs later
+      __syncwarp();  // this buffer is refilled by the issue of the next iteration
     }
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
@@ -293,13 +252,10 @@ __device__ void score_dispatch(int R, const float* rows, const float* kb_head, c
 }  // namespace sel
 
 template <int D>
-__global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelParams p) {
-  extern __shared__ __align__(16) uint8_t sel_smem_raw[];
-  uint8_t* sel_smem = sel_smem_raw + ((128u - (smem_u32(sel_smem_raw) & 127u)) & 127u);
-  const SelSmem L = select_smem(D, p.nB, p.ring);
-  uint8_t* ring = sel_smem + L.ring_off;
-  const uint32_t ring_u = smem_u32(ring);
-  const uint32_t bar_u = smem_u32(sel_smem + L.bar_off);
+__global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelParams p) {
+  extern __shared__ __align__(16) uint8_t sel_smem[];
+  const bool grouped = p.group > 1 || p.cand < p.nB;
+  const SelSmem L = select_smem(D, p.nB, grouped);
   float* qsum = reinterpret_cast<float*>(sel_smem + L.qsum_off);    // [QB][D] row sums
   float* qmean = reinterpret_cast<float*>(sel_smem + L.qmean_off);  // [QB][D] pooled queries
   float* proxy = reinterpret_cast<float*>(sel_smem + L.proxy_off);  // [groups][D] proxy queries
@@ -307,78 +263,36 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelParams 
   int16_t* cand = reinterpret_cast<int16_t*>(sel_smem + L.cand_off);
   const int cand_ld = (p.nB + 7) / 8 * 8;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  float* slab = reinterpret_cast<float*>(sel_smem + L.slab_off) + warp * 2 * kSelSlabBuf;
-  volatile int* abort_flag = reinterpret_cast<int*>(sel_smem + L.misc_off);
-
-  constexpr int SB = kSelStageRows * D * 2;  // bytes per ring stage
-  const int spb = p.block / kSelStageRows;   // stages per query block
-  const int spt = p.QB * spb;                // stages per tile
-  const int ntiles = p.total_tiles > int(blockIdx.x) ? (p.total_tiles - 1 - int(blockIdx.x)) / int(gridDim.x) + 1 : 0;
-  const bool grouped = p.group > 1 || p.cand < p.nB;
-  const int G = p.QB / p.group;              // proxies per tile
-
-  // stage u of this CTA: tile u / spt, query block (u % spt) / spb, part (u % spt) % spb
-  auto issue = [&](int u) {
-    const int it = u / spt;
-    if (it >= ntiles) return;
-    const int T = int(blockIdx.x) + it * int(gridDim.x);
-    const int k = u % spt, r = k / spb, s = k % spb;
-    const int bh = T / p.tiles_per_head;
-    const int i = (T % p.tiles_per_head) * p.QB + r;
-    int rows = 0;
-    if (i < p.nB) rows = max(0, min(kSelStageRows, min(p.block, p.N - i * p.block) - s * kSelStageRows));
-    const uint32_t bar = bar_u + 8u * uint32_t(u % p.ring);
-    sel::mbar_expect_tx(bar, uint32_t(rows) * D * 2);
-    if (rows > 0)
-      sel::bulk_load(ring_u + uint32_t(u % p.ring) * SB,
-                     p.Q + (size_t(bh) * p.N + size_t(i) * p.block + s * kSelStageRows) * D, uint32_t(rows) * D * 2,
-                     bar);
-  };
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < p.ring; ++s) sel::mbar_init(bar_u + 8u * s, 1);
-    *abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  __syncthreads();
-  if (threadIdx.x == 0)
-    for (int u = 0; u < p.ring; ++u) issue(u);
-
-  for (int it = 0; it < ntiles; ++it) {
-    const int T = int(blockIdx.x) + it * int(gridDim.x);
+  float* slab = reinterpret_cast<float*>(sel_smem + L.slab_off) + warp * kSelSlabBufs * kSelSlabBuf;
+  const int G = p.QB / p.group;  // proxies per tile
+  {
+    const int T = blockIdx.x;
     const int bh = T / p.tiles_per_head;
     const int i0 = (T % p.tiles_per_head) * p.QB;
     const int nq = min(p.QB, p.nB - i0);
 
-    // ---- 1. pool: warp r sums query block i0 + r, stage by stage ----
-    if (warp < p.QB) {
+    // ---- 1. pool: warp r sums query block i0 + r ----
+    if (warp < nq) {
       constexpr int CH = D / 8;         // 16-byte chunks per row
       constexpr int RSTEP = 32 / CH;    // rows between a lane's rows
       const int c16 = lane % CH, r0 = lane / CH;
-      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
       const int i = i0 + warp;
-      const int n = i < p.nB ? min(p.block, p.N - i * p.block) : 0;
-      for (int s = 0; s < spb; ++s) {
-        const int u = it * spt + warp * spb + s;
-        const bool ok = *abort_flag == 0 && sel::mbar_wait(bar_u + 8u * uint32_t(u % p.ring), (u / p.ring) & 1);
-        if (!ok) *abort_flag = 1;
-        const int rows = max(0, min(kSelStageRows, n - s * kSelStageRows));
-        const uint8_t* st = ring + size_t(u % p.ring) * SB;
-        if (ok) {
-#pragma unroll 4
-          for (int r = r0; r < rows; r += RSTEP) {
-            const uint4 w = *reinterpret_cast<const uint4*>(st + r * (D * 2) + c16 * 16);
-            sel::add2(acc[0], sel::pack2(w.x << 16, w.x & 0xffff0000u));
-            sel::add2(acc[1], sel::pack2(w.y << 16, w.y & 0xffff0000u));
-            sel::add2(acc[2], sel::pack2(w.z << 16, w.z & 0xffff0000u));
-            sel::add2(acc[3], sel::pack2(w.w << 16, w.w & 0xffff0000u));
-          }
+      const int n = min(p.block, p.N - i * p.block);
+      const bf16* src = p.Q + (size_t(bh) * p.N + size_t(i) * p.block) * D + c16 * 8;
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+      for (int rb = r0; rb < n; rb += kSelPoolBatch * RSTEP) {
+        uint4 w[kSelPoolBatch];
+#pragma unroll
+        for (int b = 0; b < kSelPoolBatch; ++b) {
+          const int r = rb + b * RSTEP;
+          w[b] = r < n ? ldg_stream_v4(src + size_t(r) * D) : make_uint4(0u, 0u, 0u, 0u);
         }
-        __syncwarp();
-        // every read of this slot is done: refill it with the stage `ring` ahead
-        if (lane == 0 && *abort_flag == 0) {
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          issue(u + p.ring);
+#pragma unroll
+        for (int b = 0; b < kSelPoolBatch; ++b) {
+          sel::add2(acc[0], sel::pack2(w[b].x << 16, w[b].x & 0xffff0000u));
+          sel::add2(acc[1], sel::pack2(w[b].y << 16, w[b].y & 0xffff0000u));
+          sel::add2(acc[2], sel::pack2(w[b].z << 16, w[b].z & 0xffff0000u));
+          sel::add2(acc[3], sel::pack2(w[b].w << 16, w[b].w & 0xffff0000u));
         }
       }
       // lanes holding the same chunk sit CH apart
@@ -400,9 +314,10 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelParams 
           dst[2 * e + 1] = v.y;
         }
       }
+    } else if (warp < p.QB) {
+      for (int c = lane; c < D; c += 32) qsum[warp * D + c] = 0.f;  // a tile tail without rows
     }
     __syncthreads();
-    if (*abort_flag) break;
     // pooled queries (means of the real rows) and the groups' proxies
     for (int e = threadIdx.x; e < p.QB * D; e += kSelThreads) {
       const int r = e / D, i = i0 + r;
@@ -434,8 +349,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelParams 
       sel::score_dispatch<D>(nq, qmean, kb_head, route_head, p.lambda, nullptr, p.nB, keys, p.ld, slab);
       __syncthreads();
       if (warp < nq) sel::warp_topk(keys + warp * p.ld, p.nB, p.topk, idx_tile + size_t(warp) * p.topk, nullptr);
-      __syncthreads();
-      continue;
+      return;
     }
     // ---- 4. grouped: proxies keep `cand` candidates, members keep topk of those ----
     const int ng = (nq + p.group - 1) / p.group;  // groups present in this tile
@@ -446,8 +360,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelParams 
     if (p.cand == p.topk) {  // reuse: every member takes its group's list
       for (int e = threadIdx.x; e < nq * p.topk; e += kSelThreads)
         idx_tile[e] = cand[(e / p.topk / p.group) * cand_ld + e % p.topk];
-      __syncthreads();
-      continue;
+      return;
     }
     for (int m = 0; m < ng; ++m) {
       const int rows = min(p.group, nq - m * p.group);
@@ -458,7 +371,6 @@ __global__ void __launch_bounds__(kSelThreads, 1) select_kernel(const SelParams 
     if (warp < nq)
       sel::warp_topk(keys + warp * p.ld, p.cand, p.topk, idx_tile + size_t(warp) * p.topk,
                      cand + (warp / p.group) * cand_ld);
-    __syncthreads();
   }
 }
 

@@ -226,8 +226,7 @@ stats_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
-        __syncwarp();
-        mbar_arrive(SBAR(C::B_EMPTY + s));  // per warp (count includes both sum warps)
+        warp_arrive(SBAR(C::B_EMPTY + s));  // one arrival per warp (the count is 1 commit + 2 warps)
         // the stats slot: S1 mode double-buffers per block; Hbar mode keeps the unit's blocks
         const int slot = MODE == 2 ? ab * C::UNIT + i : (t & 1);
         if (MODE != 2 && i == 0 && t >= 2) {
@@ -251,9 +250,8 @@ stats_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             reinterpret_cast<float4*>(dst_g)[1] = v1;
           }
         }
-        __syncwarp();
         const int fb = MODE == 2 ? ab : (t & 1);
-        if (MODE != 2 || i == C::UNIT - 1) mbar_arrive(SBAR(C::B_SFULL + fb));
+        if (MODE != 2 || i == C::UNIT - 1) warp_arrive(SBAR(C::B_SFULL + fb));  // one per warp
       }
     }
   } else {

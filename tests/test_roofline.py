@@ -47,3 +47,17 @@ def test_routing_and_hybrid_bytes():
     assert R.routing_bytes(1, 24, 32768, 128, 64) / 1e6 == pytest.approx(808.5, abs=1.0)
     # order 2 writes Hbar (64 KB per head) instead of per-block S1
     assert R.stats_bytes(1, 24, 32768, 128, 64, 2) / 1e6 == pytest.approx(416.8, abs=1.0)
+
+
+def test_grouped_select_flops():
+    # video: 512 query blocks, groups of 4 -> 128 proxies scored against 512 key blocks,
+    # then 512 members against 128 candidates each: half the plain 512 x 512 scores
+    plain = R.select_flops(1, 24, 32768, 128, 64)
+    assert plain == pytest.approx(24 * 2 * 512 * 512 * 128)
+    grouped = R.select_flops(1, 24, 32768, 128, 64, group=4, cand=128)
+    assert grouped == pytest.approx(24 * 2 * 128 * (128 * 512 + 512 * 128))
+    assert grouped == pytest.approx(plain / 2)
+    # group 1 with every key block a candidate is plain selection
+    assert R.select_flops(1, 24, 32768, 128, 64, group=1, cand=512) == pytest.approx(plain)
+    # a ragged group count rounds up
+    assert R.select_flops(1, 1, 64 * 10, 64, 64, group=4, cand=3) == pytest.approx(2 * 64 * (3 * 10 + 10 * 3))
