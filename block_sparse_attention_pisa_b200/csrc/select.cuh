@@ -25,9 +25,10 @@
 //      buffers: two slabs in flight while one is used; conflict-free 16-byte reads) and
 //      the products accumulate as packed f32x2 FMAs in even / odd dimension pairs.
 //      Scores become order-preserving uint32 keys in shared memory;
-//   3. top-k: one warp per row finds the k-th largest key bit by bit (starting below
-//      the row's common prefix) and emits the winners in ascending block order with
-//      ballots; among keys equal to the threshold the lowest indices are taken;
+//   3. top-k: one warp per row, the row's keys in registers (up to 1024 of them), finds
+//      the k-th largest key bit by bit (starting below the row's common prefix) and
+//      emits the winners in ascending block order with ballots; among keys equal to
+//      the threshold the lowest indices are taken;
 //   4. grouped selection only: proxies first keep `cand` candidates (steps 2-3 over all
 //      key blocks), then the members are scored against their group's candidates
 //      (kbar rows gathered by index) and keep topk of them.
@@ -155,6 +156,65 @@ __device__ void warp_topk(const uint32_t* row, int L, int k, OutT* out, const in
     written += __popc(take_mask);
     eq_seen += __popc(eq_mask);
   }
+}
+
+// warp_topk with the row's keys held in registers (KPL per lane, L <= 32 KPL): the bit
+// search then reads no shared memory. Positions past L hold key 0, which no threshold
+// of real (finite) scores reaches.
+template <int KPL, typename OutT>
+__device__ void warp_topk_reg(const uint32_t* row, int L, int k, OutT* out, const int16_t* map) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  uint32_t key[KPL];
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) {
+    const int jj = 32 * i + lane;
+    key[i] = jj < L ? row[jj] : 0u;
+    if (jj < L) {
+      kmin = min(kmin, key[i]);
+      kmax = max(kmax, key[i]);
+    }
+  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  const uint32_t diff = kmin ^ kmax;
+  const int top = diff ? 31 - __clz(diff) : -1;  // highest differing bit
+  uint32_t T = top < 0 ? kmax : (top >= 31 ? 0u : (kmax & ~((2u << top) - 1u)));
+  for (int bit = top; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    unsigned cnt = 0;
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) cnt += key[i] >= cand;
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
+    if (cnt >= unsigned(k)) T = cand;
+  }
+  unsigned gt = 0;
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) gt += key[i] > T;
+  gt = __reduce_add_sync(0xffffffffu, gt);
+  const int need_eq = k - int(gt);
+  int written = 0, eq_seen = 0;
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) {
+    const int jj = 32 * i + lane;
+    const bool in = jj < L;
+    const bool is_gt = in && key[i] > T;
+    const bool is_eq = in && key[i] == T;
+    const unsigned eq_mask = __ballot_sync(0xffffffffu, is_eq);
+    const bool take = is_gt || (is_eq && eq_seen + __popc(eq_mask & lt_mask) < need_eq);
+    const unsigned take_mask = __ballot_sync(0xffffffffu, take);
+    if (take) out[written + __popc(take_mask & lt_mask)] = OutT(map ? int(map[jj]) : jj);
+    written += __popc(take_mask);
+    eq_seen += __popc(eq_mask);
+  }
+}
+
+template <typename OutT>
+__device__ void topk_dispatch(const uint32_t* row, int L, int k, OutT* out, const int16_t* map) {
+  if (L <= 32 * 16) warp_topk_reg<16>(row, L, k, out, map);
+  else if (L <= 32 * 32) warp_topk_reg<32>(row, L, k, out, map);
+  else warp_topk(row, L, k, out, map);
 }
 
 // Scores of R rows (fp32 [R][D] in shared memory) against the key blocks list[0, L)
@@ -348,14 +408,14 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelParams 
       // ---- 2-3. plain selection ----
       sel::score_dispatch<D>(nq, qmean, kb_head, route_head, p.lambda, nullptr, p.nB, keys, p.ld, slab);
       __syncthreads();
-      if (warp < nq) sel::warp_topk(keys + warp * p.ld, p.nB, p.topk, idx_tile + size_t(warp) * p.topk, nullptr);
+      if (warp < nq) sel::topk_dispatch(keys + warp * p.ld, p.nB, p.topk, idx_tile + size_t(warp) * p.topk, nullptr);
       return;
     }
     // ---- 4. grouped: proxies keep `cand` candidates, members keep topk of those ----
     const int ng = (nq + p.group - 1) / p.group;  // groups present in this tile
     sel::score_dispatch<D>(ng, proxy, kb_head, route_head, p.lambda, nullptr, p.nB, keys, p.ld, slab);
     __syncthreads();
-    if (warp < ng) sel::warp_topk(keys + warp * p.ld, p.nB, p.cand, cand + warp * cand_ld, nullptr);
+    if (warp < ng) sel::topk_dispatch(keys + warp * p.ld, p.nB, p.cand, cand + warp * cand_ld, nullptr);
     __syncthreads();
     if (p.cand == p.topk) {  // reuse: every member takes its group's list
       for (int e = threadIdx.x; e < nq * p.topk; e += kSelThreads)
@@ -369,8 +429,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelParams 
     }
     __syncthreads();
     if (warp < nq)
-      sel::warp_topk(keys + warp * p.ld, p.cand, p.topk, idx_tile + size_t(warp) * p.topk,
-                     cand + (warp / p.group) * cand_ld);
+      sel::topk_dispatch(keys + warp * p.ld, p.cand, p.topk, idx_tile + size_t(warp) * p.topk,
+                         cand + (warp / p.group) * cand_ld);
   }
 }
 

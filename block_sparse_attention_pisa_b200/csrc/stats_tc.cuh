@@ -15,8 +15,9 @@
 //   warp 0     TMA producer: K_j and V_j (128-byte swizzled 64-column panels, rows past
 //              N zero-filled) into a ring of stages;
 //   warp 1     MMA issuer (one thread): K_j^T V_j into one of two TMEM accumulators;
-//   warps 2-3  column sums from the stage: kbar_j (mean of the real rows) and S0_j, to
-//              global memory and to shared memory for the epilogue;
+//   warps 8-11 column sums from the stage, one 64-column panel of K or V each: kbar_j
+//              (mean of the real rows) and S0_j, to global memory and to shared memory
+//              for the epilogue;
 //   warps 4-7  epilogue, one TMEM lane (= key dimension a) per thread: S1 mode
 //              subtracts kbar_j[a] S0_j[c], rounds to bf16 into a swizzled staging tile
 //              and writes it with TMA stores; Hbar mode subtracts sum_j kbar_j[a] S0_j[c]
@@ -32,7 +33,7 @@ namespace pisa {
 template <int BLK, int MODE>
 struct StatsTcCfg {
   static constexpr int D = 128;
-  static constexpr int kThreads = 256;
+  static constexpr int kThreads = 384;
   static constexpr int UNIT = (MODE == 2) ? 16 : 1;               // blocks per work unit
   static constexpr int STAGE = 2 * BLK * D * 2;                    // K and V tiles
   static constexpr int STG = D * D * 2;                            // bf16 S1 staging tile
@@ -44,10 +45,10 @@ struct StatsTcCfg {
   static_assert(NS >= 2, "ring");
   // barriers
   static constexpr int B_FULL = 0;              // [NS] stage landed (TMA tx)
-  static constexpr int B_EMPTY = B_FULL + NS;   // [NS] stage consumed (MMA commit + 2 sum warps)
+  static constexpr int B_EMPTY = B_FULL + NS;   // [NS] stage consumed (MMA commit + 4 sum warps)
   static constexpr int B_AFULL = B_EMPTY + NS;  // [2]  accumulator ready (commit)
   static constexpr int B_AEMPTY = B_AFULL + 2;  // [2]  accumulator and stats slot read (4 warps)
-  static constexpr int B_SFULL = B_AEMPTY + 2;  // [2]  kbar / S0 in shared memory (2 warps)
+  static constexpr int B_SFULL = B_AEMPTY + 2;  // [2]  kbar / S0 in shared memory (4 warps)
   static constexpr int B_DONE = B_SFULL + 2;    //      every MMA finished (commit)
   static constexpr int NBARS = B_DONE + 1;
   // shared memory (offsets from a 1024-byte aligned base)
@@ -95,7 +96,7 @@ __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" :::
 
 // MODE: kStatsS1 (1) per-block S1, kStatsHbar (2) the head's Hbar. d = 128 only.
 template <int BLK, int MODE>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
 stats_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                 const __grid_constant__ CUtensorMap tmS1, int N, int nB, int units_per_head, int total_units,
                 float* __restrict__ kbar, float* __restrict__ S0, float* __restrict__ Hbar) {
@@ -125,12 +126,12 @@ stats_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(SBAR(C::B_FULL + s), 1);
-      mbar_init(SBAR(C::B_EMPTY + s), 3);
+      mbar_init(SBAR(C::B_EMPTY + s), 5);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(SBAR(C::B_AFULL + b), 1);
       mbar_init(SBAR(C::B_AEMPTY + b), 4);
-      mbar_init(SBAR(C::B_SFULL + b), 2);
+      mbar_init(SBAR(C::B_SFULL + b), 4);
     }
     mbar_init(SBAR(C::B_DONE), 1);
     misc[1] = 0;
@@ -194,12 +195,13 @@ stats_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       umma_commit(SBAR(C::B_DONE));
       wait_drain(SBAR(C::B_DONE), 0);
     }
-  } else if (warp < 4) {
+  } else if (warp >= 8) {
     // ------------------------------------------------------------ column sums
-    // thread: tensor (warp 2: K, warp 3: V), 16-byte column chunk lane % 16, row parity lane / 16
-    const bool isV = warp == 3;
-    const int q16 = lane & 15, half = lane >> 4;
-    const int panel = q16 >> 3, qc = q16 & 7;
+    // warp 8 + 2 isV + panel: one 64-column panel of K or V; lane = 16-byte chunk lane % 8
+    // of the panel and row phase lane / 8 (rows lane / 8, + 4, + 8, ...)
+    const bool isV = warp >= 10;
+    const int panel = warp & 1;
+    const int qc = lane & 7, r0 = lane >> 3;
     int t = 0;
     for (int u = 0; u < nunits; ++u) {
       const int ab = u & 1;
@@ -215,7 +217,7 @@ stats_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll 4
-        for (int r = half; r < BLK; r += 2) {  // zero-filled rows past N add nothing
+        for (int r = r0; r < BLK; r += 4) {  // zero-filled rows past N add nothing
           const uint4 w = *reinterpret_cast<const uint4*>(tile + r * 128 + ((qc ^ (r & 7)) << 4));
           const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -225,8 +227,12 @@ stats_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
           }
         }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
-        warp_arrive(SBAR(C::B_EMPTY + s));  // one arrival per warp (the count is 1 commit + 2 warps)
+        for (int e = 0; e < 8; ++e) {
+          acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 8);
+          acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
+        }
+        warp_arrive(SBAR(C::B_EMPTY + s));  // one arrival per warp (the count is 1 commit + 4 warps)
+        const int q16 = panel * 8 + qc;  // 16-byte chunk of the row (8 columns)
         // the stats slot: S1 mode double-buffers per block; Hbar mode keeps the unit's blocks
         const int slot = MODE == 2 ? ab * C::UNIT + i : (t & 1);
         if (MODE != 2 && i == 0 && t >= 2) {
@@ -236,7 +242,7 @@ stats_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         if (MODE == 2 && i == 0 && u >= 2) {
           if (!__all_sync(0xffffffffu, wait_bounded(SBAR(C::B_AEMPTY + ab), ((u >> 1) & 1) ^ 1, abort_flag))) break;
         }
-        if (lane < 16) {
+        if (lane < 8) {
           // blocks past nB (the zero-filled tail of a head's last Hbar unit) write nothing
           float* dst_s = stats + slot * 2 * D + (isV ? D : 0) + q16 * 8;
           const float f = isV ? 1.f : (n > 0 ? 1.f / float(n) : 0.f);
@@ -254,8 +260,8 @@ stats_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         if (MODE != 2 || i == C::UNIT - 1) warp_arrive(SBAR(C::B_SFULL + fb));  // one per warp
       }
     }
-  } else {
-    // ------------------------------------------------------------ epilogue
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue (warps 4-7; 2-3 idle)
     const int et = threadIdx.x - 128;  // = TMEM lane = key dimension a
     const int quarter = warp & 3;
     const uint32_t lrow = uint32_t(quarter * 32) << 16;
