@@ -12,6 +12,7 @@
 #include "common.cuh"
 #include "stats.cuh"
 #include "select.cuh"
+#include "select_pipe.cuh"
 #include "routing.cuh"
 #include "attention_simt.cuh"
 #include "attention_tc.cuh"
@@ -144,6 +145,7 @@ pisa_status_t launch_stats_mode(const pisa_shape_t& s, const bf16* K, const bf16
 }
 
 pisa_status_t make_map(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box1);
+pisa_status_t make_plane_map(CUtensorMap* m, const float* kbar, uint64_t D, uint64_t nB, uint64_t BH, uint32_t rows);
 
 // d = 128, orders 1 and 2: the tensor-core statistics kernel (persistent, one CTA per SM)
 template <int BLK, int MODE>
@@ -187,11 +189,63 @@ pisa_status_t launch_stats(const pisa_shape_t& s, const bf16* K, const bf16* V, 
   return launch_stats_mode<D, BLK, pisa::kStatsSums>(s, K, V, kbar, S0, nullptr, nullptr, st);
 }
 
+// plain selection, nB <= 640: the persistent pipelined kernel (KL key blocks per lane)
+template <int D, int KL>
+pisa_status_t launch_select_pipe(const pisa_shape_t& s, const float* kbar, pisa::SpParams& p, int sms,
+                                 cudaStream_t st) {
+  const uint64_t BH = uint64_t(s.B) * s.H;
+  CUtensorMap m;
+  PISA_TRY(make_plane_map(&m, kbar, D, uint64_t(p.nB), BH, uint32_t(p.box_rows)));
+  auto k = pisa::select_pipe_kernel<D, KL>;
+  PISA_TRY(set_smem(k, size_t(p.smem)));
+  const int grid = p.tiles < sms ? p.tiles : sms;
+  k<<<grid, pisa::kSpThreads, p.smem, st>>>(m, p);
+  return check_launch("select_pipe_kernel");
+}
+
+template <int D>
+pisa_status_t try_select_pipe(const pisa_shape_t& s, const bf16* Q, const float* kbar, const float* route,
+                              float lambda, int topk, int32_t* idx, int sms, cudaStream_t st, bool& done) {
+  done = false;
+  const int nB = int(num_blocks(s));
+  const int need = (nB + 63) / 64;
+  const int KL = need <= 2 ? need : (need <= 4 ? 4 : (need <= 6 ? 6 : (need <= 8 ? 8 : 10)));
+  if (need > pisa::kSpMaxKL) return ok();
+  pisa::SpParams p{};
+  if (!pisa::select_pipe_plan<D>(nB, s.block, KL, p)) return ok();
+  const int64_t tiles = int64_t(s.B) * s.H * ((nB + pisa::kSpRows - 1) / pisa::kSpRows);
+  if (tiles > (int64_t(1) << 31) - 1) return ok();
+  p.Q = Q;
+  p.route = route;
+  p.lambda = lambda;
+  p.idx = idx;
+  p.N = s.N;
+  p.nB = nB;
+  p.block = s.block;
+  p.topk = topk;
+  p.tiles_per_head = (nB + pisa::kSpRows - 1) / pisa::kSpRows;
+  p.tiles = int(tiles);
+  done = true;
+  switch (KL) {
+    case 1: return launch_select_pipe<D, 1>(s, kbar, p, sms, st);
+    case 2: return launch_select_pipe<D, 2>(s, kbar, p, sms, st);
+    case 4: return launch_select_pipe<D, 4>(s, kbar, p, sms, st);
+    case 6: return launch_select_pipe<D, 6>(s, kbar, p, sms, st);
+    case 8: return launch_select_pipe<D, 8>(s, kbar, p, sms, st);
+    default: return launch_select_pipe<D, 10>(s, kbar, p, sms, st);
+  }
+}
+
 template <int D>
 pisa_status_t launch_select(const pisa_shape_t& s, const bf16* Q, const float* kbar, const float* route,
                             float lambda, int topk, int group, int cand, int32_t* idx, int sms, cudaStream_t st) {
   auto k = pisa::select_kernel<D>;
   const int nB = int(num_blocks(s));
+  if (group == 1 && cand == nB) {
+    bool done = false;
+    const pisa_status_t r = try_select_pipe<D>(s, Q, kbar, route, lambda, topk, idx, sms, st, done);
+    if (done || r != PISA_OK) return r;
+  }
   pisa::SelParams p{};
   p.Q = Q;
   p.kbar = kbar;
@@ -278,6 +332,22 @@ pisa_status_t make_map(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(PISA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return ok();
+}
+
+// kbar fp32 [BH][nB][D] as planes of kSpPlane = 8 dimensions: box = 8 dimensions x `rows`
+// key blocks (32-byte rows, 32-byte swizzle); rows past nB read as zero
+pisa_status_t make_plane_map(CUtensorMap* m, const float* kbar, uint64_t D, uint64_t nB, uint64_t BH, uint32_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(PISA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[3] = {D, nB, BH};
+  cuuint64_t strides[2] = {D * 4, D * nB * 4};
+  cuuint32_t box[3] = {uint32_t(pisa::kSpPlane), rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(kbar), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PISA_ERR_CUDA, "cuTensorMapEncodeTiled (kbar planes) failed (%d)", int(r));
   return ok();
 }
 
