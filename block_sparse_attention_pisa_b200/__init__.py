@@ -21,7 +21,7 @@ ORDER_DROP, ORDER_ZERO, ORDER_FIRST, ORDER_HYBRID = -1, 0, 1, 2
 
 __all__ = [
     "ORDER_DROP", "ORDER_ZERO", "ORDER_FIRST", "ORDER_HYBRID", "PisaError", "Shape", "HostOptions", "lib", "block_stats", "select", "attention", "attention_simt",
-    "pisa", "pisa_host", "host_workspace_bytes", "head_chunks", "device_error", "num_blocks", "LIB_PATH", "SYMBOLS", "routing_norms",
+    "pisa", "pisa_host", "pisa_host_static", "STATIC_WORKSPACE_BYTES", "host_workspace_bytes", "head_chunks", "device_error", "num_blocks", "LIB_PATH", "SYMBOLS", "routing_norms",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpisa.so")
@@ -30,8 +30,11 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpisa.so"
 SYMBOLS = (
     "pisa_block_stats", "pisa_select", "pisa_routing_norms", "pisa_attention", "pisa_attention_simt",
     "pisa_device_error", "pisa_status_string", "pisa_last_error", "pisa_version",
-    "pisa_run_host_workspace", "pisa_run_host", "pisa_select_grouped",
+    "pisa_run_host_workspace", "pisa_run_host", "pisa_select_grouped", "pisa_run_host_static",
 )
+
+# PISA_STATIC_WORKSPACE_BYTES in include/pisa.h: the device region pisa_run_host_static uses
+STATIC_WORKSPACE_BYTES = 32 << 20
 
 STATUS = {0: "PISA_OK", 1: "PISA_ERR_INVALID_ARG", 2: "PISA_ERR_UNSUPPORTED",
           3: "PISA_ERR_CUDA", 4: "PISA_ERR_TIMEOUT"}
@@ -77,6 +80,7 @@ def lib():
     opts = ctypes.POINTER(HostOptions)
     L.pisa_run_host_workspace.argtypes = [Shape, i32, i32, opts, ctypes.POINTER(ctypes.c_size_t)]
     L.pisa_run_host.argtypes = [vp, vp, vp, Shape, i32, i32, f32, opts, vp, ctypes.c_size_t, vp, vp]
+    L.pisa_run_host_static.argtypes = [vp, vp, vp, Shape, i32, i32, f32, opts, vp, vp]
     L.pisa_device_error.argtypes = [vp]
     L.pisa_status_string.argtypes = [ctypes.c_int]
     L.pisa_status_string.restype = ctypes.c_char_p
@@ -85,7 +89,7 @@ def lib():
     L.pisa_version.argtypes = []
     for name in ("pisa_block_stats", "pisa_select", "pisa_routing_norms", "pisa_attention", "pisa_attention_simt",
                  "pisa_device_error", "pisa_version", "pisa_run_host_workspace", "pisa_run_host",
-                 "pisa_select_grouped"):
+                 "pisa_select_grouped", "pisa_run_host_static"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -374,6 +378,37 @@ def pisa_host(Q, K, V, block: int, topk: int, order: int = 1, scale: float | Non
         stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
         _check(lib().pisa_run_host(_ptr(Q), _ptr(K), _ptr(V), s, int(topk), int(order), float(scale),
                                    ctypes.byref(o), _ptr(ws), nbytes.value, _ptr(out), stream))
+    return out
+
+
+def pisa_host_static(Q, K, V, block: int, topk: int, order: int = 1, scale: float | None = None,
+                     device="cuda", route_lambda: float = 0.0, chunks: int = 8, out=None,
+                     group: int = 1, candidates: int = 0):
+    """``pisa_host`` through the C ABI's ``pisa_run_host_static``: the device workspace is
+    the library's fixed region (``STATIC_WORKSPACE_BYTES`` per device) and nothing is
+    allocated on the device. Calls that overlap in time on one device race on that region.
+    Returns O on the host (``out`` if given, else a new host tensor)."""
+    import torch
+    if scale is None:
+        scale = Q.shape[-1] ** -0.5
+    s = _shape(Q, block)
+    for t, name in ((Q, "Q"), (K, "K"), (V, "V")):
+        _require(t, name, Q.shape, torch.bfloat16)
+        if t.is_cuda:
+            raise ValueError(f"{name} must be a host tensor (pisa_host_static copies it to the device)")
+    if out is None:
+        out = torch.empty(Q.shape, dtype=Q.dtype, pin_memory=Q.is_pinned())
+    _require(out, "O", Q.shape, torch.bfloat16)
+    if out.is_cuda:
+        raise ValueError("O must be a host tensor")
+    dev = torch.device(device)
+    if dev.index is None:
+        dev = torch.device("cuda", torch.cuda.current_device())
+    o = HostOptions(float(route_lambda), int(group), int(candidates or 0), int(chunks))
+    with torch.cuda.device(dev):
+        stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+        _check(lib().pisa_run_host_static(_ptr(Q), _ptr(K), _ptr(V), s, int(topk), int(order), float(scale),
+                                          ctypes.byref(o), _ptr(out), stream))
     return out
 
 

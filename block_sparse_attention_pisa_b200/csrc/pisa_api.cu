@@ -555,6 +555,35 @@ pisa_status_t host_options(const pisa_shape_t& s, int32_t topk, const pisa_host_
 
 }  // namespace
 
+// The device workspace of pisa_run_host_static: one region per device, part of the
+// library's module (no allocation at call time); its address is looked up once per device.
+static __device__ __align__(256) unsigned char g_static_workspace[PISA_STATIC_WORKSPACE_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_ptr[kMaxDevices] = {};
+
+pisa_status_t static_workspace(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(PISA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(PISA_ERR_UNSUPPORTED, "device %d (at most %d)", dev, kMaxDevices);
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (g_static_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_workspace);  // the current device's copy
+    if (e != cudaSuccess)
+      return fail(PISA_ERR_CUDA, "cudaGetSymbolAddress(static workspace): %s", cudaGetErrorString(e));
+    g_static_ptr[dev] = p;
+  }
+  *out = g_static_ptr[dev];
+  return ok();
+}
+
+}  // namespace
+
 extern "C" {
 
 pisa_status_t pisa_run_host_workspace(pisa_shape_t shape, int32_t topk, int32_t order,
@@ -711,6 +740,30 @@ pisa_status_t pisa_run_host(const void* Q, const void* K, const void* V, pisa_sh
   if (in_s) cudaStreamDestroy(in_s);
   if (out_s) cudaStreamDestroy(out_s);
   return st;
+}
+
+pisa_status_t pisa_run_host_static(const void* Q, const void* K, const void* V, pisa_shape_t shape, int32_t topk,
+                                   int32_t order, float scale, const pisa_host_options_t* options, void* O,
+                                   void* stream) {
+  size_t need = 0;
+  PISA_TRY(pisa_run_host_workspace(shape, topk, order, options, &need));
+  if (need == 0) return ok();  // empty problem: nothing touched
+  if (need > size_t(PISA_STATIC_WORKSPACE_BYTES))
+    return fail(PISA_ERR_UNSUPPORTED,
+                "the problem needs %zu bytes of workspace, the static region holds %zu (more chunks make the ranges "
+                "smaller)",
+                need, size_t(PISA_STATIC_WORKSPACE_BYTES));
+  // argument errors before the first device call
+  const void* host[4] = {Q, K, V, O};
+  const char* names[4] = {"Q", "K", "V", "O"};
+  for (int i = 0; i < 4; ++i)
+    if (host[i] == nullptr) return fail(PISA_ERR_INVALID_ARG, "%s is NULL", names[i]);
+  if (!std::isfinite(scale) || !(scale > 0.f))
+    return fail(PISA_ERR_INVALID_ARG, "scale=%g (must be finite and > 0)", double(scale));
+  void* ws = nullptr;
+  PISA_TRY(static_workspace(&ws));
+  return pisa_run_host(Q, K, V, shape, topk, order, scale, options, ws, size_t(PISA_STATIC_WORKSPACE_BYTES), O,
+                       stream);
 }
 
 pisa_status_t pisa_device_error(void* stream) {

@@ -231,6 +231,34 @@ pisa_status_t pisa_run_host(const void* Q, const void* K, const void* V, pisa_sh
                             int32_t order, float scale, const pisa_host_options_t* options, void* workspace,
                             size_t workspace_bytes, void* O, void* stream);
 
+/* Size of the library's own device workspace region used by pisa_run_host_static. */
+#define PISA_STATIC_WORKSPACE_BYTES (32u << 20)
+
+/*
+ * pisa_run_host_static -- pisa_run_host with no workspace from the caller: for callers
+ * that cannot allocate device memory. The explainer has no counterpart; this is an
+ * entry point of this library only.
+ * Arguments, result and errors are those of pisa_run_host without `workspace` and
+ * `workspace_bytes`: the device workspace is a fixed region of PISA_STATIC_WORKSPACE_BYTES
+ * (32 MiB, 256-byte aligned) that the library holds on every device as part of its
+ * loaded code, and the call allocates no memory (it creates and destroys its two copy
+ * streams and events as pisa_run_host does). A problem whose pisa_run_host_workspace
+ * figure exceeds the region is rejected with PISA_ERR_UNSUPPORTED before anything runs
+ * (more `chunks` make each range, and the figure, smaller).
+ * Nothing in the region has to start at zero: every byte the path reads there was
+ * written earlier in the same call (statistics that accumulate are zeroed on the
+ * stream first).
+ * The region is ONE PER DEVICE, shared by every call on that device: calls that overlap
+ * in time (from other host threads, or on other streams) race on it, and the caller
+ * must serialise them. Each call blocks until it is done, so consecutive calls from one
+ * thread are safe.
+ * The first call on a device looks the region's address up (cudaGetSymbolAddress, with
+ * that device current): make that first call outside any stream capture.
+ */
+pisa_status_t pisa_run_host_static(const void* Q, const void* K, const void* V, pisa_shape_t shape, int32_t topk,
+                                   int32_t order, float scale, const pisa_host_options_t* options, void* O,
+                                   void* stream);
+
 /*
  * pisa_device_error -- takes the device error word that the kernels set, after all
  * work already enqueued on `stream`, and synchronises `stream`. Returns PISA_OK,

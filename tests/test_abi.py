@@ -247,6 +247,28 @@ def test_host_entry_arguments(L):
     _passes_validation(run_host(L, Q=MISALIGNED), L)     # host buffers need no alignment
 
 
+def test_static_host_entry_arguments(L):
+    """pisa_run_host_static: the argument checks of pisa_run_host, and a problem whose
+    workspace exceeds the library's fixed region is rejected before any device work."""
+    def run(s, topk=2, order=1, chunks=1, **ptrs):
+        p = {k: FAKE for k in ("Q", "K", "V", "O")}
+        p.update(ptrs)
+        return L.pisa_run_host_static(vp(p["Q"]), vp(p["K"]), vp(p["V"]), s, topk, order, 0.1, _opts(0.0, chunks),
+                                      vp(p["O"]), None)
+    big = shape(B=1, H=2, N=32768, d=128, block=64)              # 64 MiB of Q, K, V, O in one range
+    assert _ws(L, big, 64, 1, 0.0, 1)[1] > P.STATIC_WORKSPACE_BYTES
+    assert run(big, topk=64) == UNSUPPORTED
+    assert b"static region" in L.pisa_last_error()
+    assert run(shape(), topk=9) == INVALID                        # topk > nB
+    assert run(shape(), order=5) == INVALID
+    assert run(shape(B=0), Q=0, K=0, V=0, O=0) == OK               # empty problem: nothing touched
+    assert _ws(L, shape(), 2, 1, 0.0, 1)[1] <= P.STATIC_WORKSPACE_BYTES
+    for name in ("Q", "K", "V", "O"):
+        assert run(shape(), **{name: 0}) == INVALID, name
+    _no_device()
+    _passes_validation(run(shape()), L)                           # only the device remains
+
+
 def sel_grouped(L, s=None, Q=FAKE, kbar=FAKE, topk=2, group=2, cand=3, idx=FAKE, route=0, lam=0.0):
     return L.pisa_select_grouped(vp(Q), vp(kbar), vp(route), lam, s or shape(), topk, group, cand, vp(idx), None)
 
