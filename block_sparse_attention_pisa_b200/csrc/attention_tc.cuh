@@ -160,7 +160,9 @@ struct TcCfg {
   static constexpr int OFF_XCH = OFF_MASK + 2 * (MAXB / 32) * 4;  // float [2 parity][2 half][128] row maxima
   static constexpr int OFF_XS = OFF_XCH + 2 * 2 * 128 * 4;          // float [2 half][128] alpha sums
   static constexpr int OFF_XL = OFF_XS + 2 * 128 * 4;               // float [2 half][128] denominators
-  static constexpr int OFF_BAR = OFF_XL + 2 * 128 * 4;
+  static constexpr int A0_LD = CHUNK / 2 + 1;                      // padded: conflict-free row access
+  static constexpr int OFF_A0 = OFF_XL + 2 * 128 * 4;               // uint32 [128 rows][A0_LD] packed alpha
+  static constexpr int OFF_BAR = OFF_A0 + 128 * A0_LD * 4;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
   static constexpr int SMEM = OFF_MISC + 64 + 1024;  // + alignment slack
   static_assert(OFF_BAR % 8 == 0, "barrier alignment");
@@ -413,7 +415,9 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       constexpr uint32_t idSB = idesc_bf16(128, C::CHUNK, false);  // Sbar = Q Kbar^T
       constexpr uint32_t idO = idesc_bf16(128, D, true);           // O += {P V, alpha S0, A S1}
       uint32_t o_acc = 0;
-      uint32_t g_acc[2] = {0u, 0u};  // GROUPS: each group's accumulator holds a product
+      // GROUPS: bit g set once group g's accumulator holds a product (a bit mask, not an
+      // array: a runtime index would put the array in local memory)
+      uint32_t g_acc = 0u;
       bool ok = wait_poll(BAR(C::B_Q), 0, abort_flag);
       tc_fence_after();
       auto pv = [&](int e) -> bool {
@@ -429,8 +433,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
 #pragma unroll
           for (int k = 0; k < BLK / 16; ++k)
             umma_ts(tmem + oc, tmem + C::SX_COL + sb * BLK + k * 8, sdesc_sw128(vb + k * 2048, BLK * 128, 1024), idO,
-                    (g_acc[e & 1] | uint32_t(k)) ? 1u : 0u);
-          g_acc[e & 1] = 1;
+                    (((g_acc >> (e & 1)) & 1u) | uint32_t(k)) ? 1u : 0u);
+          g_acc |= 1u << (e & 1);
         } else {
           // P of keys [16k, 16k + 16): half (k / (BLK/32)) of the row packed it at the
           // start of its own score columns
@@ -929,6 +933,9 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           float lsp[4] = {0.f, 0.f, 0.f, 0.f};
           float ssp[2] = {0.f, 0.f};
           uint32_t a0[C::CHUNK / 2];
+          // this row's packed alpha of the chunk, also in shared memory for the per-block
+          // lookups below (a register array held through the block loop lives in local memory)
+          uint32_t* a0s = reinterpret_cast<uint32_t*>(base + C::OFF_A0) + r * C::A0_LD;
 #pragma unroll
           for (int k = 0; k < C::CHUNK; k += 2) {
             const float x0 = ex2(__uint_as_float(sv[k]) - m);
@@ -942,13 +949,22 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             lsp[(k >> 1) & 3] = fmaf(n1, r1, fmaf(n0, r0, lsp[(k >> 1) & 3]));
             if (hybrid) ssp[(k >> 1) & 1] += r0 + r1;
             a0[k >> 1] = w;
+            a0s[k >> 1] = w;
           }
           l += (lsp[0] + lsp[1]) + (lsp[2] + lsp[3]);
           s_alpha += ssp[0] + ssp[1];
           // alpha of blocks [16k, 16k + 16) at columns [16k, 16k + 8) (the layout the
           // zeroth-order MMA reads)
-          tmem_st8(sa, *reinterpret_cast<const uint32_t(*)[8]>(&a0[0]));
-          tmem_st8(sa + 16, *reinterpret_cast<const uint32_t(*)[8]>(&a0[8]));
+          {
+            uint32_t lo[8], hi[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              lo[i] = a0[i];
+              hi[i] = a0[8 + i];
+            }
+            tmem_st8(sa, lo);
+            tmem_st8(sa + 16, hi);
+          }
           tmem_wait_st();
           tc_fence_before();
           warp_arrive(BAR(C::B_A0F + b));
@@ -966,7 +982,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
 #pragma unroll 1
             for (int qq = 0; qq < n; ++qq) {
               const int k = approx_list[a + qq] - c * C::CHUNK;
-              const uint32_t w = a0[k >> 1];
+              const uint32_t w = a0s[k >> 1];
               const float coef = ((k & 1) ? bf16_hi(w) : bf16_lo(w)) * p.scale;
               const __nv_bfloat162 c2 = __floats2bfloat162_rn(coef, coef);
               const uint32_t cw = *reinterpret_cast<const uint32_t*>(&c2);
