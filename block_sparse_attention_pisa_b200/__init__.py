@@ -335,7 +335,7 @@ def head_chunks(BH: int, chunks: int):
     return [(edges[c], edges[c + 1]) for c in range(chunks) if edges[c + 1] > edges[c]]
 
 
-def host_workspace_bytes(shape: Shape, topk: int, order: int, route_lambda: float = 0.0, chunks: int = 8,
+def host_workspace_bytes(shape: Shape, topk: int, order: int, route_lambda: float = 0.0, chunks: int = 0,
                          group: int = 1, candidates: int = 0) -> int:
     """Device workspace (bytes) that ``pisa_host`` needs for this problem."""
     n = ctypes.c_size_t(0)
@@ -345,7 +345,7 @@ def host_workspace_bytes(shape: Shape, topk: int, order: int, route_lambda: floa
 
 
 def pisa_host(Q, K, V, block: int, topk: int, order: int = 1, scale: float | None = None,
-              device="cuda", route_lambda: float = 0.0, chunks: int = 8, out=None,
+              device="cuda", route_lambda: float = 0.0, chunks: int = 0, out=None,
               group: int = 1, candidates: int = 0):
     """The whole path on HOST tensors [B, H, N, d] through the C ABI's ``pisa_run_host``:
     the library copies Q, K, V to the device, runs the path and copies O back, pipelined
@@ -382,7 +382,7 @@ def pisa_host(Q, K, V, block: int, topk: int, order: int = 1, scale: float | Non
 
 
 def pisa_host_static(Q, K, V, block: int, topk: int, order: int = 1, scale: float | None = None,
-                     device="cuda", route_lambda: float = 0.0, chunks: int = 8, out=None,
+                     device="cuda", route_lambda: float = 0.0, chunks: int = 0, out=None,
                      group: int = 1, candidates: int = 0):
     """``pisa_host`` through the C ABI's ``pisa_run_host_static``: the device workspace is
     the library's fixed region (``STATIC_WORKSPACE_BYTES`` per device) and nothing is

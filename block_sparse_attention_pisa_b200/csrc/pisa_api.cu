@@ -539,7 +539,7 @@ pisa_status_t host_options(const pisa_shape_t& s, int32_t topk, const pisa_host_
   pisa_host_options_t o{0.f, 1, 0, 8};
   if (in != nullptr) o = *in;
   if (o.group == 0) o.group = 1;
-  if (o.chunks == 0) o.chunks = 8;
+  if (o.chunks == 0) o.chunks = 32;  // at most B*H ranges are used
   const int32_t nB = int32_t(num_blocks(s));
   if (o.candidates == 0) o.candidates = nB;
   if (!std::isfinite(o.route_lambda) || o.route_lambda < 0.f)
@@ -641,7 +641,9 @@ pisa_status_t pisa_run_host(const void* Q, const void* K, const void* V, pisa_sh
       pisa_host::slot_layout(pisa_host::range_size(BH, nc), shape.N, shape.d, nB, topk, order, routed);
   const size_t row_bytes = size_t(shape.N) * shape.d * 2;  // one (batch, head) slice of Q, K, V or O
   auto cs = static_cast<cudaStream_t>(stream);
-  cudaStream_t in_s = nullptr, out_s = nullptr;
+  // the ranges' kernels alternate between the caller's stream and one more, so that a
+  // range's first CTAs fill the SMs the previous range's last wave leaves idle
+  cudaStream_t in_s = nullptr, out_s = nullptr, cs2 = nullptr;
   std::vector<cudaEvent_t> ev;  // entry, then landed / computed / drained per range
   pisa_status_t st = PISA_OK;
   cudaError_t e = cudaSuccess;
@@ -655,7 +657,8 @@ pisa_status_t pisa_run_host(const void* Q, const void* K, const void* V, pisa_sh
   std::vector<cudaEvent_t> landed(nc), computed(nc), drained(nc);
   do {
     if ((e = cudaStreamCreateWithFlags(&in_s, cudaStreamNonBlocking)) != cudaSuccess ||
-        (e = cudaStreamCreateWithFlags(&out_s, cudaStreamNonBlocking)) != cudaSuccess) {
+        (e = cudaStreamCreateWithFlags(&out_s, cudaStreamNonBlocking)) != cudaSuccess ||
+        (e = cudaStreamCreateWithFlags(&cs2, cudaStreamNonBlocking)) != cudaSuccess) {
       st = cuda_fail("cudaStreamCreateWithFlags");
       break;
     }
@@ -663,12 +666,14 @@ pisa_status_t pisa_run_host(const void* Q, const void* K, const void* V, pisa_sh
     // users of the workspace)
     if (!event(&entry) || (e = cudaEventRecord(entry, cs)) != cudaSuccess ||
         (e = cudaStreamWaitEvent(in_s, entry, 0)) != cudaSuccess ||
-        (e = cudaStreamWaitEvent(out_s, entry, 0)) != cudaSuccess) {
+        (e = cudaStreamWaitEvent(out_s, entry, 0)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(cs2, entry, 0)) != cudaSuccess) {
       st = cuda_fail("entry event");
       break;
     }
     for (int c = 0; c < nc && st == PISA_OK; ++c) {
       const int64_t a = BH * c / nc, b = BH * (c + 1) / nc, n = b - a;
+      cudaStream_t ks = (c & 1) ? cs2 : cs;  // this range's kernels
       uint8_t* base = static_cast<uint8_t*>(workspace) + size_t(c % slots) * L.bytes;
       if (!event(&landed[c]) || !event(&computed[c]) || !event(&drained[c])) {
         st = cuda_fail("cudaEventCreate");
@@ -685,11 +690,11 @@ pisa_status_t pisa_run_host(const void* Q, const void* K, const void* V, pisa_sh
         e = cudaMemcpyAsync(base + dst[t], static_cast<const uint8_t*>(host[t]) + off, len, cudaMemcpyHostToDevice,
                             in_s);
       if (e != cudaSuccess || (e = cudaEventRecord(landed[c], in_s)) != cudaSuccess ||
-          (e = cudaStreamWaitEvent(cs, landed[c], 0)) != cudaSuccess) {
+          (e = cudaStreamWaitEvent(ks, landed[c], 0)) != cudaSuccess) {
         st = cuda_fail("copy-in");
         break;
       }
-      // the path on the caller's stream, for this range as a [1, n, N, d] problem
+      // the path on this range's kernel stream, as a [1, n, N, d] problem
       pisa_shape_t rs{1, int32_t(n), shape.N, shape.d, shape.block};
       float* kbar = reinterpret_cast<float*>(base + L.kbar);
       float* S0 = reinterpret_cast<float*>(base + L.s0);
@@ -699,23 +704,23 @@ pisa_status_t pisa_run_host(const void* Q, const void* K, const void* V, pisa_sh
       const void* first = order == PISA_ORDER_FIRST || order == PISA_ORDER_HYBRID ? S1 : nullptr;
       const float* route = nullptr;
       if ((st = pisa_block_stats(base + L.k, base + L.v, rs, stats_order, kbar, S0,
-                                 stats_order >= PISA_ORDER_FIRST ? S1 : nullptr, cs)) != PISA_OK)
+                                 stats_order >= PISA_ORDER_FIRST ? S1 : nullptr, ks)) != PISA_OK)
         break;
       if (routed) {
         float* hbar = reinterpret_cast<float*>(base + L.hbar);
         float* M = reinterpret_cast<float*>(base + L.m);
-        if ((st = pisa_routing_norms(S1, rs, hbar, M, cs)) != PISA_OK) break;
+        if ((st = pisa_routing_norms(S1, rs, hbar, M, ks)) != PISA_OK) break;
         route = M;
         if (order == PISA_ORDER_HYBRID) first = hbar;
       }
       if ((st = pisa_select_grouped(base + L.q, kbar, route, route_lambda, rs, topk, opt.group, opt.candidates, idx,
-                                    cs)) != PISA_OK)
+                                    ks)) != PISA_OK)
         break;
       if ((st = pisa_attention(base + L.q, base + L.k, base + L.v, kbar, S0, first, idx, rs, topk, order, scale,
-                               base + L.o, cs)) != PISA_OK)
+                               base + L.o, ks)) != PISA_OK)
         break;
       // copy out, once the range's kernels are done
-      if ((e = cudaEventRecord(computed[c], cs)) != cudaSuccess ||
+      if ((e = cudaEventRecord(computed[c], ks)) != cudaSuccess ||
           (e = cudaStreamWaitEvent(out_s, computed[c], 0)) != cudaSuccess ||
           (e = cudaMemcpyAsync(static_cast<uint8_t*>(O) + off, base + L.o, len, cudaMemcpyDeviceToHost, out_s)) !=
               cudaSuccess ||
@@ -727,9 +732,9 @@ pisa_status_t pisa_run_host(const void* Q, const void* K, const void* V, pisa_sh
   } while (false);
   // whatever happened, nothing may still run on the workspace or the host buffers when
   // the call returns
-  for (int i = 0; i < 3; ++i) {
-    cudaStream_t s = i == 0 ? in_s : (i == 1 ? out_s : cs);
-    if (i < 2 && s == nullptr) continue;  // a copy stream that was never created
+  for (int i = 0; i < 4; ++i) {
+    cudaStream_t s = i == 0 ? in_s : (i == 1 ? out_s : (i == 2 ? cs2 : cs));
+    if (i < 3 && s == nullptr) continue;  // an internal stream that was never created
     cudaError_t se = cudaStreamSynchronize(s);
     if (se != cudaSuccess && st == PISA_OK) {
       e = se;
@@ -739,6 +744,7 @@ pisa_status_t pisa_run_host(const void* Q, const void* K, const void* V, pisa_sh
   for (cudaEvent_t x : ev) cudaEventDestroy(x);
   if (in_s) cudaStreamDestroy(in_s);
   if (out_s) cudaStreamDestroy(out_s);
+  if (cs2) cudaStreamDestroy(cs2);
   return st;
 }
 

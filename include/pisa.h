@@ -194,7 +194,7 @@ typedef struct {
   float route_lambda;  /* 0 (default): plain relevance; > 0: covariance-aware routing weight */
   int32_t group;       /* query blocks per proxy query for the selection (default / 0: 1)     */
   int32_t candidates;  /* proxy candidate-list length (default / 0: every key block)           */
-  int32_t chunks;      /* (batch, head) ranges pipelined through the workspace (default / 0: 8) */
+  int32_t chunks;      /* (batch, head) ranges pipelined through the workspace (default / 0: 32) */
 } pisa_host_options_t;
 
 /*
@@ -214,8 +214,10 @@ pisa_status_t pisa_run_host_workspace(pisa_shape_t shape, int32_t topk, int32_t 
  * Section 2 of the explainer, "Hardware implementation": a precompute step, routing,
  * then the fused kernel. Every step is independent across (batch, head) pairs, so the
  * call splits the B*H pairs into `chunks` contiguous ranges and pipelines them through
- * the workspace on three streams: the host-to-device copy of a range, the kernels of
- * the previous one (on `stream`) and the device-to-host copy of the one before overlap.
+ * the workspace: the host-to-device copy of a range, the kernels of the ranges before it
+ * and the device-to-host copy of earlier ones overlap. The ranges' kernels alternate
+ * between `stream` and one internal stream, so one range's first CTAs fill the SMs the
+ * previous range's last wave leaves idle; the copies run on two more internal streams.
  * The result is bit for bit that of the device calls on the whole batch.
  * Q, K, V: HOST bf16 [B, H, N, d] (page-locked memory lets the copies overlap the
  * kernels; pageable memory works, with less overlap); O: HOST bf16 [B, H, N, d],

@@ -210,7 +210,7 @@ def test_host_workspace_size(L):
     assert st == OK and n0 == 4 * up(24 * N * d * 2) + 2 * up(24 * nB * d * 4) + up(24 * nB * k * 4)
     assert _ws(L, shape(N=0)) == (OK, 0)
     assert _ws(L, chunks=-1)[0] == INVALID
-    assert _ws(L, chunks=0) == _ws(L, chunks=8)             # 0: the default
+    assert _ws(L, chunks=0) == _ws(L, chunks=32)            # 0: the default
     assert _ws(L, lam=-1.0)[0] == INVALID
     assert _ws(L, order=5)[0] == INVALID
     assert _ws(L, topk=9)[0] == INVALID
