@@ -507,7 +507,7 @@ def run_ours(args):
         **({"routing_gbs": R.routing_bytes(wl.B, wl.H, wl.N, wl.d, wl.block) / (k_ms["routing"] * 1e-3) / 1e9}
            if routed else {}),
         "e2e": e2e, "cpu_baseline": cpu, "near_ties": near,
-        "gpu_launches": (6 if routed else 3) * args.steps, "clocks": clocks,
+        "gpu_launches": (5 if routed else 3) * args.steps, "clocks": clocks,
         "attention_kernel": args.kernel,
     }
     print(json.dumps(line), flush=True)

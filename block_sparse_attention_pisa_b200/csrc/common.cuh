@@ -63,6 +63,32 @@ __device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, uint
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// ---------------------------------------------------------------- thread-block clusters
+// Head statistics reduced inside a cluster: each CTA stages its partial in its own
+// shared memory, and after one cluster barrier every CTA reads its share of all
+// partials through distributed shared memory.
+constexpr int kHbarCluster = 4;  // CTAs per head for the hybrid-order statistic
+
+// every thread of every CTA of the cluster arrives (release) and waits (acquire);
+// each thread must reach it, so no role may leave its loop without coming here
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// shared::cta address of this CTA -> shared::cluster address of the same offset in CTA `rank`
+__device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
 // Order-preserving map of a float to uint32 (larger float -> larger key). -0 is
 // folded onto +0 by the caller (x + 0.0f) so equal scores map to equal keys.
 __device__ __forceinline__ uint32_t float_order_key(float x) {

@@ -147,43 +147,72 @@ pisa_status_t launch_stats_mode(const pisa_shape_t& s, const bf16* K, const bf16
 pisa_status_t make_map(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box1);
 pisa_status_t make_plane_map(CUtensorMap* m, const float* kbar, uint64_t D, uint64_t nB, uint64_t BH, uint32_t rows);
 
-// d = 128, orders 1 and 2: the tensor-core statistics kernel (persistent, one CTA per SM)
-template <int BLK, int MODE>
+// d = 128, order 1: the tensor-core statistics kernel (persistent, one CTA per SM)
+template <int BLK>
 pisa_status_t launch_stats_tc(const pisa_shape_t& s, const bf16* K, const bf16* V, float* kbar, float* S0, bf16* S1,
-                              float* Hbar, int sms, cudaStream_t st) {
-  using C = pisa::StatsTcCfg<BLK, MODE>;
+                              int sms, cudaStream_t st) {
+  using C = pisa::StatsTcCfg<BLK>;
   const int nB = int(num_blocks(s));
   const uint64_t BH = uint64_t(s.B) * s.H;
   CUtensorMap mK, mV, mS;
   PISA_TRY(make_map(&mK, K, 128, uint64_t(s.N), BH, BLK));
   PISA_TRY(make_map(&mV, V, 128, uint64_t(s.N), BH, BLK));
-  if (MODE == pisa::kStatsS1) PISA_TRY(make_map(&mS, S1, 128, 128, BH * nB, 128));
-  else mS = mK;  // never used in Hbar mode
-  auto k = pisa::stats_tc_kernel<BLK, MODE>;
+  PISA_TRY(make_map(&mS, S1, 128, 128, BH * nB, 128));
+  auto k = pisa::stats_tc_kernel<BLK>;
   PISA_TRY(set_smem(k, C::SMEM));
-  const int uph = (nB + C::UNIT - 1) / C::UNIT;
-  const int64_t total = int64_t(BH) * uph;
-  if (total > (int64_t(1) << 30)) return fail(PISA_ERR_UNSUPPORTED, "too many statistics units");
+  const int64_t total = int64_t(BH) * nB;
+  if (total > (int64_t(1) << 30)) return fail(PISA_ERR_UNSUPPORTED, "too many statistics blocks");
   const int grid = int(total < sms ? total : sms);
-  k<<<grid, C::kThreads, C::SMEM, st>>>(mK, mV, mS, s.N, nB, uph, int(total), kbar, S0, Hbar);
+  k<<<grid, C::kThreads, C::SMEM, st>>>(mK, mV, mS, s.N, nB, int(total), kbar, S0);
   return check_launch("stats_tc_kernel");
+}
+
+// Hbar: one cluster of kHbarCluster CTAs per head, grid (kHbarCluster, B*H)
+template <typename Kernel, typename... Args>
+pisa_status_t launch_hbar_clusters(Kernel k, const pisa_shape_t& s, int threads, size_t smem, cudaStream_t st,
+                                   const char* what, Args... args) {
+  PISA_TRY(set_smem(k, smem));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pisa::kHbarCluster, unsigned(s.B) * unsigned(s.H), 1);
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = pisa::kHbarCluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, k, args...);
+  if (e != cudaSuccess) return fail(PISA_ERR_CUDA, "%s launch: %s", what, cudaGetErrorString(e));
+  return check_launch(what);
 }
 
 template <int D, int BLK>
 pisa_status_t launch_stats(const pisa_shape_t& s, const bf16* K, const bf16* V, int order, float* kbar,
                            float* S0, void* S1, int sms, cudaStream_t st) {
   if (order == PISA_ORDER_HYBRID) {
-    // Hbar is accumulated with atomics: zero it first, on the same stream
-    const size_t bytes = size_t(s.B) * s.H * D * D * sizeof(float);
-    cudaError_t e = cudaMemsetAsync(S1, 0, bytes, st);
-    if (e != cudaSuccess) return fail(PISA_ERR_CUDA, "cudaMemsetAsync(Hbar): %s", cudaGetErrorString(e));
-    if (D == 128)
-      return launch_stats_tc<BLK, pisa::kStatsHbar>(s, K, V, kbar, S0, nullptr, static_cast<float*>(S1), sms, st);
-    return launch_stats_mode<D, BLK, pisa::kStatsHbar>(s, K, V, kbar, S0, nullptr, static_cast<float*>(S1), st);
+    // every element of Hbar is stored once (no zeroing, no atomics)
+    float* Hbar = static_cast<float*>(S1);
+    const int nB = int(num_blocks(s));
+    if constexpr (D == 128) {
+      using C = pisa::StatsHbarCfg<BLK>;
+      const uint64_t BH = uint64_t(s.B) * s.H;
+      CUtensorMap mK, mV;
+      PISA_TRY(make_map(&mK, K, 128, uint64_t(s.N), BH, BLK));
+      PISA_TRY(make_map(&mV, V, 128, uint64_t(s.N), BH, BLK));
+      return launch_hbar_clusters(pisa::stats_hbar_kernel<BLK>, s, C::kThreads, size_t(C::SMEM), st,
+                                  "stats_hbar_kernel", mK, mV, s.N, nB, kbar, S0, Hbar);
+    } else {
+      using P = pisa::StatsPipeCfg<D, BLK>;
+      return launch_hbar_clusters(pisa::stats_pipe_kernel<D, BLK, pisa::kStatsHbar>, s,
+                                  pisa::StatsCfg<D, BLK>::kThreads, P::kSmem, st, "stats_pipe_kernel", K, V, s.N,
+                                  nB, kbar, S0, static_cast<bf16*>(nullptr), Hbar);
+    }
   }
   if (order == PISA_ORDER_FIRST) {
-    if (D == 128)
-      return launch_stats_tc<BLK, pisa::kStatsS1>(s, K, V, kbar, S0, static_cast<bf16*>(S1), nullptr, sms, st);
+    if (D == 128) return launch_stats_tc<BLK>(s, K, V, kbar, S0, static_cast<bf16*>(S1), sms, st);
     return launch_stats_mode<D, BLK, pisa::kStatsS1>(s, K, V, kbar, S0, static_cast<bf16*>(S1), nullptr, st);
   }
   return launch_stats_mode<D, BLK, pisa::kStatsSums>(s, K, V, kbar, S0, nullptr, nullptr, st);
@@ -275,19 +304,14 @@ pisa_status_t launch_select(const pisa_shape_t& s, const bf16* Q, const float* k
 pisa_status_t launch_routing(const pisa_shape_t& s, const bf16* S1, float* Hbar, float* M, cudaStream_t st) {
   const int nB = int(num_blocks(s));
   const int dd = s.d * s.d;
-  const size_t BH = size_t(s.B) * s.H;
-  cudaError_t e;
-  if ((e = cudaMemsetAsync(Hbar, 0, BH * dd * sizeof(float), st)) != cudaSuccess ||
-      (e = cudaMemsetAsync(M, 0, BH * nB * sizeof(float), st)) != cudaSuccess)
-    return fail(PISA_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
-  dim3 grid(dd / pisa::kRouteSlice, (nB + pisa::kRouteChunk - 1) / pisa::kRouteChunk, unsigned(BH));
-  pisa::routing_hbar_kernel<<<grid, pisa::kRouteThreads, 0, st>>>(S1, nB, dd, Hbar);
+  const unsigned BH = unsigned(s.B) * unsigned(s.H);
+  // every element of Hbar and M is stored once (no zeroing, no atomics)
+  pisa::routing_hbar_kernel<<<dim3(dd / pisa::kRouteSlice, BH), pisa::kRouteThreads, 0, st>>>(S1, nB, dd, Hbar);
   PISA_TRY(check_launch("routing_hbar_kernel"));
-  pisa::routing_norm_kernel<<<grid, pisa::kRouteThreads, 0, st>>>(S1, Hbar, nB, dd, M);
-  PISA_TRY(check_launch("routing_norm_kernel"));
-  const size_t n = BH * nB;
-  pisa::routing_sqrt_kernel<<<unsigned((n + 255) / 256), 256, 0, st>>>(M, n);
-  return check_launch("routing_sqrt_kernel");
+  const dim3 grid((nB + pisa::kRouteChunk - 1) / pisa::kRouteChunk, BH);
+  if (s.d == 128) pisa::routing_norm_kernel<128><<<grid, pisa::kRouteThreads, 0, st>>>(S1, Hbar, nB, M);
+  else pisa::routing_norm_kernel<64><<<grid, pisa::kRouteThreads, 0, st>>>(S1, Hbar, nB, M);
+  return check_launch("routing_norm_kernel");
 }
 
 template <int D>

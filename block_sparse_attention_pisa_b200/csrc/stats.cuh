@@ -23,10 +23,14 @@
 //
 // Hybrid order (section 2, "Core algorithm": one global first-order statistic
 // Hbar, the mean of the per-block first-order matrices over all blocks of a head;
-// "Hardware implementation": formed in the precompute step). The CTA keeps the
-// sum of its blocks' S1_j (fp32) in registers and adds it, scaled by 1/nB, into
-// the fp32 Hbar of the head with vector atomics. Per-block S1 is never written.
-// The fp32 atomic sum makes Hbar reproducible to fp32 rounding, not bit for bit.
+// "Hardware implementation": formed in the precompute step). A cluster of
+// kHbarCluster CTAs takes one head, CTA r the contiguous blocks
+// [r nB / G, (r + 1) nB / G); each keeps the sum of its blocks' S1_j (fp32) in
+// registers and stages it in its idle tile buffers. After a cluster barrier, CTA r
+// sums its share of the rows over the G partials in rank order (distributed shared
+// memory), scales by 1/nB and stores them. The split and every summation order depend
+// on nB alone, so Hbar is the same bit for bit for any B, H, stream or device, and it
+// needs no zeroing. Per-block S1 is never written.
 #pragma once
 
 #include "common.cuh"
@@ -131,8 +135,9 @@ stats_pipe_kernel(const bf16* __restrict__ K, const bf16* __restrict__ V, int N,
   const int r0 = tid / C::kChunks;
   const int a_base = (warp >> 1) * TM;
   const int g = lane >> 2, t4 = lane & 3;
-  const int j0 = blockIdx.x * G;
-  const int j1 = min(nB, j0 + G);
+  // Hbar mode: the grid's x extent is the cluster, and x is the CTA's rank in it
+  const int j0 = MODE == kStatsHbar ? int((int64_t(blockIdx.x) * nB) / kHbarCluster) : int(blockIdx.x) * G;
+  const int j1 = MODE == kStatsHbar ? int((int64_t(blockIdx.x + 1) * nB) / kHbarCluster) : min(nB, j0 + G);
   const uint32_t buf_u = smem_u32(sBuf);
 
   // copies of block j into buffer b: thread (ch, r0) takes 16-byte chunk ch of rows
@@ -299,9 +304,11 @@ stats_pipe_kernel(const bf16* __restrict__ K, const bf16* __restrict__ V, int N,
     __syncthreads();  // this block's buffer, sums and staging tile are free again
   }
 
-  if (MODE == kStatsHbar && j0 < j1) {
-    const float inv = 1.f / float(nB);
-    float* gH = Hbar + bh * size_t(D) * D;
+  if (MODE == kStatsHbar) {
+    // the CTA's partial (zero for an empty slice) -> its idle tile buffers, [D][D + 4] fp32
+    constexpr int PD = D + 4;
+    static_assert(size_t(D) * PD * 4 <= size_t(4) * P::kTileBytes, "partial staging");
+    float* sP = reinterpret_cast<float*>(smem_raw);
 #pragma unroll
     for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -310,11 +317,30 @@ stats_pipe_kernel(const bf16* __restrict__ K, const bf16* __restrict__ V, int N,
         for (int nt = 0; nt < NT; ++nt) {
           const int a = a_base + mt * 16 + g;
           const int c = h * (D / 2) + (warp & 1) * TN + nt * 8 + 2 * t4;
-          atomicAdd(reinterpret_cast<float2*>(gH + size_t(a) * D + c),
-                    make_float2(acc[h][mt][nt][0] * inv, acc[h][mt][nt][1] * inv));
-          atomicAdd(reinterpret_cast<float2*>(gH + size_t(a + 8) * D + c),
-                    make_float2(acc[h][mt][nt][2] * inv, acc[h][mt][nt][3] * inv));
+          *reinterpret_cast<float2*>(sP + a * PD + c) = make_float2(acc[h][mt][nt][0], acc[h][mt][nt][1]);
+          *reinterpret_cast<float2*>(sP + (a + 8) * PD + c) = make_float2(acc[h][mt][nt][2], acc[h][mt][nt][3]);
         }
+    cluster_sync_all();  // every partial of the cluster is staged
+    constexpr int ROWS = D / kHbarCluster;
+    const int rank = int(blockIdx.x);
+    const float inv = 1.f / float(nB);
+    float* gH = Hbar + bh * size_t(D) * D;
+    for (int i = tid; i < ROWS * (D / 4); i += C::kThreads) {
+      const int a = rank * ROWS + i / (D / 4), q = i % (D / 4);
+      const uint32_t off = smem_u32(sP + a * PD + 4 * q);
+      float4 sum = ld_cluster_f4(cluster_map(off, 0));
+#pragma unroll
+      for (int src = 1; src < kHbarCluster; ++src) {
+        const float4 v = ld_cluster_f4(cluster_map(off, uint32_t(src)));
+        sum.x += v.x;
+        sum.y += v.y;
+        sum.z += v.z;
+        sum.w += v.w;
+      }
+      *reinterpret_cast<float4*>(gH + size_t(a) * D + 4 * q) =
+          make_float4(sum.x * inv, sum.y * inv, sum.z * inv, sum.w * inv);
+    }
+    cluster_sync_all();  // no CTA leaves while another still reads its partial
   }
 }
 

@@ -92,9 +92,11 @@ typedef struct {
  *   Hbar   = (1/nB) sum_j S1_j                        fp32  [B, H, d, d]
  * K, V: bf16 [B, H, N, d]. order (-1, 0, 1 or 2) selects what the S1 argument receives:
  *   order 1: S1 = the per-block matrices, bf16 [B, H, nB, d, d];
- *   order 2: S1 = Hbar, fp32 [B, H, d, d]. The call zeroes it on `stream`, then
- *            accumulates it with fp32 atomics (reproducible to fp32 rounding, not bit
- *            for bit); per-block S1 is not written;
+ *   order 2: S1 = Hbar, fp32 [B, H, d, d], every element stored once (it need not be
+ *            zeroed); per-block S1 is not written. A cluster of 4 CTAs per head takes
+ *            the head's blocks in 4 contiguous slices and adds the 4 partial sums in
+ *            a fixed order, without atomics, so the result depends only on K, V, N,
+ *            d and b: the same bits for any B, H, stream or device;
  *   order 0, -1: S1 is not touched and may be NULL.
  */
 pisa_status_t pisa_block_stats(const void* K, const void* V, pisa_shape_t shape, int32_t order,
@@ -144,8 +146,8 @@ pisa_status_t pisa_select_grouped(const void* Q, const float* kbar, const float*
  * (the pages write a 2-norm without naming it; this is the Frobenius norm). S1 is the
  * per-block bf16 output of pisa_block_stats at order 1, read as stored, so this Hbar
  * is the mean of the stored bf16 matrices; it serves as the Hbar argument of
- * pisa_attention at order 2 as well. Hbar and M are overwritten (zeroed on `stream`,
- * then accumulated with fp32 atomics: reproducible to fp32 rounding).
+ * pisa_attention at order 2 as well. Hbar and M are overwritten, each element stored
+ * once after sums taken in a fixed order (no atomics): the same bits on every call.
  */
 pisa_status_t pisa_routing_norms(const void* S1, pisa_shape_t shape, float* Hbar, float* M,
                                  void* stream);
@@ -248,8 +250,7 @@ pisa_status_t pisa_run_host(const void* Q, const void* K, const void* V, pisa_sh
  * figure exceeds the region is rejected with PISA_ERR_UNSUPPORTED before anything runs
  * (more `chunks` make each range, and the figure, smaller).
  * Nothing in the region has to start at zero: every byte the path reads there was
- * written earlier in the same call (statistics that accumulate are zeroed on the
- * stream first).
+ * written earlier in the same call.
  * The region is ONE PER DEVICE, shared by every call on that device: calls that overlap
  * in time (from other host threads, or on other streams) race on it, and the caller
  * must serialise them. Each call blocks until it is done, so consecutive calls from one
