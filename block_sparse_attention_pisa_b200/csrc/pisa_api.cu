@@ -306,7 +306,7 @@ pisa_status_t launch_routing(const pisa_shape_t& s, const bf16* S1, float* Hbar,
   const int dd = s.d * s.d;
   const unsigned BH = unsigned(s.B) * unsigned(s.H);
   // every element of Hbar and M is stored once (no zeroing, no atomics)
-  pisa::routing_hbar_kernel<<<dim3(dd / pisa::kRouteSlice, BH), pisa::kRouteThreads, 0, st>>>(S1, nB, dd, Hbar);
+  pisa::routing_hbar_kernel<<<dim3(dd / pisa::kHbarSlice, BH), pisa::kHbarThreads, 0, st>>>(S1, nB, dd, Hbar);
   PISA_TRY(check_launch("routing_hbar_kernel"));
   const dim3 grid((nB + pisa::kRouteChunk - 1) / pisa::kRouteChunk, BH);
   if (s.d == 128) pisa::routing_norm_kernel<128><<<grid, pisa::kRouteThreads, 0, st>>>(S1, Hbar, nB, M);

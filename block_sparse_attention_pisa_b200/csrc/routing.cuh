@@ -10,10 +10,10 @@
 //
 // Both kernels stream the per-block S1 of a head once, and every sum runs in a fixed
 // order (no atomics), so Hbar and M are the same bit for bit on every call:
-//   routing_hbar_kernel: grid (slice, head); a slice is 2048 consecutive elements of the
-//                        d x d matrix, 8 per thread (one 16-byte load per block); each
-//                        thread sums its elements over all blocks j = 0 .. nB - 1 in
-//                        turn, then Hbar = sum / nB;
+//   routing_hbar_kernel: grid (slice, head); a slice is 1024 consecutive elements of the
+//                        d x d matrix, 8 per thread (one 16-byte load per block, 16 blocks
+//                        in flight); each thread sums its elements over all blocks
+//                        j = 0 .. nB - 1 in turn, then Hbar = sum / nB;
 //   routing_norm_kernel: grid (chunk of kRouteChunk blocks, head); per block, each
 //                        thread sums (S1_j - Hbar)^2 over its D*D/256 elements, the
 //                        warps reduce by shuffles, and after one CTA barrier thread jj
@@ -24,28 +24,38 @@
 
 namespace pisa {
 
-constexpr int kRouteThreads = 256;
-constexpr int kRouteSlice = kRouteThreads * 8;  // matrix elements per Hbar CTA
+constexpr int kRouteThreads = 256;              // norm kernel
+constexpr int kRouteSlice = kRouteThreads * 8;  // matrix elements per norm-kernel pass
 constexpr int kRouteChunk = 16;                 // key blocks per norm CTA
+constexpr int kHbarThreads = 128;               // Hbar kernel
+constexpr int kHbarSlice = kHbarThreads * 8;    // matrix elements per Hbar CTA
 
-__global__ void __launch_bounds__(kRouteThreads)
+__global__ void __launch_bounds__(kHbarThreads)
 routing_hbar_kernel(const bf16* __restrict__ S1, int nB, int dd, float* __restrict__ Hbar) {
-  const int e0 = blockIdx.x * kRouteSlice + threadIdx.x * 8;  // first element of this thread
+  const int e0 = blockIdx.x * kHbarSlice + threadIdx.x * 8;  // first element of this thread
   const size_t bh = blockIdx.y;
   const bf16* src = S1 + (bh * size_t(nB)) * dd + e0;
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-#pragma unroll 8
-  for (int j = 0; j < nB; ++j) {
-    const uint4 w = ldg_stream_v4(src + size_t(j) * dd);
+  auto add = [&](const uint4& w) {
     const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       acc[2 * e] += bf16_lo(ww[e]);
       acc[2 * e + 1] += bf16_hi(ww[e]);
     }
+  };
+  // 16 blocks' loads in flight, then their sums in block order
+  int j = 0;
+  for (; j + 16 <= nB; j += 16) {
+    uint4 w[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) w[u] = __ldg(reinterpret_cast<const uint4*>(src + size_t(j + u) * dd));
+#pragma unroll
+    for (int u = 0; u < 16; ++u) add(w[u]);
   }
+  for (; j < nB; ++j) add(ldg_stream_v4(src + size_t(j) * dd));
   const float inv = 1.f / float(nB);
   float4* dst = reinterpret_cast<float4*>(Hbar + bh * size_t(dd) + e0);
   dst[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
