@@ -103,6 +103,13 @@ struct TcCfg {
   static constexpr int CHUNK = 32;                          // key blocks per approximate chunk
   static constexpr int CV_HALF = CHUNK * D * 2;             // bf16 kbar (or S0) chunk
   static constexpr int CV_STAGE = 2 * CV_HALF;
+  // conversion stages: two of their own; at orders 0 and 2 two more in ring stage 1,
+  // which no copy uses once the exact stage is done
+  static constexpr int NCV_MAX = 4;
+  static_assert(2 * CV_STAGE <= STAGE && NS >= 2, "two conversion stages in ring stage 1");
+  __host__ __device__ static constexpr int cv_off(int s) {
+    return s < 2 ? OFF_CV + s * CV_STAGE : OFF_RING + STAGE + (s - 2) * CV_STAGE;
+  }
   static constexpr int GROUP = 2;                           // approximated blocks per hand-off
   static constexpr int NA = 2 * GROUP;                      // A operand slots (two groups)
   // exact score buffers. At d = 128 as many as the columns after Q hold (the approximate
@@ -135,16 +142,16 @@ struct TcCfg {
   static constexpr int B_SF = B_Q + 1;            // [NSB] S ready (commit)
   static constexpr int B_PF = B_SF + NSB;         // [NSB] P written (8 row warps)
   static constexpr int B_PV = B_PF + NSB;         // [NSB] P V done (commit)
-  static constexpr int B_CVF = B_PV + NSB;        // [2]   kbar / S0 chunk converted (2 warps)
-  static constexpr int B_CVE = B_CVF + 2;         // [2]   chunk operands consumed (commit)
-  static constexpr int B_SBF = B_CVE + 2;         // [2]   Sbar ready (commit)
+  static constexpr int B_CVF = B_PV + NSB;        // [4]   kbar / S0 chunk converted (2 warps)
+  static constexpr int B_CVE = B_CVF + NCV_MAX;   // [4]   chunk operands consumed (commit)
+  static constexpr int B_SBF = B_CVE + NCV_MAX;   // [2]   Sbar ready (commit)
   static constexpr int B_A0F = B_SBF + 2;         // [2]   alpha operand written (8 warps)
   static constexpr int B_SBE = B_A0F + 2;         // [2]   alpha MMA done (commit)
   static constexpr int B_GA = B_SBE + 2;          // [2]   a pair of A_j written (8 warps)
   static constexpr int B_AE = B_GA + 2;           // [2]   a pair of A_j consumed (commit)
   static constexpr int B_OSYNC = B_AE + 2;        //       end of the exact stage / of a chunk (commit)
   static constexpr int B_ODONE = B_OSYNC + 1;     //       all MMAs done (commit)
-  static constexpr int B_XD = B_ODONE + 1;        //       exact stage done, ring idle (commit; hybrid)
+  static constexpr int B_XD = B_ODONE + 1;        //       exact stage done, ring idle (commit; orders 0, 2)
   static constexpr int B_HF = B_XD + 1;           //       Hbar operand converted (4 warps; hybrid)
   static constexpr int B_AH = B_HF + 1;           //       A_H = s x written (4 warps; hybrid)
   static constexpr int B_MG = B_AH + 1;           //       group accumulators merged (8 row warps; GROUPS)
@@ -220,6 +227,48 @@ __device__ __forceinline__ void rescale_row(uint32_t taddr, float f) {
   tmem_wait_st();
 }
 
+// One approximate chunk's kbar and S0 (fp32 [rows][D], `rows` real blocks, the rest
+// zero) -> bf16 UMMA operands at dk (kbar) and dk + CHUNK*D*2 (S0): [CHUNK blocks][D]
+// row-major, 128-byte rows per 64-column panel, 16-byte chunks swizzled by (row % 8).
+// The K-major (kbar) and MN-major (S0) operand layouts coincide for this storage.
+// Thread ct of NT takes 16-byte output chunks ct, ct + NT, ...; the loads of a batch are
+// all issued before the first conversion (one L2 round trip per batch).
+template <int D, int CHUNK, int NT, int BATCH>
+__device__ __forceinline__ void convert_chunk(uint8_t* dk, const float* gk, const float* gs, int rows, int ct) {
+  constexpr int ITEMS = CHUNK * (D / 8) / NT;
+  static_assert(ITEMS * NT == CHUNK * (D / 8) && ITEMS % BATCH == 0, "converter items");
+  uint8_t* ds = dk + CHUNK * D * 2;
+#pragma unroll 1
+  for (int b0 = 0; b0 < ITEMS; b0 += BATCH) {
+    float4 kf[BATCH][2], sf[BATCH][2];
+#pragma unroll
+    for (int i = 0; i < BATCH; ++i) {
+      const int q = ct + (b0 + i) * NT;
+      const int r = q / (D / 8), c16 = q % (D / 8);
+      if (r < rows) {
+        kf[i][0] = __ldg(reinterpret_cast<const float4*>(gk + r * D + c16 * 8));
+        kf[i][1] = __ldg(reinterpret_cast<const float4*>(gk + r * D + c16 * 8 + 4));
+        sf[i][0] = __ldg(reinterpret_cast<const float4*>(gs + r * D + c16 * 8));
+        sf[i][1] = __ldg(reinterpret_cast<const float4*>(gs + r * D + c16 * 8 + 4));
+      } else {
+        kf[i][0] = kf[i][1] = sf[i][0] = sf[i][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < BATCH; ++i) {
+      const int q = ct + (b0 + i) * NT;
+      const int r = q / (D / 8), c16 = q % (D / 8);
+      const uint4 kv = make_uint4(pack_bf16x2(kf[i][0].x, kf[i][0].y), pack_bf16x2(kf[i][0].z, kf[i][0].w),
+                                  pack_bf16x2(kf[i][1].x, kf[i][1].y), pack_bf16x2(kf[i][1].z, kf[i][1].w));
+      const uint4 sv = make_uint4(pack_bf16x2(sf[i][0].x, sf[i][0].y), pack_bf16x2(sf[i][0].z, sf[i][0].w),
+                                  pack_bf16x2(sf[i][1].x, sf[i][1].y), pack_bf16x2(sf[i][1].z, sf[i][1].w));
+      const int off = (c16 >> 3) * (CHUNK * 128) + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
+      *reinterpret_cast<uint4*>(dk + off) = kv;
+      *reinterpret_cast<uint4*>(ds + off) = sv;
+    }
+  }
+}
+
 }  // namespace tc
 
 template <int D, int BLK>
@@ -262,9 +311,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       mbar_init(BAR(C::B_PF + s), C::GROUPS ? kRowWarps / 2 : kRowWarps);  // a group, or both halves
       mbar_init(BAR(C::B_PV + s), 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < C::NCV_MAX; ++s) {
       mbar_init(BAR(C::B_CVF + s), 2);
       mbar_init(BAR(C::B_CVE + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(BAR(C::B_SBF + s), 1);
       mbar_init(BAR(C::B_A0F + s), kApproxWarps);
       mbar_init(BAR(C::B_SBE + s), 1);
@@ -361,6 +412,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   const int n_exact = misc[2];
   const int n_active = misc[4];
   const bool hybrid = p.order == 2 && n_active > 0;
+  // orders 0 and 2: four conversion stages (two in the idle ring), and each chunk's pooled
+  // scores are issued before the previous chunk's alpha is awaited
+  const bool deep = (p.order == 0 || p.order == 2) && n_active > 0;
+  const int ncv = deep ? C::NCV_MAX : 2;
 
   if (warp == 0) {
     // ----------------------------------------------------------- TMA producer
@@ -479,7 +534,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         if (ok && e + kLook < n_exact) ok = qk(e + kLook);
       }
       umma_commit(BAR(C::B_OSYNC));  // completion 0: end of the exact stage
-      if (hybrid) umma_commit(BAR(C::B_XD));
+      if (deep) umma_commit(BAR(C::B_XD));
 
       if (ok && n_active > 0) {
         // the pooled-score and operand columns reuse the exact score buffers (and, with two
@@ -489,11 +544,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         else
           ok = wait_poll(BAR(C::B_PV + (n_exact - 1) % C::NSB), ((n_exact - 1) / C::NSB) & 1, abort_flag);
         auto sbar = [&](int ac) -> bool {
-          const int b = ac & 1;
-          if (!wait_poll(BAR(C::B_CVF + b), (ac >> 1) & 1, abort_flag)) return false;
+          const int b = ac & 1, cs = ac % ncv;
+          if (!wait_poll(BAR(C::B_CVF + cs), (ac / ncv) & 1, abort_flag)) return false;
           if (ac >= 2 && !wait_poll(BAR(C::B_SBE + b), ((ac - 2) >> 1) & 1, abort_flag)) return false;
           tc_fence_after();
-          const uint32_t kb = base_u + C::OFF_CV + b * C::CV_STAGE;
+          const uint32_t kb = base_u + C::cv_off(cs);
 #pragma unroll
           for (int k = 0; k < D / 16; ++k)
             umma_ts(tmem + C::R_COL + b * C::CHUNK, tmem + C::Q_COL + k * 8,
@@ -507,10 +562,14 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         int u = n_exact;         // load-unit counter
         for (int ac = 0; ac < n_active && ok; ++ac) {
           const int c = active[ac];
-          const int b = ac & 1;
+          const int b = ac & 1, cs = ac % ncv;
+          // deep: the next chunk's pooled scores first, so that they are ready when the
+          // row threads finish this chunk's alpha (their TMEM buffer's last alpha MMA, of
+          // chunk ac - 1, was issued in the previous iteration, and sbar waits for it)
+          if (deep && ac + 1 < n_active && !(ok = sbar(ac + 1))) break;
           if (!(ok = wait_poll(BAR(C::B_A0F + b), (ac >> 1) & 1, abort_flag))) break;
           tc_fence_after();
-          const uint32_t sb = base_u + C::OFF_CV + b * C::CV_STAGE + C::CV_HALF;
+          const uint32_t sb = base_u + C::cv_off(cs) + C::CV_HALF;
           // alpha of blocks [16k, 16k + 16): packed by half k of the row at the start of
           // its own pooled-score columns
 #pragma unroll
@@ -519,8 +578,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                     sdesc_sw128(sb + k * 2048, C::CHUNK * 128, 1024), idO, (o_acc | uint32_t(k)) ? 1u : 0u);
           o_acc = 1;
           umma_commit(BAR(C::B_SBE + b));
-          umma_commit(BAR(C::B_CVE + b));
-          if (ac + 1 < n_active && !(ok = sbar(ac + 1))) break;
+          umma_commit(BAR(C::B_CVE + cs));
+          if (!deep && ac + 1 < n_active && !(ok = sbar(ac + 1))) break;
           if (p.order == 1) {
             const int a_end = chunk_off[c + 1];
             for (int a = chunk_off[c]; a < a_end; a += C::GROUP, ++g, ++u) {
@@ -562,51 +621,22 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     }
   } else if (warp < 4) {
     // ----------------------------------------------------------- kbar / S0 converter
+    // Warps 2-3 convert every chunk; in deep mode chunks 0, 1 and the even ones, while
+    // warps 8-9 (idle in the approximate stage there) take the odd ones from 3 on.
     const int ct = threadIdx.x - 64;
+    bool ring_idle = false;  // deep: the exact stage is done, ring stage 1 holds stages 2, 3
     for (int ac = 0; ac < n_active; ++ac) {
+      if (deep && ac >= 3 && (ac & 1)) continue;
       const int c = active[ac];
-      const int s = ac & 1;
-      if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_CVE + s), ((ac >> 1) & 1) ^ 1, abort_flag))) break;
-      uint8_t* dk = base + C::OFF_CV + s * C::CV_STAGE;
-      uint8_t* ds = dk + C::CV_HALF;
-      const float* gk = p.kbar + (size_t(bh) * nB + size_t(c) * C::CHUNK) * D;
-      const float* gs = p.S0 + (size_t(bh) * nB + size_t(c) * C::CHUNK) * D;
-      // [CHUNK blocks][D] row-major, 128-byte rows per 64-column panel, 16-byte
-      // chunks swizzled by (row % 8): the K-major (kbar) and MN-major (S0) UMMA
-      // operand layouts coincide for this row = block, column = d storage
-      // all loads of a batch are issued before the first conversion (one L2 round
-      // trip per batch, not per item)
-      constexpr int ITEMS = C::CHUNK * (D / 8) / 64, BATCH = 4;
-      static_assert(ITEMS % BATCH == 0, "converter batches");
-#pragma unroll 1
-      for (int b0 = 0; b0 < ITEMS; b0 += BATCH) {
-        float4 kf[BATCH][2], sf[BATCH][2];
-#pragma unroll
-        for (int i = 0; i < BATCH; ++i) {
-          const int q = ct + (b0 + i) * 64;
-          const int r = q / (D / 8), c16 = q % (D / 8);
-          if (c * C::CHUNK + r < nB) {
-            kf[i][0] = __ldg(reinterpret_cast<const float4*>(gk + r * D + c16 * 8));
-            kf[i][1] = __ldg(reinterpret_cast<const float4*>(gk + r * D + c16 * 8 + 4));
-            sf[i][0] = __ldg(reinterpret_cast<const float4*>(gs + r * D + c16 * 8));
-            sf[i][1] = __ldg(reinterpret_cast<const float4*>(gs + r * D + c16 * 8 + 4));
-          } else {
-            kf[i][0] = kf[i][1] = sf[i][0] = sf[i][1] = make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < BATCH; ++i) {
-          const int q = ct + (b0 + i) * 64;
-          const int r = q / (D / 8), c16 = q % (D / 8);
-          const uint4 kv = make_uint4(pack_bf16x2(kf[i][0].x, kf[i][0].y), pack_bf16x2(kf[i][0].z, kf[i][0].w),
-                                      pack_bf16x2(kf[i][1].x, kf[i][1].y), pack_bf16x2(kf[i][1].z, kf[i][1].w));
-          const uint4 sv = make_uint4(pack_bf16x2(sf[i][0].x, sf[i][0].y), pack_bf16x2(sf[i][0].z, sf[i][0].w),
-                                      pack_bf16x2(sf[i][1].x, sf[i][1].y), pack_bf16x2(sf[i][1].z, sf[i][1].w));
-          const int off = (c16 >> 3) * (C::CHUNK * 128) + r * 128 + (((c16 & 7) ^ (r & 7)) << 4);
-          *reinterpret_cast<uint4*>(dk + off) = kv;
-          *reinterpret_cast<uint4*>(ds + off) = sv;
-        }
+      const int s = ac % ncv;
+      if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_CVE + s), ((ac / ncv) & 1) ^ 1, abort_flag))) break;
+      if (s >= 2 && !ring_idle) {
+        if (!__all_sync(0xffffffffu, wait_bounded(BAR(C::B_XD), 0, abort_flag))) break;
+        ring_idle = true;
       }
+      convert_chunk<D, C::CHUNK, 64, 4>(base + C::cv_off(s), p.kbar + (size_t(bh) * nB + size_t(c) * C::CHUNK) * D,
+                                        p.S0 + (size_t(bh) * nB + size_t(c) * C::CHUNK) * D,
+                                        min(C::CHUNK, nB - c * C::CHUNK), ct);
       fence_proxy_async_smem();
       warp_arrive(BAR(C::B_CVF + s));
     }
@@ -885,6 +915,22 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             }
             fence_proxy_async_smem();
             warp_arrive(BAR(C::B_HF));
+          }
+        }
+        if (ok && deep && warp < 10) {
+          // the odd chunks from 3 on (ring stage 1 is idle: B_XD)
+          ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_XD), 0, abort_flag));
+          for (int ac = 3; ac < n_active && ok; ac += 2) {
+            const int c = active[ac];
+            const int s = ac % ncv;
+            if (!(ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_CVE + s), ((ac / ncv) & 1) ^ 1, abort_flag))))
+              break;
+            convert_chunk<D, C::CHUNK, 64, 4>(base + C::cv_off(s),
+                                              p.kbar + (size_t(bh) * nB + size_t(c) * C::CHUNK) * D,
+                                              p.S0 + (size_t(bh) * nB + size_t(c) * C::CHUNK) * D,
+                                              min(C::CHUNK, nB - c * C::CHUNK), int(threadIdx.x) - 256);
+            fence_proxy_async_smem();
+            warp_arrive(BAR(C::B_CVF + s));
           }
         }
       } else if (ok) {
