@@ -101,7 +101,21 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
-    def stop(self):
+    def wait_first(self, timeout: float = 3.0):
+        """Block until nvidia-smi has printed its first sample (bounded), so that the
+        sampler is running when the timed region starts."""
+        t0 = time.time()
+        while self.proc is not None and not self.lines and time.time() - t0 < timeout:
+            time.sleep(0.01)
+        return self
+
+    def mark(self) -> int:
+        return len(self.lines)
+
+    def stop(self, mark: int = 0):
+        """Median SM clock and throttle reasons of the samples taken after `mark` (the
+        timed region); a region shorter than the sampling interval keeps the latest
+        sample before it."""
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -110,9 +124,16 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.t.join(timeout=2)
+        return self.summarize(self.lines, mark)
+
+    @staticmethod
+    def summarize(all_lines, mark: int = 0):
+        """Median SM clock, max clock and active throttle reasons of the CSV sample lines
+        after `mark`, or of the last line before it when there are none after it."""
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        lines = all_lines[mark:] if len(all_lines) > mark else all_lines[-1:]
+        for ln in lines:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
@@ -127,7 +148,7 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "in_timed_region": len(all_lines) > mark}
 
 
 def _dist():
@@ -413,11 +434,11 @@ def run_ours(args):
     P.device_error()
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    sampler = ClockSampler(_physical_gpu(local)).start() if rank == 0 else None
-    time.sleep(0.3 if sampler else 0)
+    sampler = ClockSampler(_physical_gpu(local)).start().wait_first() if rank == 0 else None
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
+    mark = sampler.mark() if sampler else 0
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for i in range(args.steps):
@@ -426,7 +447,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     if pg:
         pg.barrier()
-    clocks = sampler.stop() if sampler else None
+    clocks = sampler.stop(mark) if sampler else None
     P.device_error()
     ms_region = start.elapsed_time(end)
     ms_total = max_over_ranks(ms_region, pg, dev)
