@@ -21,7 +21,9 @@
 //               shared-memory stages;
 //   warp 1      MMA issuer (one thread): every tcgen05.mma of the tile;
 //   warps 2-3   build the block lists, then convert fp32 kbar / S0 chunks of 32
-//               blocks into bf16 swizzled shared-memory operands;
+//               blocks into bf16 swizzled shared-memory operands (at orders 0 and 2,
+//               where the approximate stage is short per chunk, warps 8-9 convert every
+//               other chunk as well, into a four-stage conversion ring);
 //   warps 4-11  two threads per query row (= TMEM lane): warps w and w + 4 share a
 //               lane quarter. Exact stage at b = 64: two independent groups, warps 4-7
 //               taking the even exact blocks and warps 8-11 the odd ones, each thread
@@ -32,7 +34,9 @@
 //               columns and half of O's columns, and a pair agrees on its running
 //               maximum through shared memory at one named barrier per block. The
 //               approximate stage runs on warps 4-7 alone with full-width operands
-//               (its hand-offs are short; fewer warps to wait for pays more there).
+//               (its hand-offs are short; fewer warps to wait for pays more there);
+//               at orders 0 and 2 the MMA thread issues each chunk's pooled scores
+//               before it waits for the previous chunk's alpha.
 // Tensor memory (512 columns): O accumulator (D), the tile's queries Q (D/2; the A
 // operand of Q K^T and Q Kbar^T), then, in the exact stage, the second group's
 // accumulator O_1 (D, b = 64 only) and a ring of exact score buffers S (P overwrites
