@@ -152,8 +152,7 @@ struct TcCfg {
   static constexpr int B_A0F = B_SBF + 2;         // [2]   alpha operand written (8 warps)
   static constexpr int B_SBE = B_A0F + 2;         // [2]   alpha MMA done (commit)
   static constexpr int B_GA = B_SBE + 2;          // [2]   a pair of A_j written (8 warps)
-  static constexpr int B_AE = B_GA + 2;           // [2]   a pair of A_j consumed (commit)
-  static constexpr int B_OSYNC = B_AE + 2;        //       end of the exact stage / of a chunk (commit)
+  static constexpr int B_OSYNC = B_GA + 2;        //       end of the exact stage / of a chunk (commit)
   static constexpr int B_ODONE = B_OSYNC + 1;     //       all MMAs done (commit)
   static constexpr int B_XD = B_ODONE + 1;        //       exact stage done, ring idle (commit; orders 0, 2)
   static constexpr int B_HF = B_XD + 1;           //       Hbar operand converted (4 warps; hybrid)
@@ -324,7 +323,6 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       mbar_init(BAR(C::B_A0F + s), kApproxWarps);
       mbar_init(BAR(C::B_SBE + s), 1);
       mbar_init(BAR(C::B_GA + s), kApproxWarps);
-      mbar_init(BAR(C::B_AE + s), 1);
     }
     mbar_init(BAR(C::B_Q), kRowWarps);
     mbar_init(BAR(C::B_OSYNC), 1);
@@ -602,7 +600,6 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                   umma_ts(tmem + C::O_COL, aa + k * 8, sdesc_sw128(s1 + k * 2048, D * 128, 1024), idO, 1u);
                 umma_commit(BAR(C::B_SE + s));
               }
-              umma_commit(BAR(C::B_AE + gs));
             }
           }
           umma_commit(BAR(C::B_OSYNC));  // completion ac + 1: end of active chunk ac
@@ -951,6 +948,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         }
         const int nlast = N - (nB - 1) * BLK;
         int g = 0;
+        int tl1 = -1, tl2 = -1;  // stage use of the last block of pairs g - 1, g - 2
         for (int ac = 0; ac < n_active && ok; ++ac) {
           const int c = active[ac];
           const int b = ac & 1;
@@ -1031,8 +1029,14 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           for (int a = chunk_off[c]; a < a_end; a += C::GROUP, ++g) {
             const int n = min(C::GROUP, a_end - a);
             const int gs = g & 1;
-            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_AE + gs), ((g >> 1) & 1) ^ 1, abort_flag));
-            if (!ok) break;
+            // operand slots gs were last read by pair g - 2: free once the ring stage of
+            // that pair's last block is released (its commit follows every MMA of the pair)
+            if (g >= 2) {
+              ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SE + tl2 % C::NS), (tl2 / C::NS) & 1, abort_flag));
+              if (!ok) break;
+            }
+            tl2 = tl1;
+            tl1 = C::TPB * n_exact + a + n - 1;  // stage use of this pair's last block
             tc_fence_after();
 #pragma unroll 1
             for (int qq = 0; qq < n; ++qq) {
