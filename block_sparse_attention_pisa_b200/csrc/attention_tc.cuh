@@ -104,6 +104,10 @@ struct TcCfg {
   // d = 64): twice the blocks in flight for the same shared memory
   static constexpr bool KV_PACKED = 2 * BLK * D * 2 <= STAGE;
   static constexpr int TPB = KV_PACKED ? 1 : 2;             // ring stages per exact block
+  // exact block e's V tile is ring-stage use TPB e + TPB - 1; that stage's release (an MMA
+  // commit after the block's P V) is also the signal that P V(e) is done
+  __host__ __device__ static constexpr int v_stage(int e) { return (TPB * e + TPB - 1) % NS; }
+  __host__ __device__ static constexpr uint32_t v_parity(int e) { return uint32_t((TPB * e + TPB - 1) / NS) & 1u; }
   static constexpr int CHUNK = 32;                          // key blocks per approximate chunk
   static constexpr int CV_HALF = CHUNK * D * 2;             // bf16 kbar (or S0) chunk
   static constexpr int CV_STAGE = 2 * CV_HALF;
@@ -145,8 +149,7 @@ struct TcCfg {
   static constexpr int B_Q = B_TF + NTF;          //       queries in TMEM (8 row warps)
   static constexpr int B_SF = B_Q + 1;            // [NSB] S ready (commit)
   static constexpr int B_PF = B_SF + NSB;         // [NSB] P written (8 row warps)
-  static constexpr int B_PV = B_PF + NSB;         // [NSB] P V done (commit)
-  static constexpr int B_CVF = B_PV + NSB;        // [4]   kbar / S0 chunk converted (2 warps)
+  static constexpr int B_CVF = B_PF + NSB;        // [4]   kbar / S0 chunk converted (2 warps)
   static constexpr int B_CVE = B_CVF + NCV_MAX;   // [4]   chunk operands consumed (commit)
   static constexpr int B_SBF = B_CVE + NCV_MAX;   // [2]   Sbar ready (commit)
   static constexpr int B_A0F = B_SBF + 2;         // [2]   alpha operand written (8 warps)
@@ -312,7 +315,6 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     for (int s = 0; s < C::NSB; ++s) {
       mbar_init(BAR(C::B_SF + s), 1);
       mbar_init(BAR(C::B_PF + s), C::GROUPS ? kRowWarps / 2 : kRowWarps);  // a group, or both halves
-      mbar_init(BAR(C::B_PV + s), 1);
     }
     for (int s = 0; s < C::NCV_MAX; ++s) {
       mbar_init(BAR(C::B_CVF + s), 2);
@@ -482,6 +484,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       uint32_t g_acc = 0u;
       bool ok = wait_poll(BAR(C::B_Q), 0, abort_flag);
       tc_fence_after();
+      // P V(e) done: the release of block e's V ring stage (committed right after it)
+      auto wait_pv = [&](int e) -> bool {
+        return wait_poll(BAR(C::B_SE + C::v_stage(e)), C::v_parity(e), abort_flag);
+      };
       auto pv = [&](int e) -> bool {
         const int sb = e % C::NSB;
         if (!wait_poll(BAR(C::B_PF + sb), (e / C::NSB) & 1, abort_flag)) return false;
@@ -508,13 +514,12 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         }
         o_acc = 1;
         umma_commit(BAR(C::B_SE + sv));
-        umma_commit(BAR(C::B_PV + sb));
         return true;
       };
       // S = Q K_j^T for block e (its buffer was last used by block e - NSB)
       auto qk = [&](int e) -> bool {
         const int sb = e % C::NSB;
-        if (e >= C::NSB && !wait_poll(BAR(C::B_PV + sb), ((e - C::NSB) / C::NSB) & 1, abort_flag)) return false;
+        if (e >= C::NSB && !wait_pv(e - C::NSB)) return false;
         if (!wait_poll(BAR(C::B_TF + e % C::NTF), (e / C::NTF) & 1, abort_flag)) return false;
         tc_fence_after();
         const int sk = (C::TPB * e) % C::NS;
@@ -544,7 +549,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         if constexpr (C::GROUPS)
           ok = wait_poll(BAR(C::B_MG), 0, abort_flag);
         else
-          ok = wait_poll(BAR(C::B_PV + (n_exact - 1) % C::NSB), ((n_exact - 1) / C::NSB) & 1, abort_flag);
+          ok = wait_pv(n_exact - 1);
         auto sbar = [&](int ac) -> bool {
           const int b = ac & 1, cs = ac % ncv;
           if (!wait_poll(BAR(C::B_CVF + cs), (ac / ncv) & 1, abort_flag)) return false;
@@ -731,8 +736,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           if (__any_sync(0xffffffffu, need_o)) {
             // the group's previous product must be in O_hf before it is rescaled
             if (e >= 2)
-              ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_PV + (e - 2) % C::NSB), ((e - 2) / C::NSB) & 1,
-                                                        abort_flag));
+              ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SE + C::v_stage(e - 2)), C::v_parity(e - 2), abort_flag));
             if (ok) {
               tc_fence_after();
               const float f = need_o ? ex2(m - mx) : 1.f;
@@ -838,8 +842,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         const bool need_o = grow_max && m != -INFINITY;
         if (__any_sync(0xffffffffu, need_o)) {
           if (e >= 1)
-            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_PV + (e - 1) % C::NSB), ((e - 1) / C::NSB) & 1,
-                                                      abort_flag));
+            ok = __all_sync(0xffffffffu, wait_bounded(BAR(C::B_SE + C::v_stage(e - 1)), C::v_parity(e - 1), abort_flag));
           if (ok) {
             tc_fence_after();
             const float f = need_o ? ex2(m - mx) : 1.f;
