@@ -130,6 +130,9 @@ struct TcCfg {
   static constexpr int O1_COL = D + D / 2;              // second exact accumulator (GROUPS)
   static constexpr int SX_COL = GROUPS ? O1_COL + D : D + D / 2;  // exact score buffers
   static constexpr int NSB = GROUPS ? (512 - SX_COL) / BLK : ((D == 128) ? (512 - (D + D / 2)) / BLK : 2);
+  // the scores run kLook blocks ahead of the row threads' softmax (two groups: one block
+  // further, since the two groups' blocks alternate)
+  static constexpr int kLook = GROUPS ? NSB - 1 : (NSB >= 3 ? NSB - 2 : 1);
   static constexpr int MAXB = 2048;
   static constexpr int MAXC = MAXB / CHUNK;
   // tensor-memory columns
@@ -517,10 +520,14 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         return true;
       };
       // S = Q K_j^T for block e (its buffer was last used by block e - NSB)
-      auto qk = [&](int e) -> bool {
+      // `waits`: K(e) landed and P V(e - NSB) done are awaited here; after the prologue the
+      // row group that signals P(e - kLook) has awaited both before its signal
+      auto qk = [&](int e, bool waits) -> bool {
         const int sb = e % C::NSB;
-        if (e >= C::NSB && !wait_pv(e - C::NSB)) return false;
-        if (!wait_poll(BAR(C::B_TF + e % C::NTF), (e / C::NTF) & 1, abort_flag)) return false;
+        if (waits) {
+          if (e >= C::NSB && !wait_pv(e - C::NSB)) return false;
+          if (!wait_poll(BAR(C::B_TF + e % C::NTF), (e / C::NTF) & 1, abort_flag)) return false;
+        }
         tc_fence_after();
         const int sk = (C::TPB * e) % C::NS;
         const uint32_t kb = base_u + C::OFF_RING + sk * C::STAGE;
@@ -532,13 +539,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         umma_commit(BAR(C::B_SF + sb));
         return true;
       };
-      // the scores run kLook blocks ahead of the row threads' softmax
-      // (two groups: one block further, since the two groups' blocks alternate)
-      constexpr int kLook = C::GROUPS ? C::NSB - 1 : (C::NSB >= 3 ? C::NSB - 2 : 1);
-      for (int e = 0; e < kLook && e < n_exact && ok; ++e) ok = qk(e);
+      for (int e = 0; e < C::kLook && e < n_exact && ok; ++e) ok = qk(e, true);
       for (int e = 0; e < n_exact && ok; ++e) {
         ok = pv(e);
-        if (ok && e + kLook < n_exact) ok = qk(e + kLook);
+        if (ok && e + C::kLook < n_exact) ok = qk(e + C::kLook, false);
       }
       umma_commit(BAR(C::B_OSYNC));  // completion 0: end of the exact stage
       if (deep) umma_commit(BAR(C::B_XD));
@@ -765,6 +769,18 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         l += (rsp[0] + rsp[1]) + (rsp[2] + rsp[3]);
         tmem_wait_st();
         tc_fence_before();
+        // what the MMA thread's Q K^T of block e + kLook (issued right after P V(e)) needs:
+        // that block's K landed and P V(e + kLook - NSB) done, awaited here so that it
+        // issues without a wait (a wait that runs out has raised the abort flag)
+        {
+          const int en = e + C::kLook;
+          if (en < n_exact) {
+            bool w = wait_bounded(BAR(C::B_TF + en % C::NTF), (en / C::NTF) & 1, abort_flag);
+            if (w && en >= C::NSB)
+              w = wait_bounded(BAR(C::B_SE + C::v_stage(en - C::NSB)), C::v_parity(en - C::NSB), abort_flag);
+            __syncwarp();
+          }
+        }
         warp_arrive(BAR(C::B_PF + sb));
       }
       // merge: O_0 <- f_0 O_0 + f_1 O_1 against the common maximum, each group over its own
@@ -873,6 +889,18 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         l += (rsp[0] + rsp[1]) + (rsp[2] + rsp[3]);
         tmem_wait_st();
         tc_fence_before();
+        // what the MMA thread's Q K^T of block e + kLook (issued right after P V(e)) needs:
+        // that block's K landed and P V(e + kLook - NSB) done, awaited here so that it
+        // issues without a wait (a wait that runs out has raised the abort flag)
+        {
+          const int en = e + C::kLook;
+          if (en < n_exact) {
+            bool w = wait_bounded(BAR(C::B_TF + en % C::NTF), (en / C::NTF) & 1, abort_flag);
+            if (w && en >= C::NSB)
+              w = wait_bounded(BAR(C::B_SE + C::v_stage(en - C::NSB)), C::v_parity(en - C::NSB), abort_flag);
+            __syncwarp();
+          }
+        }
         warp_arrive(BAR(C::B_PF + sb));
       }
       ok = pair_sync_and(pair_id, ok);
